@@ -1,0 +1,431 @@
+#!/usr/bin/env python
+"""Benchmark: cached-step attention TFLOP/s and ms per 40-step attention.
+
+One bench step = the whole attention hot path of one generation at the chosen
+workload: for each of the 40 denoising steps and each of the 32 layers, step 1
+runs bca_prefill (block-causal attention over the whole sequence, storing the
+prefix K/V into that layer's cache slot) and steps 2..40 run bca_step_attend
+(target rows over [cached prefix ; own K/V]).  A new request epoch is used for
+every bench step, so the cache is rebuilt each time (per-request rebuild).
+
+value  = attention FLOPs of the step (4*d*H per allowed query-key pair, prefill
+         plus cached steps) / device time, TFLOP/s, summed over ranks.
+e2e    = the same through the Python/C-ABI calls with pinned HOST buffers: every
+         call's Q/K/V is copied host->device and its output device->host inside
+         the timed region.
+roofline: the dominant kernel (cached-step attention) against the measured
+         dense bf16 tensor peak; cpu_baseline: the fp64 oracle on the host cores.
+
+Inputs: seeded synthetic bf16 N(0,1) (see block_causal_attention_dit_b200.workloads);
+per-layer prefill inputs; cached-step inputs cycle through a pool of distinct
+seeded target sets larger than L2 (126 MB).
+
+Multi-GPU (torchrun): replicas -- each rank runs its own independent requests,
+no collective on the data path; the step time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "cached-step attention TFLOP/s & % of BF16 tensor peak; ms per 40-step attn"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ---------------------------------------------------------------------------
+# Algorithmic work
+# ---------------------------------------------------------------------------
+def prefill_flops(req, H, d=128) -> float:
+    tot, cum = 0, 0
+    for b in req.blocks:
+        cum += b
+        tot += b * cum
+    return 4.0 * d * H * tot
+
+
+def step_flops(req, H, d=128) -> float:
+    return 4.0 * d * H * req.target * (req.prefix + req.target)
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            pk = json.load(f)
+        return pk, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ---------------------------------------------------------------------------
+# Clock sampling during the timed region
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.proc = None
+        self.device = device_index
+
+    def start(self):
+        try:
+            import torch
+            uuid = str(torch.cuda.get_device_properties(self.device).uuid)
+            sel = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", sel, f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:  # noqa: BLE001 - clocks are best effort
+            self.proc = None
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
+        time.sleep(0.3)
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        rows = [r.split(",") for r in out.strip().splitlines() if r.count(",") >= 8]
+        sm, mx, reasons, power = [], None, set(), []
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            r = [x.strip() for x in r]
+            try:
+                sm.append(float(r[1]))
+                mx = float(r[2])
+                power.append(float(r[3]))
+            except ValueError:
+                continue
+            for n, val in zip(names, r[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(n)
+        loaded = [s for s, p in zip(sm, power) if p > 300.0] or sm
+        return {"sm_mhz": statistics.median(loaded) if loaded else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm),
+                "power_w_max": max(power) if power else None}
+
+
+# ---------------------------------------------------------------------------
+# Our arm
+# ---------------------------------------------------------------------------
+class Runner:
+    """Holds the resident inputs, cache slots and outputs of one workload."""
+
+    def __init__(self, wl, layers: int, device, rank: int, pool: int):
+        import torch
+
+        import block_causal_attention_dit_b200 as bca
+        from block_causal_attention_dit_b200 import workloads as W
+        self.bca, self.W, self.wl, self.layers, self.device = bca, W, wl, layers, device
+        self.rank = rank
+        H = wl.heads
+        self.H = H
+        reqs = wl.requests
+        self.cu = [0]
+        for r in reqs:
+            self.cu.append(self.cu[-1] + r.target)
+        seed_base = 1000 * rank
+        # per-layer prefill inputs (one per request) and per-layer cache slots
+        self.pre = [[W.qkv(wl, l, 0, i, device) for i in range(len(reqs))] for l in range(layers)]
+        if rank:
+            for l in range(layers):
+                for i in range(len(reqs)):
+                    self.pre[l][i] = tuple(W.randn_bf16(tuple(t.shape),
+                                                        seed_base + W.seed_for(wl.index, l, 0, i, j),
+                                                        device)
+                                           for j, t in enumerate(self.pre[l][i]))
+        self.slots = [[bca.KVSlot(max(r.prefix, 1), H, wl.kv_dtype, device=device) for r in reqs]
+                      for _ in range(layers)]
+        self.o_pre = [torch.empty_like(self.pre[0][i][0]) for i in range(len(reqs))]
+        # cached-step input pool: packed target rows of all requests
+        self.pool = []
+        for p in range(pool):
+            per = [W.qkv(wl, p % layers, 1 + p // layers, i, device) if rank == 0 else
+                   tuple(W.randn_bf16((r.target, H, 128),
+                                      seed_base + W.seed_for(wl.index, p % layers, 1 + p // layers,
+                                                             i, j), device) for j in range(3))
+                   for i, r in enumerate(reqs)]
+            self.pool.append(tuple(torch.cat([x[j] for x in per]) for j in range(3)))
+        self.o_step = torch.empty_like(self.pool[0][0])
+        self.status = torch.zeros(1, dtype=torch.int32, device=device)
+        self.epoch = 0
+        self.flops_prefill = sum(prefill_flops(r, H) for r in reqs) * layers
+        self.flops_step_call = sum(step_flops(r, H) for r in reqs)
+        self.flops_steps = self.flops_step_call * layers * (wl.steps - 1)
+        self.flops = self.flops_prefill + self.flops_steps
+        kv_store_launches = 1 if wl.kv_dtype == "bf16" else 4
+        self.launches_per_step = (layers * len(reqs) * (1 + kv_store_launches)
+                                  + layers * (wl.steps - 1))
+
+    def step(self, events=None):
+        """One pass of the hot path.  events: optional list collecting
+        (start, end) CUDA event pairs around every cached-step call."""
+        import torch
+        bca, wl = self.bca, self.wl
+        self.epoch += 1
+        for s in range(wl.steps):
+            for l in range(self.layers):
+                if s == 0:
+                    for i, r in enumerate(wl.requests):
+                        q, k, v = self.pre[l][i]
+                        bca.prefill(q, k, v, self.o_pre[i], r.offsets, wl.scale,
+                                    slot=self.slots[l][i], epoch=self.epoch,
+                                    dev_status=self.status)
+                else:
+                    q, k, v = self.pool[(l * (wl.steps - 1) + s - 1) % len(self.pool)]
+                    if events is not None:
+                        e0 = torch.cuda.Event(enable_timing=True)
+                        e1 = torch.cuda.Event(enable_timing=True)
+                        e0.record()
+                    bca.step_attend(q, k, v, self.o_step, self.cu, self.slots[l], wl.scale,
+                                    dev_status=self.status)
+                    if events is not None:
+                        e1.record()
+                        events.append((e0, e1))
+
+
+class E2ERunner:
+    """The same step through the public calls with pinned host buffers: each call's
+    inputs are copied host->device and its output read back inside the timing."""
+
+    def __init__(self, runner, host_sets: int = 2):
+        import torch
+        self.r = runner
+        wl = runner.wl
+        pin = lambda t: t.cpu().pin_memory()
+        self.h_pre = [[tuple(pin(x) for x in runner.pre[l % runner.layers][i])
+                       for i in range(len(wl.requests))] for l in range(host_sets)]
+        self.h_pool = [tuple(pin(x) for x in runner.pool[p]) for p in range(host_sets)]
+        self.d_pre = [tuple(torch.empty_like(x) for x in runner.pre[0][i])
+                      for i in range(len(wl.requests))]
+        self.d_step = tuple(torch.empty_like(x) for x in runner.pool[0])
+        self.h_out_pre = [torch.empty(x[0].shape, dtype=x[0].dtype).pin_memory()
+                          for x in self.d_pre]
+        self.h_out_step = torch.empty(self.d_step[0].shape, dtype=self.d_step[0].dtype).pin_memory()
+        layers, steps = runner.layers, wl.steps
+        self.h2d = (layers * sum(3 * x[0].numel() * 2 for x in self.d_pre)
+                    + layers * (steps - 1) * 3 * self.d_step[0].numel() * 2)
+        self.d2h = (layers * sum(x[0].numel() * 2 for x in self.d_pre)
+                    + layers * (steps - 1) * self.d_step[0].numel() * 2)
+
+    def step(self):
+        bca, r, wl = self.r.bca, self.r, self.r.wl
+        r.epoch += 1
+        for s in range(wl.steps):
+            for l in range(r.layers):
+                if s == 0:
+                    for i, req in enumerate(wl.requests):
+                        hq, hk, hv = self.h_pre[l % len(self.h_pre)][i]
+                        q, k, v = self.d_pre[i]
+                        q.copy_(hq, non_blocking=True)
+                        k.copy_(hk, non_blocking=True)
+                        v.copy_(hv, non_blocking=True)
+                        bca.prefill(q, k, v, r.o_pre[i], req.offsets, wl.scale,
+                                    slot=r.slots[l][i], epoch=r.epoch, dev_status=r.status)
+                        self.h_out_pre[i].copy_(r.o_pre[i], non_blocking=True)
+                else:
+                    hq, hk, hv = self.h_pool[(l + s) % len(self.h_pool)]
+                    q, k, v = self.d_step
+                    q.copy_(hq, non_blocking=True)
+                    k.copy_(hk, non_blocking=True)
+                    v.copy_(hv, non_blocking=True)
+                    bca.step_attend(q, k, v, r.o_step, r.cu, r.slots[l], wl.scale,
+                                    dev_status=r.status)
+                    self.h_out_step.copy_(r.o_step, non_blocking=True)
+
+
+def timed(fn, steps: int, warmup: int, dist_on: bool):
+    import torch
+    import torch.distributed as dist
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    if dist_on:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        fn()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1)
+    if dist_on:
+        t = torch.tensor([ms], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+        dist.barrier()
+    return ms
+
+
+# ---------------------------------------------------------------------------
+# Oracle timing (CPU baseline and the reference arm)
+# ---------------------------------------------------------------------------
+def oracle_sample(wl, target_seconds: float, layer: int = 0):
+    """Time the fp64 oracle on a bounded sample of one cached step of request 0:
+    all heads x the first n target rows, n sized to ~target_seconds."""
+    import oracle
+    from block_causal_attention_dit_b200 import workloads as W
+    req = wl.requests[0]
+    H, P, T = wl.heads, req.prefix, req.target
+    q0, k0, v0 = W.qkv(wl, layer, 0, 0, "cpu")
+    q, k, v = W.qkv(wl, layer, 1, 0, "cpu")
+    kc = k0[:P].permute(1, 0, 2).contiguous()
+    vc = v0[:P].permute(1, 0, 2).contiguous()
+    n = 4
+    while True:
+        rows = list(range(n))
+        t0 = time.perf_counter()
+        oracle.cached_step(q, k, v, kc, vc, P, wl.scale, rows=rows)
+        dt = time.perf_counter() - t0
+        if dt >= 0.5 * target_seconds or n >= T:
+            break
+        n = min(T, max(n * 2, int(n * target_seconds / max(dt, 1e-3))))
+    flops = 4.0 * 128 * H * n * (P + T)
+    return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": oracle.max_threads(),
+            "kind": "oracle", "seconds": dt,
+            "sample": f"one cached step of layer {layer}: {H} heads x {n} of {T} target rows, "
+                      f"{P + T} keys each, fp64"}
+
+
+# ---------------------------------------------------------------------------
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=3)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", type=int, default=1)
+    ap.add_argument("--layers", type=int, default=None)
+    ap.add_argument("--pool", type=int, default=8)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    args = ap.parse_args()
+
+    from block_causal_attention_dit_b200 import workloads as W
+    wl = W.workload(args.workload)
+    layers = args.layers or wl.layers
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    n_gpus = max(world, 1)
+    config = {"workload": wl.name, "heads": wl.heads, "head_dim": wl.head_dim,
+              "blocks": [r.blocks for r in wl.requests], "layers": layers, "steps": wl.steps,
+              "kv_cache": wl.kv_dtype, "parallelism": f"replicas x{n_gpus}",
+              "l2": f"inputs larger than L2: per-layer prefill inputs and a pool of "
+                    f"{args.pool} cached-step input sets cycled over (layer, step)"}
+
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        samples = []
+        for i in range(args.warmup + args.steps):
+            s = oracle_sample(wl, min(args.cpu_seconds, 8.0))
+            if i >= args.warmup:
+                samples.append(s)
+        val = statistics.median(s["value"] for s in samples)
+        cpu = dict(samples[-1], value=val)
+        print(json.dumps({"impl": "reference", "metric": METRIC, "value": val,
+                          "unit": "TFLOP/s", "n_gpus": n_gpus, "steps": args.steps,
+                          "warmup": args.warmup, "higher_is_better": True, "scaling": "weak",
+                          "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+                          "config": config, "cpu_baseline": cpu,
+                          "e2e": {"value": val, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                                  "d2h_bytes_per_step": 0}}), flush=True)
+        return 0
+
+    import torch
+    import torch.distributed as dist
+    dist_on = world > 1
+    if dist_on:
+        torch.cuda.set_device(local_rank)
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    device = torch.device("cuda", torch.cuda.current_device())
+    import block_causal_attention_dit_b200 as bca
+    bca.lib()
+
+    runner = Runner(wl, layers, device, rank, args.pool)
+    torch.cuda.synchronize()
+
+    # main measurement (device-resident inputs)
+    for _ in range(args.warmup):
+        runner.step()
+    torch.cuda.synchronize()
+    sampler = ClockSampler(device.index)
+    sampler.start()
+    events = []
+    ms = timed(lambda: runner.step(events), args.steps, 0, dist_on)
+    clocks = sampler.stop()
+    status = int(runner.status.item())
+    if status != 0:
+        raise RuntimeError(f"device status {status}")
+    step_ms = [a.elapsed_time(b) for a, b in events]
+    avg_step_ms = sum(step_ms) / len(step_ms)
+    ms_per_step = ms / args.steps
+    flops_total = runner.flops * n_gpus
+    value = flops_total * args.steps / (ms / 1e3) / 1e12
+
+    peaks, peak_src = load_peaks()
+    achieved = runner.flops_step_call / (avg_step_ms / 1e3) / 1e12
+    peak_sus = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
+    peak_burst = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    roofline = {"bound": "tensor", "kernel": "attn_fwd_kernel (cached step)",
+                "achieved": achieved, "peak": peak_sus, "unit": "TFLOP/s",
+                "frac": achieved / peak_sus, "peak_kind": f"bf16 sustained ({peak_src})",
+                "frac_of_burst_peak": achieved / peak_burst, "peak_burst": peak_burst,
+                "flops_per_launch": runner.flops_step_call, "avg_launch_ms": avg_step_ms,
+                "traffic": None}
+
+    e2e = None
+    if not args.no_e2e:
+        e = E2ERunner(runner)
+        e_ms = timed(e.step, max(1, min(args.steps, 2)), 1, dist_on)
+        e_steps = max(1, min(args.steps, 2))
+        e2e = {"value": flops_total * e_steps / (e_ms / 1e3) / 1e12, "unit": "TFLOP/s",
+               "h2d_bytes_per_step": e.h2d, "d2h_bytes_per_step": e.d2h,
+               "ms_per_step": e_ms / e_steps, "steps": e_steps}
+
+    cpu = None
+    if rank == 0 and n_gpus == 1 and not args.no_cpu_baseline:
+        cpu = oracle_sample(wl, args.cpu_seconds)
+
+    line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": n_gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded bf16 N(0,1), shapes of the workload)", "config": config,
+            "ms_per_40step_attn": ms_per_step,
+            "cached_step_tflops": achieved,
+            "pct_of_bf16_peak": {"sustained": 100 * achieved / peak_sus,
+                                 "burst": 100 * achieved / peak_burst, "source": peak_src},
+            "prefill_and_store_ms_per_step": ms_per_step - sum(step_ms) / args.steps,
+            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+            "gpu_launches": runner.launches_per_step * args.steps, "clocks": clocks}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if dist_on:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

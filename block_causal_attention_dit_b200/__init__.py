@@ -1,0 +1,233 @@
+"""block_causal_attention_dit_b200 -- Python binding of libbca.so.
+
+Block-causal attention with cross-step prefix K/V reuse on B200 (sm_100a).  The
+three calls of the method mirror include/bca.h one to one:
+
+  prefill(q, k, v, o, block_offsets, scale, slot=None, epoch=0)
+      step-1 block-causal attention over [S, H, 128]; optionally stores the prefix
+      (every block but the last) into a KVSlot.
+  kv_store(k, v, n_prefix, slot, epoch)
+      prefix K/V into a KVSlot, bf16 or OFP8 E4M3 with per-head scales.
+  step_attend(q_t, k_t, v_t, o_t, cu_target, slots, scale)
+      cached-step attention of packed target rows over [cache ; own K/V] for a
+      ragged batch of requests at the same phase.
+
+This module only marshals arguments (device pointers, sizes, the current CUDA
+stream) into the C ABI: every step of the path runs in the library's kernels.
+PyTorch is used for device memory and streams.  If the library is missing the
+calls raise; there is no other implementation behind them.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+__all__ = [
+    "BcaError", "KVSlot", "KV_BF16", "KV_FP8_V", "KV_FP8_KV", "MAX_BLOCKS", "MAX_BATCH",
+    "lib", "prefill", "kv_store", "step_attend", "slot_bytes", "set_wait_timeout_ns",
+    "selftest_wait_timeout", "status_string", "version", "LIB_PATH",
+]
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libbca.so")
+
+KV_BF16, KV_FP8_V, KV_FP8_KV = 0, 1, 2
+_DTYPE_NAMES = {"bf16": KV_BF16, "fp8_v": KV_FP8_V, "fp8": KV_FP8_KV}
+MAX_BLOCKS = 64
+MAX_BATCH = 64
+
+STATUS_NAMES = {
+    0: "BCA_OK", 1: "BCA_ERR_INVALID_ARG", 2: "BCA_ERR_UNSUPPORTED", 3: "BCA_ERR_CAPACITY",
+    4: "BCA_ERR_STATE", 5: "BCA_ERR_CUDA", 6: "BCA_ERR_DEVICE_TIMEOUT",
+}
+
+
+class BcaError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = int(status)
+        super().__init__(f"{where}: {STATUS_NAMES.get(self.status, self.status)}")
+
+
+class SlotStruct(ctypes.Structure):
+    """Mirror of bca_kv_slot."""
+    _fields_ = [
+        ("k", ctypes.c_void_p), ("v", ctypes.c_void_p),
+        ("k_scale", ctypes.c_void_p), ("v_scale", ctypes.c_void_p),
+        ("cap_tokens", ctypes.c_int32), ("n_tokens", ctypes.c_int32),
+        ("num_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32),
+        ("dtype", ctypes.c_int32), ("epoch", ctypes.c_uint32),
+    ]
+
+
+_lib = None
+
+
+def lib():
+    """Load libbca.so (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(
+            f"{LIB_PATH} is missing: build it with "
+            "`python -m block_causal_attention_dit_b200.build`")
+    L = ctypes.CDLL(LIB_PATH)
+    P, i32, u32, u64, f32 = (ctypes.c_void_p, ctypes.c_int32, ctypes.c_uint32,
+                             ctypes.c_uint64, ctypes.c_float)
+    SP = ctypes.POINTER(SlotStruct)
+    L.bca_kv_slot_bytes.restype = ctypes.c_size_t
+    L.bca_kv_slot_bytes.argtypes = [i32, i32, i32, ctypes.c_int]
+    L.bca_kv_slot_init.restype = ctypes.c_int
+    L.bca_kv_slot_init.argtypes = [SP, P, i32, i32, i32, ctypes.c_int]
+    L.bca_kv_store.restype = ctypes.c_int
+    L.bca_kv_store.argtypes = [P, P, i32, i32, SP, u32, P, P]
+    L.bca_prefill.restype = ctypes.c_int
+    L.bca_prefill.argtypes = [P, P, P, P, i32, P, i32, i32, i32, f32, SP, u32, P, P]
+    L.bca_step_attend.restype = ctypes.c_int
+    L.bca_step_attend.argtypes = [P, P, P, P, P, SP, i32, i32, i32, f32, P, P]
+    L.bca_status_string.restype = ctypes.c_char_p
+    L.bca_status_string.argtypes = [ctypes.c_int]
+    L.bca_set_wait_timeout_ns.restype = None
+    L.bca_set_wait_timeout_ns.argtypes = [u64]
+    L.bca_selftest_wait_timeout.restype = ctypes.c_int
+    L.bca_selftest_wait_timeout.argtypes = [P, u64, P]
+    L.bca_version.restype = ctypes.c_char_p
+    L.bca_version.argtypes = []
+    _lib = L
+    return L
+
+
+def _check(status: int, where: str):
+    if status != 0:
+        raise BcaError(status, where)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream, device=None):
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _i32_array(values):
+    vals = [int(x) for x in values]
+    return (ctypes.c_int32 * len(vals))(*vals)
+
+
+def status_string(status: int) -> str:
+    return lib().bca_status_string(int(status)).decode()
+
+
+def version() -> str:
+    return lib().bca_version().decode()
+
+
+def slot_bytes(cap_tokens: int, heads: int, head_dim: int = 128, dtype="bf16") -> int:
+    dt = _DTYPE_NAMES.get(dtype, dtype)
+    return int(lib().bca_kv_slot_bytes(cap_tokens, heads, head_dim, dt))
+
+
+def set_wait_timeout_ns(ns: int):
+    lib().bca_set_wait_timeout_ns(int(ns))
+
+
+class KVSlot:
+    """One (request, layer) prefix K/V cache slot carved from one device buffer.
+
+    `buffer` is a torch uint8 CUDA tensor of slot_bytes(...) bytes (allocated here
+    when not given); `struct` is the bca_kv_slot the library reads and updates."""
+
+    def __init__(self, cap_tokens: int, heads: int, dtype="bf16", head_dim: int = 128,
+                 device="cuda", buffer=None):
+        import torch
+        self.dtype = _DTYPE_NAMES.get(dtype, dtype)
+        n = slot_bytes(cap_tokens, heads, head_dim, self.dtype)
+        if n == 0:
+            raise BcaError(1, "KVSlot")
+        if buffer is None:
+            buffer = torch.empty(n, dtype=torch.uint8, device=device)
+        assert buffer.numel() >= n and buffer.dtype == torch.uint8
+        self.buffer = buffer
+        self.struct = SlotStruct()
+        _check(lib().bca_kv_slot_init(ctypes.byref(self.struct), _ptr(buffer), cap_tokens,
+                                      heads, head_dim, self.dtype), "bca_kv_slot_init")
+
+    # Views of the slot's device memory (for tests and inspection).
+    def _view(self, addr, nbytes, torch_dtype, shape):
+        import torch
+        off = addr - self.buffer.data_ptr()
+        return self.buffer[off:off + nbytes].view(torch_dtype).view(*shape)
+
+    def k_view(self):
+        import torch
+        s = self.struct
+        fp8 = self.dtype == KV_FP8_KV
+        es = 1 if fp8 else 2
+        return self._view(s.k, s.num_heads * s.cap_tokens * s.head_dim * es,
+                          torch.uint8 if fp8 else torch.bfloat16,
+                          (s.num_heads, s.cap_tokens, s.head_dim))
+
+    def v_view(self):
+        import torch
+        s = self.struct
+        fp8 = self.dtype in (KV_FP8_V, KV_FP8_KV)
+        es = 1 if fp8 else 2
+        return self._view(s.v, s.num_heads * s.cap_tokens * s.head_dim * es,
+                          torch.uint8 if fp8 else torch.bfloat16,
+                          (s.num_heads, s.cap_tokens, s.head_dim))
+
+    def k_scale_view(self):
+        import torch
+        return self._view(self.struct.k_scale, 4 * self.struct.num_heads, torch.float32,
+                          (self.struct.num_heads,))
+
+    def v_scale_view(self):
+        import torch
+        return self._view(self.struct.v_scale, 4 * self.struct.num_heads, torch.float32,
+                          (self.struct.num_heads,))
+
+    @property
+    def n_tokens(self) -> int:
+        return int(self.struct.n_tokens)
+
+    @property
+    def epoch(self) -> int:
+        return int(self.struct.epoch)
+
+
+def kv_store(k, v, n_prefix: int, slot: KVSlot, epoch: int, row_stride: int | None = None,
+             dev_status=None, stream=None):
+    if row_stride is None:
+        row_stride = k.shape[1] * k.shape[2] if k.dim() == 3 else k.stride(0)
+    _check(lib().bca_kv_store(_ptr(k), _ptr(v), int(n_prefix), int(row_stride),
+                              ctypes.byref(slot.struct), int(epoch), _ptr(dev_status),
+                              _stream(stream, k.device)), "bca_kv_store")
+
+
+def prefill(q, k, v, o, block_offsets, scale: float, slot: KVSlot | None = None,
+            epoch: int = 0, dev_status=None, stream=None):
+    S, H, d = q.shape
+    off = _i32_array(block_offsets)
+    _check(lib().bca_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(o), S, off, len(off) - 1, H, d,
+                             float(scale), None if slot is None else ctypes.byref(slot.struct),
+                             int(epoch), _ptr(dev_status), _stream(stream, q.device)),
+           "bca_prefill")
+
+
+def step_attend(q_t, k_t, v_t, o_t, cu_target, slots, scale: float, dev_status=None,
+                stream=None):
+    _, H, d = q_t.shape
+    cu = _i32_array(cu_target)
+    arr = (SlotStruct * len(slots))(*[s.struct for s in slots])
+    _check(lib().bca_step_attend(_ptr(q_t), _ptr(k_t), _ptr(v_t), _ptr(o_t), cu, arr,
+                                 len(slots), H, d, float(scale), _ptr(dev_status),
+                                 _stream(stream, q_t.device)), "bca_step_attend")
+
+
+def selftest_wait_timeout(dev_status, timeout_ns: int, stream=None):
+    _check(lib().bca_selftest_wait_timeout(_ptr(dev_status), int(timeout_ns),
+                                           _stream(stream, dev_status.device)),
+           "bca_selftest_wait_timeout")

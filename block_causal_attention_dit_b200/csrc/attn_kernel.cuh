@@ -1,0 +1,473 @@
+// attn_kernel.cuh -- block-causal / cached-step attention forward for sm_100a.
+//
+// What it computes (cited by page title and section):
+//  * "Qwen-Image-2.1 + vLLM-Omni day-0", "What is Qwen-Image-2.1" and "Serving
+//    architecture: the cross-step prefix KV cache": ordered blocks (text, refs,
+//    target); row i of block b attends to every key of blocks 0..b.  Prefill
+//    mode computes this over the whole sequence (denoising step 1).
+//  * same section + "Qwen/Qwen-Image-2.1" (vLLM recipe), "Prefix KV cache": in
+//    later steps only the target rows are recomputed; they attend to the cached
+//    prefix K/V followed by their own K/V.  Step mode computes this for a ragged
+//    batch of requests at the same phase ("Online serving": step-level batching).
+//
+// Design (B200): one CTA owns a (request, head, pair of 128-row Q tiles) unit.
+//  * warp 8      : TMA producer -- Q tiles once, then K_j, V_j tiles into a
+//                  4-stage ring of 32 KiB bf16 tiles (128-byte swizzle).
+//  * warp 9      : tcgen05 issuer -- S_w = Q_w K_j^T (both operands in smem) and
+//                  O_w += P_w V_j (P from TMEM, V in smem, MN-major), fp32 in TMEM.
+//  * warps 0..3  : softmax of Q tile 0, warps 4..7: Q tile 1.  One thread per row:
+//                  load S from TMEM, mask ragged / block-causal keys, online softmax
+//                  in the exp2 domain, write P (bf16) back over S in TMEM.  O is
+//                  only rescaled when the running max grows by more than 2^8
+//                  (exact: numerator and denominator use the same stale max).
+//  * TMEM (512 columns): S0 | S1 | O0 | O1, 128 columns each; P_w aliases S_w.
+//  * Block-mask tile skipping: a Q tile only visits KV tiles below the largest key
+//    limit of its rows; masks are applied only inside the boundary tile.
+// Every mbarrier wait is bounded (see ptx.cuh); on expiry the CTA raises an abort
+// flag, reports BCA_ERR_DEVICE_TIMEOUT, drains and frees TMEM.
+#pragma once
+#include <cuda_bf16.h>
+
+#include "../../include/bca.h"
+#include "ptx.cuh"
+
+namespace bca {
+
+constexpr int kHeadDim = 128;
+constexpr int kBM = 128;  // Q rows per tile
+constexpr int kBN = 128;  // keys per KV tile
+constexpr int kStages = 4;
+constexpr int kTileBytes = kBM * kHeadDim * 2;  // 32 KiB bf16 tile
+constexpr int kHalfBytes = kTileBytes / 2;      // one 64-column swizzled box
+constexpr int kAttnThreads = 384;
+constexpr int kWarpProducer = 8;
+constexpr int kWarpMma = 9;
+constexpr float kRescaleThreshold = 8.0f;  // log2 units
+constexpr int kNoLimit = 1 << 30;
+
+enum : int { kModePrefill = 0, kModeStep = 1 };
+
+template <int MAXR>
+struct AttnParams {
+  CUtensorMap tm_q;  // [rows, H, 128] bf16, dims (128, H, rows), box (64, 1, 128)
+  CUtensorMap tm_k;  // own keys, same geometry
+  CUtensorMap tm_v;
+  CUtensorMap tm_kc[MAXR];  // cache K of request r: dims (128, n_tokens, H), box (64, 128, 1)
+  CUtensorMap tm_vc[MAXR];
+  __nv_bfloat16* o;
+  int32_t* dev_status;
+  unsigned long long timeout_ns;
+  int32_t heads;
+  int32_t mode;
+  float scale_log2;  // softmax scale * log2(e)
+  // prefill
+  int32_t seq_len;
+  int32_t n_blocks;
+  int32_t block_off[BCA_MAX_BLOCKS + 1];
+  // step: requests in scheduling order
+  int32_t n_req;
+  int32_t unit_start[MAXR + 1];
+  int32_t q_start[MAXR];
+  int32_t q_len[MAXR];
+  int32_t n_cache[MAXR];
+};
+
+// Shared memory map (offsets from a 1024-byte aligned base).
+struct Smem {
+  static constexpr int kQ0 = 0;
+  static constexpr int kQ1 = kTileBytes;
+  static constexpr int kRing = 2 * kTileBytes;
+  static constexpr int kBars = kRing + kStages * kTileBytes;
+  // barrier indices
+  static constexpr int bQFull = 0;                 // 2
+  static constexpr int bKvFull = 2;                // kStages
+  static constexpr int bKvEmpty = 2 + kStages;     // kStages
+  static constexpr int bSFull = 2 + 2 * kStages;   // 2
+  static constexpr int bPFull = 4 + 2 * kStages;   // 2
+  static constexpr int bOFull = 6 + 2 * kStages;   // 2
+  static constexpr int bDone = 8 + 2 * kStages;    // 1
+  static constexpr int kNumBars = 9 + 2 * kStages;
+  static constexpr int kTmemSlot = kBars + 8 * kNumBars;
+  static constexpr int kAbort = kTmemSlot + 4;
+  static constexpr int kBytes = kAbort + 4;
+  static constexpr int kDynamicBytes = kBytes + 1024;  // + alignment slack
+};
+
+// TMEM column bases: S0 | S1 | O0 | O1.
+__host__ __device__ constexpr uint32_t col_s(int w) { return w == 0 ? 0u : 128u; }
+__host__ __device__ constexpr uint32_t col_o(int w) { return w == 0 ? 256u : 384u; }
+
+struct Unit {
+  int req;        // request slot in the params arrays (step mode)
+  int h;          // head
+  int q_row0;     // row of Q tile 0 in the Q/O tensors
+  int rows[2];    // valid rows of each Q tile (<= 0: tile absent)
+  int ntiles[2];  // KV tiles each Q tile visits
+  int n_total;    // max(ntiles)
+  int n_cache_tiles;
+};
+
+template <int MAXR>
+__device__ __forceinline__ int block_end(const AttnParams<MAXR>& p, int row) {
+  for (int b = 1; b <= p.n_blocks; ++b)
+    if (row < p.block_off[b]) return p.block_off[b];
+  return p.seq_len;
+}
+
+template <int MAXR>
+__device__ __forceinline__ Unit decode_unit(const AttnParams<MAXR>& p, int unit) {
+  Unit u;
+  if (p.mode == kModePrefill) {
+    const int S = p.seq_len;
+    const int nqp = (S + 2 * kBM - 1) / (2 * kBM);
+    u.req = 0;
+    u.h = unit / nqp;
+    const int qp = nqp - 1 - unit % nqp;  // heaviest (latest) rows first within a head
+    u.q_row0 = qp * 2 * kBM;
+    u.n_cache_tiles = 0;
+#pragma unroll
+    for (int w = 0; w < 2; ++w) {
+      u.rows[w] = min(kBM, S - u.q_row0 - w * kBM);
+      u.ntiles[w] = 0;
+      if (u.rows[w] > 0) {
+        const int lim = block_end(p, u.q_row0 + w * kBM + u.rows[w] - 1);
+        u.ntiles[w] = (lim + kBN - 1) / kBN;
+      }
+    }
+  } else {
+    int r = 0;
+    while (r + 1 < p.n_req && unit >= p.unit_start[r + 1]) ++r;
+    const int T = p.q_len[r];
+    const int nqp = (T + 2 * kBM - 1) / (2 * kBM);
+    const int local = unit - p.unit_start[r];
+    u.req = r;
+    u.h = local / nqp;
+    const int qp = local % nqp;
+    u.q_row0 = p.q_start[r] + qp * 2 * kBM;
+    u.n_cache_tiles = (p.n_cache[r] + kBN - 1) / kBN;
+    const int nt = u.n_cache_tiles + (T + kBN - 1) / kBN;
+#pragma unroll
+    for (int w = 0; w < 2; ++w) {
+      u.rows[w] = min(kBM, T - qp * 2 * kBM - w * kBM);
+      u.ntiles[w] = u.rows[w] > 0 ? nt : 0;
+    }
+  }
+  u.n_total = max(u.ntiles[0], u.ntiles[1]);
+  return u;
+}
+
+// Geometry of KV tile j of a unit: number of valid keys and index of its first
+// key in the row's key sequence (for the block-causal limit).
+template <int MAXR>
+__device__ __forceinline__ void kv_tile_extent(const AttnParams<MAXR>& p, const Unit& u, int j,
+                                               int& valid, int& key_base) {
+  if (p.mode == kModePrefill) {
+    key_base = j * kBN;
+    valid = min(kBN, p.seq_len - key_base);
+  } else if (j < u.n_cache_tiles) {
+    key_base = j * kBN;
+    valid = min(kBN, p.n_cache[u.req] - key_base);
+  } else {
+    const int jj = j - u.n_cache_tiles;
+    key_base = p.n_cache[u.req] + jj * kBN;
+    valid = min(kBN, p.q_len[u.req] - jj * kBN);
+  }
+}
+
+__device__ __forceinline__ void raise_abort(volatile int* abort, int32_t* dev_status) {
+  *abort = 1;
+  if (dev_status) atomicExch(dev_status, static_cast<int32_t>(BCA_ERR_DEVICE_TIMEOUT));
+}
+
+// ---------------------------------------------------------------------------
+// Producer: one thread.
+// ---------------------------------------------------------------------------
+template <int MAXR>
+__device__ void producer_role(const AttnParams<MAXR>& p, const Unit& u, uint32_t sbase,
+                              uint32_t bars, volatile int* abort) {
+  auto bar = [&](int i) { return bars + 8u * static_cast<uint32_t>(i); };
+#pragma unroll
+  for (int w = 0; w < 2; ++w) {
+    if (u.rows[w] <= 0) continue;
+    const uint32_t dst = sbase + (w == 0 ? Smem::kQ0 : Smem::kQ1);
+    const int z = u.q_row0 + w * kBM;
+    mbar_arrive_expect_tx(bar(Smem::bQFull + w), kTileBytes);
+    tma_load_3d(dst, &p.tm_q, bar(Smem::bQFull + w), 0, u.h, z);
+    tma_load_3d(dst + kHalfBytes, &p.tm_q, bar(Smem::bQFull + w), 64, u.h, z);
+  }
+  int it = 0;
+  bool ok = true;
+  for (int j = 0; j < u.n_total && ok; ++j) {
+    for (int kv = 0; kv < 2; ++kv, ++it) {
+      const int st = it % kStages;
+      const uint32_t ph = static_cast<uint32_t>(it / kStages) & 1u;
+      if (!mbar_wait_bounded(bar(Smem::bKvEmpty + st), ph ^ 1u, abort, p.timeout_ns)) {
+        raise_abort(abort, p.dev_status);
+        ok = false;
+        break;
+      }
+      const uint32_t dst = sbase + Smem::kRing + st * kTileBytes;
+      const uint32_t fb = bar(Smem::bKvFull + st);
+      mbar_arrive_expect_tx(fb, kTileBytes);
+      if (p.mode == kModeStep && j < u.n_cache_tiles) {
+        const CUtensorMap* m = kv ? &p.tm_vc[u.req] : &p.tm_kc[u.req];
+        tma_load_3d(dst, m, fb, 0, j * kBN, u.h);
+        tma_load_3d(dst + kHalfBytes, m, fb, 64, j * kBN, u.h);
+      } else {
+        const CUtensorMap* m = kv ? &p.tm_v : &p.tm_k;
+        const int z = p.mode == kModePrefill ? j * kBN
+                                             : p.q_start[u.req] + (j - u.n_cache_tiles) * kBN;
+        tma_load_3d(dst, m, fb, 0, u.h, z);
+        tma_load_3d(dst + kHalfBytes, m, fb, 64, u.h, z);
+      }
+    }
+  }
+  if (!ok) {
+    // Drain: wait (bounded) for the loads this thread still has in flight.
+    for (int i = max(0, it - kStages); i < it; ++i)
+      mbar_wait_bounded(bar(Smem::bKvFull + i % kStages), static_cast<uint32_t>(i / kStages) & 1u,
+                        abort, p.timeout_ns);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// MMA issuer: one thread.
+// ---------------------------------------------------------------------------
+template <int MAXR>
+__device__ void mma_role(const AttnParams<MAXR>& p, const Unit& u, uint32_t sbase, uint32_t bars,
+                         uint32_t tmem, volatile int* abort) {
+  auto bar = [&](int i) { return bars + 8u * static_cast<uint32_t>(i); };
+  constexpr uint32_t kIdescS = idesc_bf16_f32(kBM, kBN, false);      // Q K^T: K-major B
+  constexpr uint32_t kIdescO = idesc_bf16_f32(kBM, kHeadDim, true);  // P V: MN-major B
+  bool ok = true;
+  auto wait = [&](int b, uint32_t parity) {
+    if (ok && !mbar_wait_bounded(bar(b), parity, abort, p.timeout_ns)) {
+      raise_abort(abort, p.dev_status);
+      ok = false;
+    }
+    return ok;
+  };
+  for (int w = 0; w < 2; ++w)
+    if (u.rows[w] > 0) wait(Smem::bQFull + w, 0);
+  tc_fence_after();
+  const uint32_t sq[2] = {sbase + Smem::kQ0, sbase + Smem::kQ1};
+  for (int j = 0; j <= u.n_total && ok; ++j) {
+    const int itK = 2 * j, itV = 2 * (j - 1) + 1;
+    const int stK = itK % kStages, stV = (itV + kStages) % kStages;
+    if (j < u.n_total) wait(Smem::bKvFull + stK, static_cast<uint32_t>(itK / kStages) & 1u);
+    if (j > 0) wait(Smem::bKvFull + stV, static_cast<uint32_t>(itV / kStages) & 1u);
+    if (!ok) break;
+    tc_fence_after();
+    const uint32_t kt = sbase + Smem::kRing + stK * kTileBytes;
+    const uint32_t vt = sbase + Smem::kRing + stV * kTileBytes;
+#pragma unroll
+    for (int w = 0; w < 2; ++w) {
+      if (j > 0 && j - 1 < u.ntiles[w]) {
+        // O_w += P_w(j-1) V_{j-1}; P must be consumed before S_w(j) overwrites it.
+        if (!wait(Smem::bPFull + w, static_cast<uint32_t>(j - 1) & 1u)) break;
+        tc_fence_after();
+#pragma unroll
+        for (int s = 0; s < kBN / 16; ++s) {
+          const uint64_t bdesc = sdesc_sw128(vt + s * 2048, kHalfBytes, 1024);
+          mma_bf16_ts(tmem + col_o(w), tmem + col_s(w) + s * 8, bdesc, kIdescO,
+                      (j - 1 > 0 || s > 0) ? 1u : 0u);
+        }
+        if (j - 1 == u.ntiles[w] - 1) mma_commit(bar(Smem::bOFull + w));
+      }
+      if (j < u.ntiles[w]) {
+        // S_w = Q_w K_j^T
+#pragma unroll
+        for (int s = 0; s < kHeadDim / 16; ++s) {
+          const uint32_t koff = (s / 4) * kHalfBytes + (s % 4) * 32;
+          mma_bf16_ss(tmem + col_s(w), sdesc_sw128(sq[w] + koff, 16, 1024),
+                      sdesc_sw128(kt + koff, 16, 1024), kIdescS, s > 0 ? 1u : 0u);
+        }
+        mma_commit(bar(Smem::bSFull + w));
+      }
+    }
+    if (!ok) break;
+    if (j < u.n_total) mma_commit(bar(Smem::bKvEmpty + stK));
+    if (j > 0) mma_commit(bar(Smem::bKvEmpty + stV));
+  }
+  // Everything issued must be complete before TMEM is released.
+  mma_commit(bar(Smem::bDone));
+  mbar_wait_bounded(bar(Smem::bDone), 0, abort, p.timeout_ns);
+}
+
+// ---------------------------------------------------------------------------
+// Softmax + epilogue: 128 threads (one warpgroup) per Q tile, one row each.
+// ---------------------------------------------------------------------------
+template <int MAXR>
+__device__ void softmax_role(const AttnParams<MAXR>& p, const Unit& u, int w, uint32_t bars,
+                             uint32_t tmem, volatile int* abort, float v_out_scale) {
+  auto bar = [&](int i) { return bars + 8u * static_cast<uint32_t>(i); };
+  const int rows_w = w ? u.rows[1] : u.rows[0];
+  const int ntiles_w = w ? u.ntiles[1] : u.ntiles[0];
+  if (rows_w <= 0) return;
+  const int warp = (threadIdx.x / 32) % 4;
+  const int lane = threadIdx.x % 32;
+  const int row = warp * 32 + lane;
+  const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+  const uint32_t tS = tmem + lane_off + col_s(w);
+  const uint32_t tO = tmem + lane_off + col_o(w);
+  const int grow = u.q_row0 + w * kBM + row;
+  int lim = kNoLimit;
+  if (p.mode == kModePrefill) lim = row < rows_w ? block_end(p, grow) : p.seq_len;
+  const float sl2 = p.scale_log2;
+  const uint32_t b_s = bar(Smem::bSFull + w), b_p = bar(Smem::bPFull + w);
+  float m_run = -INFINITY, l_run = 0.f;
+  bool ok = true;
+  for (int j = 0; j < ntiles_w; ++j) {
+    const bool got = mbar_wait_bounded(b_s, static_cast<uint32_t>(j) & 1u, abort, p.timeout_ns);
+    if (!__all_sync(0xffffffffu, got)) {
+      raise_abort(abort, p.dev_status);
+      ok = false;
+      break;
+    }
+    tc_fence_after();
+    uint32_t r[128];
+#pragma unroll
+    for (int c = 0; c < 4; ++c)
+      tmem_ld_32x32b_x32(tS + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&r[32 * c]));
+    tmem_wait_ld();
+    int valid, key_base;
+    kv_tile_extent(p, u, j, valid, key_base);
+    const int nv = min(valid, lim - key_base);
+    if (nv < kBN) {
+#pragma unroll
+      for (int c = 0; c < 128; ++c)
+        if (c >= nv) r[c] = __float_as_uint(-INFINITY);
+    }
+    float mx = -INFINITY;
+#pragma unroll
+    for (int c = 0; c < 128; ++c) mx = fmaxf(mx, __uint_as_float(r[c]));
+    const float m_new = mx * sl2;
+    const bool need = m_new > m_run + kRescaleThreshold;
+    float f = 1.0f;
+    if (need) {
+      f = ex2_approx(m_run - m_new);  // 0 on the first tile (m_run = -inf)
+      l_run *= f;
+      m_run = m_new;
+    }
+    const float neg_m = -m_run;
+    float sum = 0.f;
+#pragma unroll
+    for (int c = 0; c < 64; ++c) {
+      const float p0 = ex2_approx(fmaf(__uint_as_float(r[2 * c]), sl2, neg_m));
+      const float p1 = ex2_approx(fmaf(__uint_as_float(r[2 * c + 1]), sl2, neg_m));
+      sum += p0 + p1;
+      r[c] = pack_bf16x2(p0, p1);
+    }
+    l_run += sum;
+    tmem_st_32x32b_x32(tS, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
+    tmem_st_32x32b_x32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
+    // O was last written by P(j-1) V_{j-1}, complete before S(j) was signalled; it
+    // must be rescaled before P(j) V_j is issued (that waits for our arrival).
+    if (j > 0 && __any_sync(0xffffffffu, need)) {
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        uint32_t o[16];
+        tmem_ld_32x32b_x16(tO + 16 * c, o);
+        tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 16; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * f);
+        tmem_st_32x32b_x16(tO + 16 * c, o);
+      }
+    }
+    tmem_wait_st();
+    tc_fence_before();
+    mbar_arrive(b_p);
+  }
+  if (!ok) return;
+  {
+    const bool got = mbar_wait_bounded(bar(Smem::bOFull + w), 0, abort, p.timeout_ns);
+    if (!__all_sync(0xffffffffu, got)) {
+      raise_abort(abort, p.dev_status);
+      return;
+    }
+  }
+  tc_fence_after();
+  const float inv = v_out_scale / l_run;
+  const bool store = row < rows_w;
+  uint4* dst = reinterpret_cast<uint4*>(p.o + (static_cast<size_t>(grow) * p.heads + u.h) * kHeadDim);
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    uint32_t o[32];
+    tmem_ld_32x32b_x32(tO + 32 * c, o);
+    tmem_wait_ld();
+    uint32_t pk[16];
+#pragma unroll
+    for (int e = 0; e < 16; ++e)
+      pk[e] = pack_bf16x2(__uint_as_float(o[2 * e]) * inv, __uint_as_float(o[2 * e + 1]) * inv);
+    if (store) {
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+        dst[4 * c + e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// The kernel
+// ---------------------------------------------------------------------------
+template <int MAXR>
+__global__ void __launch_bounds__(kAttnThreads, 1)
+    attn_fwd_kernel(const __grid_constant__ AttnParams<MAXR> p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t bars = sbase + Smem::kBars;
+  volatile int* abort = reinterpret_cast<volatile int*>(smem + Smem::kAbort);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Smem::kTmemSlot);
+  const int warp = threadIdx.x / 32;
+  const int lane = threadIdx.x % 32;
+  const Unit u = decode_unit(p, blockIdx.x);
+
+  if (threadIdx.x == 0) {
+    auto bar = [&](int i) { return bars + 8u * static_cast<uint32_t>(i); };
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bar(Smem::bQFull + i), 1);
+      mbar_init(bar(Smem::bSFull + i), 1);
+      mbar_init(bar(Smem::bPFull + i), 128);
+      mbar_init(bar(Smem::bOFull + i), 1);
+    }
+    for (int i = 0; i < kStages; ++i) {
+      mbar_init(bar(Smem::bKvFull + i), 1);
+      mbar_init(bar(Smem::bKvEmpty + i), 1);
+    }
+    mbar_init(bar(Smem::bDone), 1);
+    *abort = 0;
+    fence_barrier_init();
+  }
+  if (warp == kWarpProducer && lane == 0) {
+    tma_prefetch_desc(&p.tm_q);
+    tma_prefetch_desc(&p.tm_k);
+    tma_prefetch_desc(&p.tm_v);
+  }
+  if (warp == kWarpMma) {
+    tmem_alloc(smem_u32(tmem_slot), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp < 8) {
+    softmax_role(p, u, warp / 4, bars, tmem, abort, 1.0f);
+  } else if (warp == kWarpProducer) {
+    if (lane == 0) producer_role(p, u, sbase, bars, abort);
+  } else if (warp == kWarpMma) {
+    if (lane == 0) mma_role(p, u, sbase, bars, tmem, abort);
+    __syncwarp();
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kWarpMma) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace bca

@@ -1,0 +1,419 @@
+// bca.cu -- host side of libbca.so: argument validation, TMA descriptors, launches.
+//
+// The three calls of the method (see include/bca.h for the contract of each):
+//   bca_prefill      step-1 block-causal attention (+ prefix K/V into a slot)
+//   bca_kv_store     prefix K/V cache layout, bf16 or OFP8 E4M3 with per-head scales
+//   bca_step_attend  cached-step target attention for a ragged same-phase batch
+// Every step of the path runs in the kernels of attn_kernel.cuh and
+// kv_store_kernel.cuh; this file only checks arguments and enqueues them.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <atomic>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+#include <numeric>
+#include <vector>
+
+#include "../../include/bca.h"
+#include "attn_kernel.cuh"
+#include "kv_store_kernel.cuh"
+
+namespace {
+
+using bca::AttnParams;
+
+std::atomic<unsigned long long> g_timeout_ns{2000000000ull};
+
+// ---------------------------------------------------------------------------
+// Driver entry point for cuTensorMapEncodeTiled (no link-time libcuda dependency)
+// ---------------------------------------------------------------------------
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn g_encode = nullptr;
+std::once_flag g_encode_once;
+
+bool get_encode() {
+  std::call_once(g_encode_once, [] {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+  });
+  return g_encode != nullptr;
+}
+
+// 3-D tiled map over a row-major tensor whose innermost dimension is the 128-wide
+// head dimension.  dims/strides as the driver expects (dims[0] innermost, strides
+// in bytes for dims 1..2).
+bool make_map_3d(CUtensorMap* m, const void* base, CUtensorMapDataType dt, uint64_t d0,
+                 uint64_t d1, uint64_t d2, uint64_t stride1, uint64_t stride2, uint32_t b0,
+                 uint32_t b1, uint32_t b2) {
+  const cuuint64_t dims[3] = {d0, d1, d2};
+  const cuuint64_t strides[2] = {stride1, stride2};
+  const cuuint32_t box[3] = {b0, b1, b2};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return g_encode(m, dt, 3, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// [rows, H, 128] bf16 activations: box = 64 head-dim elements x 1 head x 128 rows.
+bool map_thd(CUtensorMap* m, const void* base, int64_t rows, int heads) {
+  return make_map_3d(m, base, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 128, heads,
+                     static_cast<uint64_t>(rows), 128 * 2, static_cast<uint64_t>(heads) * 128 * 2,
+                     64, 1, 128);
+}
+
+// [H, cap, 128] bf16 cache, exposing only the first n_tokens rows of each head
+// (rows beyond read as zero and are masked by the kernel).
+bool map_cache_bf16(CUtensorMap* m, const void* base, int n_tokens, int cap, int heads) {
+  return make_map_3d(m, base, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 128,
+                     static_cast<uint64_t>(std::max(n_tokens, 1)), static_cast<uint64_t>(heads),
+                     128 * 2, static_cast<uint64_t>(cap) * 128 * 2, 64, 128, 1);
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Per-device one-time kernel attribute setup.
+template <typename K>
+bool ensure_smem_attr(K kernel, int bytes, std::vector<char>& done) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return false;
+  static std::mutex mu;
+  std::lock_guard<std::mutex> lk(mu);
+  if (done.size() <= static_cast<size_t>(dev)) done.resize(dev + 1, 0);
+  if (!done[dev]) {
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) !=
+        cudaSuccess)
+      return false;
+    done[dev] = 1;
+  }
+  return true;
+}
+
+bool dtype_valid(int32_t dt) { return dt == BCA_KV_BF16 || dt == BCA_KV_FP8_V || dt == BCA_KV_FP8_KV; }
+bool k_is_fp8(int32_t dt) { return dt == BCA_KV_FP8_KV; }
+bool v_is_fp8(int32_t dt) { return dt == BCA_KV_FP8_V || dt == BCA_KV_FP8_KV; }
+
+size_t round256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+struct SlotLayout {
+  size_t k_off, v_off, ks_off, vs_off, total;
+};
+
+SlotLayout slot_layout(int32_t cap, int32_t heads, int32_t hd, int32_t dt) {
+  SlotLayout L{};
+  const size_t elems = static_cast<size_t>(cap) * heads * hd;
+  const size_t kb = elems * (k_is_fp8(dt) ? 1 : 2);
+  const size_t vb = elems * (v_is_fp8(dt) ? 1 : 2);
+  L.k_off = 0;
+  L.v_off = round256(kb);
+  L.ks_off = L.v_off + round256(vb);
+  L.vs_off = L.ks_off + round256(static_cast<size_t>(heads) * 4);
+  L.total = L.vs_off + round256(static_cast<size_t>(heads) * 4);
+  return L;
+}
+
+bca_status check_slot_shape(const bca_kv_slot* s, int heads, int hd) {
+  if (!s || !s->k || !s->v) return BCA_ERR_INVALID_ARG;
+  if (!dtype_valid(s->dtype) || s->cap_tokens < 0 || s->num_heads != heads ||
+      s->head_dim != hd)
+    return BCA_ERR_INVALID_ARG;
+  if (!aligned16(s->k) || !aligned16(s->v)) return BCA_ERR_INVALID_ARG;
+  if ((k_is_fp8(s->dtype) && (!s->k_scale || !aligned16(s->k_scale))) ||
+      (v_is_fp8(s->dtype) && (!s->v_scale || !aligned16(s->v_scale))))
+    return BCA_ERR_INVALID_ARG;
+  return BCA_OK;
+}
+
+std::vector<char> g_attr_attn1, g_attr_attn8, g_attr_attn64;
+
+template <int MAXR>
+std::vector<char>& attr_flags() {
+  if (MAXR == 1) return g_attr_attn1;
+  if (MAXR == 8) return g_attr_attn8;
+  return g_attr_attn64;
+}
+
+template <int MAXR>
+bca_status launch_attn(const AttnParams<MAXR>& p, int n_units, cudaStream_t stream) {
+  if (n_units <= 0) return BCA_OK;
+  if (!ensure_smem_attr(bca::attn_fwd_kernel<MAXR>, bca::Smem::kDynamicBytes, attr_flags<MAXR>()))
+    return BCA_ERR_CUDA;
+  bca::attn_fwd_kernel<MAXR>
+      <<<n_units, bca::kAttnThreads, bca::Smem::kDynamicBytes, stream>>>(p);
+  return cudaGetLastError() == cudaSuccess ? BCA_OK : BCA_ERR_CUDA;
+}
+
+// Enqueue the store passes for one slot (no host-side slot updates).
+bca_status enqueue_kv_store(const void* k, const void* v, int32_t n_prefix, int64_t row_stride,
+                            const bca_kv_slot* slot, int32_t* dev_status, cudaStream_t stream) {
+  (void)dev_status;  // the store kernels contain no waits
+  if (n_prefix == 0) return BCA_OK;
+  bca::KvStoreParams p{};
+  p.src[0] = static_cast<const uint16_t*>(k);
+  p.src[1] = static_cast<const uint16_t*>(v);
+  p.dst[0] = slot->k;
+  p.dst[1] = slot->v;
+  p.scale[0] = slot->k_scale;
+  p.scale[1] = slot->v_scale;
+  p.quant[0] = k_is_fp8(slot->dtype) ? 1 : 0;
+  p.quant[1] = v_is_fp8(slot->dtype) ? 1 : 0;
+  p.row_stride = row_stride;
+  p.n_prefix = n_prefix;
+  p.heads = slot->num_heads;
+  p.cap = slot->cap_tokens;
+  const bool any_quant = p.quant[0] || p.quant[1];
+  if (any_quant) {
+    bca::kv_amax_init_kernel<<<dim3(1, 2), 256, 0, stream>>>(p);
+    const int tpb = std::max(8, (n_prefix + 295) / 296);  // ~2 blocks per SM per tensor
+    const int nb = (n_prefix + tpb - 1) / tpb;
+    bca::kv_amax_kernel<<<dim3(nb, 2), bca::kStoreThreads, 0, stream>>>(p, tpb);
+  }
+  const int64_t chunks = static_cast<int64_t>(n_prefix) * p.heads * 16;
+  const int64_t want = (chunks + bca::kStoreThreads - 1) / bca::kStoreThreads;
+  const int grid = static_cast<int>(std::min<int64_t>(want, 148 * 8));
+  bca::kv_write_kernel<<<dim3(grid, 2), bca::kStoreThreads, 0, stream>>>(p);
+  if (any_quant) bca::kv_scale_finalize_kernel<<<dim3(1, 2), 256, 0, stream>>>(p);
+  return cudaGetLastError() == cudaSuccess ? BCA_OK : BCA_ERR_CUDA;
+}
+
+bca_status validate_store(const void* k, const void* v, int32_t n_prefix, int64_t row_stride,
+                          const bca_kv_slot* slot, uint32_t epoch) {
+  if (!slot) return BCA_ERR_INVALID_ARG;
+  if (slot->head_dim != 128) return BCA_ERR_UNSUPPORTED;
+  if (slot->num_heads < 1 || slot->num_heads > 256) return BCA_ERR_INVALID_ARG;
+  bca_status st = check_slot_shape(slot, slot->num_heads, 128);
+  if (st != BCA_OK) return st;
+  if (epoch == 0 || n_prefix < 0) return BCA_ERR_INVALID_ARG;
+  if (n_prefix > slot->cap_tokens) return BCA_ERR_CAPACITY;
+  if (n_prefix > 0) {
+    if (!k || !v || !aligned16(k) || !aligned16(v)) return BCA_ERR_INVALID_ARG;
+    if (row_stride < static_cast<int64_t>(slot->num_heads) * 128 || row_stride % 8 != 0)
+      return BCA_ERR_INVALID_ARG;
+  }
+  return BCA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* bca_status_string(bca_status s) {
+  switch (s) {
+    case BCA_OK: return "BCA_OK";
+    case BCA_ERR_INVALID_ARG: return "BCA_ERR_INVALID_ARG";
+    case BCA_ERR_UNSUPPORTED: return "BCA_ERR_UNSUPPORTED";
+    case BCA_ERR_CAPACITY: return "BCA_ERR_CAPACITY";
+    case BCA_ERR_STATE: return "BCA_ERR_STATE";
+    case BCA_ERR_CUDA: return "BCA_ERR_CUDA";
+    case BCA_ERR_DEVICE_TIMEOUT: return "BCA_ERR_DEVICE_TIMEOUT";
+  }
+  return "BCA_UNKNOWN_STATUS";
+}
+
+const char* bca_version(void) { return "bca 0.1.0 (sm_100a)"; }
+
+void bca_set_wait_timeout_ns(uint64_t ns) {
+  g_timeout_ns.store(std::max<uint64_t>(ns, 1000000ull));
+}
+
+size_t bca_kv_slot_bytes(int32_t cap, int32_t heads, int32_t hd, bca_kv_dtype dt) {
+  if (cap < 0 || heads < 1 || hd < 1 || !dtype_valid(dt)) return 0;
+  return slot_layout(cap, heads, hd, dt).total;
+}
+
+bca_status bca_kv_slot_init(bca_kv_slot* slot, void* base, int32_t cap, int32_t heads,
+                            int32_t hd, bca_kv_dtype dt) {
+  if (!slot || !base || (reinterpret_cast<uintptr_t>(base) & 255u) != 0) return BCA_ERR_INVALID_ARG;
+  if (cap < 0 || heads < 1 || hd < 1 || !dtype_valid(dt)) return BCA_ERR_INVALID_ARG;
+  const SlotLayout L = slot_layout(cap, heads, hd, dt);
+  char* b = static_cast<char*>(base);
+  slot->k = b + L.k_off;
+  slot->v = b + L.v_off;
+  slot->k_scale = reinterpret_cast<float*>(b + L.ks_off);
+  slot->v_scale = reinterpret_cast<float*>(b + L.vs_off);
+  slot->cap_tokens = cap;
+  slot->n_tokens = 0;
+  slot->num_heads = heads;
+  slot->head_dim = hd;
+  slot->dtype = dt;
+  slot->epoch = 0;
+  return BCA_OK;
+}
+
+bca_status bca_kv_store(const void* k, const void* v, int32_t n_prefix, int32_t row_stride_elems,
+                        bca_kv_slot* slot, uint32_t epoch, int32_t* dev_status, void* stream) {
+  bca_status st = validate_store(k, v, n_prefix, row_stride_elems, slot, epoch);
+  if (st != BCA_OK) return st;
+  st = enqueue_kv_store(k, v, n_prefix, row_stride_elems, slot, dev_status,
+                        static_cast<cudaStream_t>(stream));
+  if (st != BCA_OK) return st;
+  slot->n_tokens = n_prefix;
+  slot->epoch = epoch;
+  return BCA_OK;
+}
+
+bca_status bca_prefill(const void* q, const void* k, const void* v, void* o, int32_t seq_len,
+                       const int32_t* off, int32_t n_blocks, int32_t heads, int32_t head_dim,
+                       float scale, bca_kv_slot* slot, uint32_t epoch, int32_t* dev_status,
+                       void* stream) {
+  if (!q || !k || !v || !o || !off) return BCA_ERR_INVALID_ARG;
+  if (head_dim != 128) return BCA_ERR_UNSUPPORTED;
+  if (heads < 1 || heads > 256 || seq_len < 1) return BCA_ERR_INVALID_ARG;
+  if (n_blocks < 1 || n_blocks > BCA_MAX_BLOCKS) return BCA_ERR_INVALID_ARG;
+  if (!(scale > 0.0f) || !std::isfinite(scale)) return BCA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return BCA_ERR_INVALID_ARG;
+  if (off[0] != 0 || off[n_blocks] != seq_len) return BCA_ERR_INVALID_ARG;
+  for (int b = 0; b < n_blocks; ++b)
+    if (off[b + 1] <= off[b]) return BCA_ERR_INVALID_ARG;
+  const int32_t n_prefix = off[n_blocks - 1];
+  if (slot) {
+    if (slot->num_heads != heads) return BCA_ERR_INVALID_ARG;
+    bca_status st = validate_store(k, v, n_prefix, static_cast<int64_t>(heads) * 128, slot, epoch);
+    if (st != BCA_OK) return st;
+  }
+  if (!get_encode()) return BCA_ERR_CUDA;
+  AttnParams<1> p;
+  std::memset(&p, 0, sizeof(p));
+  if (!map_thd(&p.tm_q, q, seq_len, heads) || !map_thd(&p.tm_k, k, seq_len, heads) ||
+      !map_thd(&p.tm_v, v, seq_len, heads))
+    return BCA_ERR_CUDA;
+  p.tm_kc[0] = p.tm_k;  // unused in prefill mode
+  p.tm_vc[0] = p.tm_v;
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.dev_status = dev_status;
+  p.timeout_ns = g_timeout_ns.load();
+  p.heads = heads;
+  p.mode = bca::kModePrefill;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.seq_len = seq_len;
+  p.n_blocks = n_blocks;
+  for (int b = 0; b <= n_blocks; ++b) p.block_off[b] = off[b];
+  const int nqp = (seq_len + 2 * bca::kBM - 1) / (2 * bca::kBM);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  bca_status st = launch_attn(p, nqp * heads, s);
+  if (st != BCA_OK) return st;
+  if (slot) {
+    st = enqueue_kv_store(k, v, n_prefix, static_cast<int64_t>(heads) * 128, slot, dev_status, s);
+    if (st != BCA_OK) return st;
+    slot->n_tokens = n_prefix;
+    slot->epoch = epoch;
+  }
+  return BCA_OK;
+}
+
+bca_status bca_step_attend(const void* q_t, const void* k_t, const void* v_t, void* o_t,
+                           const int32_t* cu, const bca_kv_slot* slots, int32_t n_req,
+                           int32_t heads, int32_t head_dim, float scale, int32_t* dev_status,
+                           void* stream) {
+  if (!cu || !slots) return BCA_ERR_INVALID_ARG;
+  if (head_dim != 128) return BCA_ERR_UNSUPPORTED;
+  if (heads < 1 || heads > 256 || n_req < 1 || n_req > BCA_MAX_BATCH) return BCA_ERR_INVALID_ARG;
+  if (!(scale > 0.0f) || !std::isfinite(scale)) return BCA_ERR_INVALID_ARG;
+  if (cu[0] != 0) return BCA_ERR_INVALID_ARG;
+  for (int r = 0; r < n_req; ++r)
+    if (cu[r + 1] < cu[r]) return BCA_ERR_INVALID_ARG;
+  const int32_t total = cu[n_req];
+  if (total > 0) {
+    if (!q_t || !k_t || !v_t || !o_t) return BCA_ERR_INVALID_ARG;
+    if (!aligned16(q_t) || !aligned16(k_t) || !aligned16(v_t) || !aligned16(o_t))
+      return BCA_ERR_INVALID_ARG;
+  }
+  for (int r = 0; r < n_req; ++r) {
+    bca_status st = check_slot_shape(&slots[r], heads, 128);
+    if (st != BCA_OK) return st;
+    if (slots[r].epoch == 0) return BCA_ERR_STATE;
+    if (slots[r].n_tokens < 0 || slots[r].n_tokens > slots[r].cap_tokens)
+      return BCA_ERR_INVALID_ARG;
+    if (slots[r].dtype != slots[0].dtype) return BCA_ERR_UNSUPPORTED;
+  }
+  if (slots[0].dtype != BCA_KV_BF16) return BCA_ERR_UNSUPPORTED;
+  if (total == 0) return BCA_OK;
+  if (!get_encode()) return BCA_ERR_CUDA;
+
+  // Longest key sequence first (largest per-unit work scheduled first).
+  std::vector<int> order;
+  for (int r = 0; r < n_req; ++r)
+    if (cu[r + 1] > cu[r]) order.push_back(r);
+  std::stable_sort(order.begin(), order.end(), [&](int a, int b) {
+    return slots[a].n_tokens + (cu[a + 1] - cu[a]) > slots[b].n_tokens + (cu[b + 1] - cu[b]);
+  });
+  const int nr = static_cast<int>(order.size());
+  auto fill = [&](auto& p) -> bca_status {
+    std::memset(&p, 0, sizeof(p));
+    if (!map_thd(&p.tm_q, q_t, total, heads) || !map_thd(&p.tm_k, k_t, total, heads) ||
+        !map_thd(&p.tm_v, v_t, total, heads))
+      return BCA_ERR_CUDA;
+    p.o = static_cast<__nv_bfloat16*>(o_t);
+    p.dev_status = dev_status;
+    p.timeout_ns = g_timeout_ns.load();
+    p.heads = heads;
+    p.mode = bca::kModeStep;
+    p.scale_log2 = scale * 1.4426950408889634f;
+    p.n_req = nr;
+    int units = 0;
+    for (int i = 0; i < nr; ++i) {
+      const int r = order[i];
+      const bca_kv_slot& sl = slots[r];
+      if (!map_cache_bf16(&p.tm_kc[i], sl.k, sl.n_tokens, sl.cap_tokens, heads) ||
+          !map_cache_bf16(&p.tm_vc[i], sl.v, sl.n_tokens, sl.cap_tokens, heads))
+        return BCA_ERR_CUDA;
+      p.q_start[i] = cu[r];
+      p.q_len[i] = cu[r + 1] - cu[r];
+      p.n_cache[i] = sl.n_tokens;
+      p.unit_start[i] = units;
+      units += heads * ((p.q_len[i] + 2 * bca::kBM - 1) / (2 * bca::kBM));
+    }
+    p.unit_start[nr] = units;
+    return launch_attn(p, units, static_cast<cudaStream_t>(stream));
+  };
+  if (nr <= 1) {
+    AttnParams<1> p;
+    return fill(p);
+  } else if (nr <= 8) {
+    AttnParams<8> p;
+    return fill(p);
+  }
+  AttnParams<64> p;
+  return fill(p);
+}
+
+}  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Bounded-wait self-check
+// ---------------------------------------------------------------------------
+namespace {
+__global__ void selftest_wait_kernel(int32_t* dev_status, unsigned long long timeout_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort;
+  const uint32_t b = bca::smem_u32(&bar);
+  if (threadIdx.x == 0) {
+    bca::mbar_init(b, 1);  // nothing ever arrives
+    abort = 0;
+    bca::fence_barrier_init();
+  }
+  __syncthreads();
+  const bool ok = bca::mbar_wait_bounded(b, 0, &abort, timeout_ns);
+  if (!__all_sync(0xffffffffu, ok) && threadIdx.x == 0)
+    bca::raise_abort(reinterpret_cast<volatile int*>(&abort), dev_status);
+}
+}  // namespace
+
+extern "C" bca_status bca_selftest_wait_timeout(int32_t* dev_status, uint64_t timeout_ns,
+                                                void* stream) {
+  if (!dev_status) return BCA_ERR_INVALID_ARG;
+  if (timeout_ns < 1000000ull || timeout_ns > 10000000000ull) return BCA_ERR_INVALID_ARG;
+  selftest_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(dev_status, timeout_ns);
+  return cudaGetLastError() == cudaSuccess ? BCA_OK : BCA_ERR_CUDA;
+}

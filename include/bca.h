@@ -1,0 +1,179 @@
+/*
+ * bca.h -- block-causal attention with cross-step prefix K/V reuse, sm_100a.
+ *
+ * C ABI of libbca.so.  Plain pointers and sizes only; no framework types.
+ *
+ * The method (cited by page title and section):
+ *  - "Qwen-Image-2.1 + vLLM-Omni day-0" (thakicloud.com), "What is Qwen-Image-2.1":
+ *    the single-stream DiT uses block-causal attention.  The sequence is split
+ *    into ordered blocks (text prompt, reference images 1..k, target latents);
+ *    block b attends to blocks 0..b, with full attention inside a block.
+ *  - same page, "Serving architecture: the cross-step prefix KV cache": since the
+ *    prefix blocks never see the target, their K/V from the first denoising step
+ *    are exact for every later step, so they are stored once and reused; the cache
+ *    is rebuilt for every new request, so nothing leaks between requests.
+ *  - "Qwen/Qwen-Image-2.1" (recipes.vllm.ai), "Prefix KV cache": reuse is exact;
+ *    the cache may be stored in FP8 -- "fp8_v" quantises V only, "fp8" K too.
+ *  - same page, "Online serving": requests at the same KV-cache phase are batched
+ *    together (--step-execution --max-num-seqs 8).
+ *
+ * Conventions common to every call:
+ *  - Element types: activations are bf16; softmax and accumulation are fp32.
+ *  - Activation layout ("THD"): [tokens, heads, head_dim], head_dim contiguous,
+ *    token rows heads*head_dim elements apart unless a stride is given.
+ *  - Cache layout: per (request, layer) slot, K and V each [heads, cap_tokens,
+ *    head_dim]; bf16, or OFP8 E4M3 codes (1 byte) with one fp32 scale per head.
+ *  - All device memory is owned by the caller.  The library allocates no device
+ *    memory; it keeps only host-side state (a driver entry point).
+ *  - Calls enqueue work on `stream` and return at once.  Argument and state
+ *    errors are reported synchronously, before anything is launched, and then
+ *    nothing is written.  A failed launch returns BCA_ERR_CUDA.
+ *  - Every device-side wait is bounded.  When a bound expires the kernel stores
+ *    BCA_ERR_DEVICE_TIMEOUT into *dev_status (if dev_status is not NULL), drains
+ *    and returns; the host reads *dev_status after synchronising.
+ *  - Supported now: head_dim == 128, heads in [1, 256], device pointers 16-byte
+ *    aligned, finite inputs.
+ *  - A softmax scale is passed in (1/sqrt(head_dim) for the DiT).
+ */
+#ifndef BCA_H_
+#define BCA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  BCA_OK = 0,
+  BCA_ERR_INVALID_ARG = 1,    /* a pointer, size, stride or offset is invalid      */
+  BCA_ERR_UNSUPPORTED = 2,    /* valid but not implemented (e.g. head_dim != 128)  */
+  BCA_ERR_CAPACITY = 3,       /* prefix longer than the slot's cap_tokens          */
+  BCA_ERR_STATE = 4,          /* slot not filled for the current request (epoch 0) */
+  BCA_ERR_CUDA = 5,           /* a CUDA runtime/driver call or a launch failed     */
+  BCA_ERR_DEVICE_TIMEOUT = 6  /* a bounded device-side wait expired                */
+} bca_status;
+
+/* Cache element type, mirroring the recipe's prefix_kv_cache_dtype values. */
+typedef enum {
+  BCA_KV_BF16 = 0,   /* K and V bf16                      ("bf16", default)  */
+  BCA_KV_FP8_V = 1,  /* K bf16, V e4m3 + per-head scale   ("fp8_v")          */
+  BCA_KV_FP8_KV = 2  /* K and V e4m3 + per-head scales    ("fp8")            */
+} bca_kv_dtype;
+
+/* Maximum number of blocks in one prefill sequence and of requests in one
+ * cached-step call. */
+#define BCA_MAX_BLOCKS 64
+#define BCA_MAX_BATCH 64
+
+/* One (request, layer) prefix K/V cache slot.  The struct lives in host memory
+ * and is owned by the caller; the buffers it points to are device memory owned
+ * by the caller.
+ *   k, v      : [num_heads, cap_tokens, head_dim]; bf16, or e4m3 bytes when the
+ *               dtype quantises that tensor.
+ *   k_scale,
+ *   v_scale   : device fp32 [num_heads]; read/written only for e4m3 tensors
+ *               (may be NULL otherwise).  Dequantised value = fp32(decode(code) * scale).
+ *   n_tokens  : prefix rows currently stored (set by bca_kv_store / bca_prefill).
+ *   epoch     : 0 = empty.  Storing stamps the caller's (non-zero) request epoch;
+ *               a new request stores again with a new epoch (per-request rebuild).
+ * Use bca_kv_slot_init to carve a slot from one caller allocation. */
+typedef struct bca_kv_slot {
+  void* k;
+  void* v;
+  float* k_scale;
+  float* v_scale;
+  int32_t cap_tokens;
+  int32_t n_tokens;
+  int32_t num_heads;
+  int32_t head_dim;
+  int32_t dtype; /* bca_kv_dtype */
+  uint32_t epoch;
+} bca_kv_slot;
+
+/* Bytes of one device allocation that bca_kv_slot_init can carve into a slot
+ * (K, V and both scale arrays, each 256-byte aligned).  Returns 0 for invalid
+ * sizes. */
+size_t bca_kv_slot_bytes(int32_t cap_tokens, int32_t num_heads, int32_t head_dim,
+                         bca_kv_dtype dtype);
+
+/* Fill *slot with pointers into `base` (device, 256-byte aligned, at least
+ * bca_kv_slot_bytes(...) bytes) and mark it empty (n_tokens = 0, epoch = 0).
+ * Host-only; touches no device memory.
+ * Errors: BCA_ERR_INVALID_ARG (NULL, misaligned base or invalid sizes). */
+bca_status bca_kv_slot_init(bca_kv_slot* slot, void* base, int32_t cap_tokens,
+                            int32_t num_heads, int32_t head_dim, bca_kv_dtype dtype);
+
+/* Store prefix K/V rows [0, n_prefix) of one request/layer into `slot`, in the
+ * slot's dtype (the cache layout step of the method; "Prefix KV cache" on the
+ * recipe page for the FP8 modes).
+ *   k, v            : device bf16, token t / head h at element t*row_stride + h*head_dim.
+ *   n_prefix        : 0 <= n_prefix <= slot->cap_tokens (else BCA_ERR_CAPACITY).
+ *   row_stride_elems: elements between consecutive token rows (>= heads*head_dim,
+ *                     multiple of 8).
+ *   epoch           : non-zero request epoch stamped into the slot.
+ * For an e4m3 tensor: amax = max |x| over the n_prefix rows of each head,
+ * scale = fp32(amax)/448 (1 when amax == 0), code = e4m3 RNE-satfinite of the
+ * correctly rounded fp32 quotient x/scale.  Rows [n_prefix, cap) are not written.
+ * Host side effects (at enqueue): slot->n_tokens = n_prefix, slot->epoch = epoch.
+ * dev_status: nullable device int32, see the conventions above. */
+bca_status bca_kv_store(const void* k, const void* v, int32_t n_prefix,
+                        int32_t row_stride_elems, bca_kv_slot* slot, uint32_t epoch,
+                        int32_t* dev_status, void* stream);
+
+/* Step 1 (prefill) of one request at one layer: block-causal attention over the
+ * whole sequence ("What is Qwen-Image-2.1" and "Serving architecture: the
+ * cross-step prefix KV cache" on the thakicloud page).
+ *   q, k, v, o   : device bf16 [seq_len, heads, 128]; o is written.
+ *   block_offsets: HOST int32[n_blocks + 1], 0 = off[0] < off[1] < ... <
+ *                  off[n_blocks] = seq_len; row i attends to keys [0, end of its block).
+ *   n_blocks     : 1..BCA_MAX_BLOCKS.  The last block is the target.
+ *   slot         : nullable.  When given, rows [0, off[n_blocks-1]) (every block
+ *                  but the target) of k and v are stored into it exactly as
+ *                  bca_kv_store does, stamped with `epoch` (non-zero).
+ * o and q/k/v must not overlap. */
+bca_status bca_prefill(const void* q, const void* k, const void* v, void* o, int32_t seq_len,
+                       const int32_t* block_offsets, int32_t n_blocks, int32_t heads,
+                       int32_t head_dim, float scale, bca_kv_slot* slot, uint32_t epoch,
+                       int32_t* dev_status, void* stream);
+
+/* Steps 2..N of a batch of requests at the same phase: every target row of
+ * request r attends to [slot r's cached prefix rows ; request r's own target
+ * rows], with no mask (the target is the last block, so it sees everything).
+ *   q_t, k_t, v_t, o_t: device bf16, packed target rows of all requests,
+ *                      [sum_r T_r, heads, 128]; request r owns rows
+ *                      [cu_target[r], cu_target[r+1]).
+ *   cu_target        : HOST int32[n_req + 1], cu_target[0] = 0, non-decreasing.
+ *   slots            : HOST array of n_req slots; each filled (epoch != 0) with
+ *                      num_heads == heads, head_dim == 128, and all the same dtype.
+ *   n_req            : 1..BCA_MAX_BATCH.
+ * For e4m3 tensors the per-head scales are folded in: K's into the softmax scale,
+ * V's into the output normalisation.  A request with T_r == 0 is skipped.
+ * Errors: BCA_ERR_STATE for an empty slot, BCA_ERR_UNSUPPORTED for mixed dtypes. */
+bca_status bca_step_attend(const void* q_t, const void* k_t, const void* v_t, void* o_t,
+                           const int32_t* cu_target, const bca_kv_slot* slots, int32_t n_req,
+                           int32_t heads, int32_t head_dim, float scale, int32_t* dev_status,
+                           void* stream);
+
+/* Human-readable name of a status code (static storage). */
+const char* bca_status_string(bca_status status);
+
+/* Upper bound, in nanoseconds, of every device-side wait (default 2e9 = 2 s).
+ * Values < 1e6 are raised to 1e6.  Applies to launches enqueued afterwards. */
+void bca_set_wait_timeout_ns(uint64_t timeout_ns);
+
+/* Self-check of the bounded-wait path: launches one CTA that waits on a barrier
+ * nothing will ever complete, for at most timeout_ns, then stores
+ * BCA_ERR_DEVICE_TIMEOUT into *dev_status and returns.  Lets a host test see a
+ * device timeout without hanging or faulting the GPU. */
+bca_status bca_selftest_wait_timeout(int32_t* dev_status, uint64_t timeout_ns, void* stream);
+
+/* Library version string. */
+const char* bca_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BCA_H_ */

@@ -1,0 +1,140 @@
+"""The C ABI without a GPU: the library loads, exports every function that
+include/bca.h declares, and rejects invalid arguments on the host before any CUDA
+call (so these checks never touch a device)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import block_causal_attention_dit_b200 as bca
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "bca.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    from block_causal_attention_dit_b200 import build
+    build.build()
+    return bca.lib()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    names = re.findall(r"\b(bca_[a-z0-9_]+)\s*\(", text)
+    return sorted(set(names))
+
+
+def test_header_declares_the_three_calls():
+    names = declared_functions()
+    for n in ("bca_prefill", "bca_kv_store", "bca_step_attend"):
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported(L):
+    for name in declared_functions():
+        assert hasattr(L, name), name
+
+
+def test_status_strings(L):
+    for code, name in bca.STATUS_NAMES.items():
+        assert bca.status_string(code) == name
+    assert "sm_100a" in bca.version()
+
+
+def test_slot_bytes_and_layout(L):
+    H, cap = 4, 100
+    nb = bca.slot_bytes(cap, H, 128, "bf16")
+    assert nb >= 2 * cap * H * 128 * 2
+    assert bca.slot_bytes(cap, H, 128, "fp8") < nb
+    assert bca.slot_bytes(-1, H, 128, "bf16") == 0
+    assert bca.slot_bytes(cap, 0, 128, "bf16") == 0
+    s = bca.SlotStruct()
+    base = 1 << 20  # host-side carving only: no memory is touched
+    assert L.bca_kv_slot_init(ctypes.byref(s), ctypes.c_void_p(base), cap, H, 128, bca.KV_FP8_KV) == 0
+    assert s.k == base and s.v > s.k and s.k_scale > s.v and s.v_scale > s.k_scale
+    assert all(x % 256 == 0 for x in (s.k, s.v, s.k_scale, s.v_scale))
+    assert s.v - s.k >= cap * H * 128 and s.epoch == 0 and s.n_tokens == 0
+    assert L.bca_kv_slot_init(ctypes.byref(s), ctypes.c_void_p(base + 16), cap, H, 128, 0) == 1
+
+
+def _slot(L, cap=64, H=2, dt=0, epoch=1, n=10):
+    s = bca.SlotStruct()
+    assert L.bca_kv_slot_init(ctypes.byref(s), ctypes.c_void_p(1 << 20), cap, H, 128, dt) == 0
+    s.epoch, s.n_tokens = epoch, n
+    return s
+
+
+FAKE = ctypes.c_void_p(1 << 24)  # never dereferenced: every case fails validation first
+
+
+def test_prefill_argument_errors(L):
+    off = (ctypes.c_int32 * 3)(0, 64, 128)
+    args = lambda **kw: dict(dict(q=FAKE, k=FAKE, v=FAKE, o=FAKE, S=128, off=off, nb=2, H=2,
+                                  d=128, scale=0.1, slot=None, epoch=0), **kw)
+    call = lambda a: L.bca_prefill(a["q"], a["k"], a["v"], a["o"], a["S"], a["off"], a["nb"],
+                                   a["H"], a["d"], a["scale"], a["slot"], a["epoch"], None, None)
+    assert call(args(q=None)) == 1
+    assert call(args(d=64)) == 2
+    assert call(args(H=0)) == 1
+    assert call(args(S=100)) == 1  # offsets do not end at S
+    assert call(args(nb=0)) == 1
+    assert call(args(scale=0.0)) == 1
+    assert call(args(scale=float("nan"))) == 1
+    assert call(args(q=ctypes.c_void_p((1 << 24) + 8))) == 1  # misaligned
+    bad = (ctypes.c_int32 * 3)(0, 0, 128)
+    assert call(args(off=bad)) == 1  # empty block
+    s = _slot(L, cap=32, H=2)
+    assert call(args(slot=ctypes.pointer(s), epoch=1)) == 3  # prefix 64 > cap 32
+    s = _slot(L, cap=128, H=2)
+    assert call(args(slot=ctypes.pointer(s), epoch=0)) == 1  # epoch 0
+    s = _slot(L, cap=128, H=3)
+    assert call(args(slot=ctypes.pointer(s), epoch=1)) == 1  # head mismatch
+
+
+def test_kv_store_argument_errors(L):
+    s = _slot(L, cap=16, H=2)
+    st = lambda **kw: L.bca_kv_store(kw.get("k", FAKE), kw.get("v", FAKE), kw.get("n", 8),
+                                     kw.get("stride", 256), ctypes.byref(kw.get("slot", s)),
+                                     kw.get("epoch", 1), None, None)
+    assert st(n=17) == 3
+    assert st(n=-1) == 1
+    assert st(epoch=0) == 1
+    assert st(stride=128) == 1  # < heads * 128
+    assert st(stride=260) == 1  # not a multiple of 8
+    assert st(k=None) == 1
+    assert L.bca_kv_store(FAKE, FAKE, 4, 256, None, 1, None, None) == 1
+    s2 = _slot(L, cap=16, H=2, dt=2)
+    s2.k_scale = None
+    assert st(slot=s2) == 1
+    s3 = _slot(L, cap=16, H=2)
+    s3.head_dim = 64
+    assert st(slot=s3) == 2
+
+
+def test_step_attend_argument_errors(L):
+    cu = (ctypes.c_int32 * 3)(0, 100, 228)
+    s0, s1 = _slot(L, n=10), _slot(L, n=20)
+    arr = (bca.SlotStruct * 2)(s0, s1)
+    call = lambda **kw: L.bca_step_attend(FAKE, FAKE, FAKE, FAKE, kw.get("cu", cu),
+                                          kw.get("arr", arr), kw.get("n", 2), kw.get("H", 2),
+                                          kw.get("d", 128), kw.get("scale", 0.1), None, None)
+    assert call(d=96) == 2
+    assert call(n=0) == 1
+    assert call(n=65) == 1
+    assert call(H=4) == 1  # slots have 2 heads
+    assert call(cu=(ctypes.c_int32 * 3)(0, 100, 50)) == 1
+    assert call(cu=(ctypes.c_int32 * 3)(1, 100, 228)) == 1
+    empty = (bca.SlotStruct * 2)(s0, _slot(L, epoch=0))
+    assert call(arr=empty) == 4
+    mixed = (bca.SlotStruct * 2)(s0, _slot(L, dt=2))
+    assert call(arr=mixed) == 2
+    over = _slot(L, cap=64, n=65)
+    assert call(arr=(bca.SlotStruct * 2)(s0, over)) == 1
+
+
+def test_selftest_wait_rejects_bad_bounds(L):
+    assert L.bca_selftest_wait_timeout(None, 10_000_000, None) == 1
+    assert L.bca_selftest_wait_timeout(FAKE, 10, None) == 1

@@ -1,0 +1,94 @@
+"""bca_kv_store on the GPU against the oracle: bf16 copies exact, e4m3 cache bytes
+and per-head scales bit-exact ("Qwen/Qwen-Image-2.1" vLLM recipe, "Prefix KV
+cache": "fp8_v" quantises V only, "fp8" K and V)."""
+import numpy as np
+import pytest
+import torch
+
+import block_causal_attention_dit_b200 as bca
+import oracle
+from block_causal_attention_dit_b200.workloads import randn_bf16
+
+pytestmark = pytest.mark.gpu
+
+
+def _fill_sentinel(slot):
+    slot.buffer.fill_(0x5A)
+
+
+@pytest.mark.parametrize("P,H,cap", [(128, 4, 128), (77, 3, 200), (1, 2, 5), (513, 32, 600)])
+def test_bf16_copy_exact(cuda_device, P, H, cap):
+    k = randn_bf16((P + 9, H, 128), 11, cuda_device)
+    v = randn_bf16((P + 9, H, 128), 12, cuda_device)
+    slot = bca.KVSlot(cap, H, "bf16")
+    _fill_sentinel(slot)
+    bca.kv_store(k, v, P, slot, epoch=7)
+    torch.cuda.synchronize()
+    assert slot.n_tokens == P and slot.epoch == 7
+    assert torch.equal(slot.k_view()[:, :P], k[:P].permute(1, 0, 2))
+    assert torch.equal(slot.v_view()[:, :P], v[:P].permute(1, 0, 2))
+    # rows beyond the prefix are untouched
+    tail = slot.k_view()[:, P:].contiguous().view(torch.uint8)
+    assert bool((tail == 0x5A).all())
+
+
+@pytest.mark.parametrize("mode", ["fp8", "fp8_v"])
+@pytest.mark.parametrize("P,H,cap,amp", [(128, 4, 128, 1.0), (77, 3, 100, 37.0),
+                                         (1000, 32, 1024, 0.01), (3, 2, 3, 300.0)])
+def test_fp8_bytes_and_scales_bit_exact(cuda_device, mode, P, H, cap, amp):
+    k = (randn_bf16((P, H, 128), 21, cuda_device).float() * amp).to(torch.bfloat16)
+    v = (randn_bf16((P, H, 128), 22, cuda_device).float() * amp * 0.5).to(torch.bfloat16)
+    slot = bca.KVSlot(cap, H, mode)
+    _fill_sentinel(slot)
+    bca.kv_store(k, v, P, slot, epoch=3)
+    torch.cuda.synchronize()
+    vc, vs = oracle.quantize_prefix(v.cpu(), P, cap)
+    assert np.array_equal(slot.v_view()[:, :P].cpu().numpy(), vc[:, :P])
+    assert np.array_equal(slot.v_scale_view().cpu().numpy(), vs)
+    if mode == "fp8":
+        kc, ks = oracle.quantize_prefix(k.cpu(), P, cap)
+        assert np.array_equal(slot.k_view()[:, :P].cpu().numpy(), kc[:, :P])
+        assert np.array_equal(slot.k_scale_view().cpu().numpy(), ks)
+    else:
+        assert torch.equal(slot.k_view()[:, :P], k.permute(1, 0, 2))
+
+
+def test_fp8_strided_source_and_zero_head(cuda_device):
+    P, H = 300, 4
+    big = randn_bf16((P, H * 128 + 64), 31, cuda_device)
+    big[:, 128:256] = 0  # head 1 all zeros -> scale 1, codes 0
+    k = big[:, : H * 128]
+    v = big[:, 64: 64 + H * 128]
+    slot = bca.KVSlot(P, H, "fp8")
+    bca.kv_store(k, v, P, slot, epoch=1, row_stride=big.stride(0))
+    torch.cuda.synchronize()
+    kc, ks = oracle.quantize_prefix(k.contiguous().view(P, H, 128).cpu(), P)
+    vc, vs = oracle.quantize_prefix(v.contiguous().view(P, H, 128).cpu(), P)
+    assert ks[1] == 1.0 and (kc[1] == 0).all()
+    assert np.array_equal(slot.k_view().cpu().numpy(), kc)
+    assert np.array_equal(slot.v_view().cpu().numpy(), vc)
+    assert np.array_equal(slot.k_scale_view().cpu().numpy(), ks)
+    assert np.array_equal(slot.v_scale_view().cpu().numpy(), vs)
+
+
+def test_restore_for_a_new_request(cuda_device):
+    """Per-request rebuild: a slot reused by a shorter second request holds exactly
+    the second request's prefix (its epoch and length), never the first's."""
+    H = 2
+    slot = bca.KVSlot(256, H, "fp8")
+    a = randn_bf16((200, H, 128), 41, cuda_device)
+    b = randn_bf16((60, H, 128), 42, cuda_device) * 3
+    bca.kv_store(a, a, 200, slot, epoch=1)
+    bca.kv_store(b, b, 60, slot, epoch=2)
+    torch.cuda.synchronize()
+    assert slot.epoch == 2 and slot.n_tokens == 60
+    bc, bs = oracle.quantize_prefix(b.cpu(), 60)
+    assert np.array_equal(slot.k_view()[:, :60].cpu().numpy(), bc)
+    assert np.array_equal(slot.k_scale_view().cpu().numpy(), bs)
+
+
+def test_empty_prefix_only_stamps(cuda_device):
+    slot = bca.KVSlot(16, 2, "bf16")
+    x = torch.zeros((1, 2, 128), dtype=torch.bfloat16, device=cuda_device)
+    bca.kv_store(x, x, 0, slot, epoch=5)
+    assert slot.n_tokens == 0 and slot.epoch == 5

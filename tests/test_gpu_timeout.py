@@ -1,0 +1,18 @@
+"""Bounded device waits: a wait on a barrier that nothing completes ends after its
+limit with BCA_ERR_DEVICE_TIMEOUT in the status word, and the context stays usable."""
+import pytest
+import torch
+
+import block_causal_attention_dit_b200 as bca
+
+pytestmark = pytest.mark.gpu
+
+
+def test_wait_expires_with_status(cuda_device):
+    status = torch.zeros(1, dtype=torch.int32, device=cuda_device)
+    bca.selftest_wait_timeout(status, 5_000_000)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 6
+    # the context is still usable
+    x = torch.ones(4, device=cuda_device)
+    assert float((x * 2).sum().item()) == 8.0
