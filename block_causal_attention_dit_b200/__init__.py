@@ -25,10 +25,13 @@ import os
 __all__ = [
     "BcaError", "KVSlot", "KV_BF16", "KV_FP8_V", "KV_FP8_KV", "MAX_BLOCKS", "MAX_BATCH",
     "lib", "prefill", "kv_store", "step_attend", "slot_bytes", "set_wait_timeout_ns",
-    "selftest_wait_timeout", "status_string", "version", "LIB_PATH",
+    "selftest_wait_timeout", "selftest_exp2", "status_string", "version", "LIB_PATH",
 ]
 
-LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libbca.so")
+# BCA_LIBRARY may name another build of the same library (e.g. the self-checking
+# libbca_checked.so); there is no other implementation behind these calls.
+LIB_PATH = os.environ.get("BCA_LIBRARY") or os.path.join(
+    os.path.dirname(os.path.abspath(__file__)), "libbca.so")
 
 KV_BF16, KV_FP8_V, KV_FP8_KV = 0, 1, 2
 _DTYPE_NAMES = {"bf16": KV_BF16, "fp8_v": KV_FP8_V, "fp8": KV_FP8_KV}
@@ -90,6 +93,10 @@ def lib():
     L.bca_set_wait_timeout_ns.argtypes = [u64]
     L.bca_selftest_wait_timeout.restype = ctypes.c_int
     L.bca_selftest_wait_timeout.argtypes = [P, u64, P]
+    L.bca_selftest_exp2.restype = ctypes.c_int
+    L.bca_selftest_exp2.argtypes = [P, P, P, i32, P]
+    L.bca_debug_set_trace.restype = ctypes.c_int
+    L.bca_debug_set_trace.argtypes = [P, i32]
     L.bca_version.restype = ctypes.c_char_p
     L.bca_version.argtypes = []
     _lib = L
@@ -231,3 +238,12 @@ def selftest_wait_timeout(dev_status, timeout_ns: int, stream=None):
     _check(lib().bca_selftest_wait_timeout(_ptr(dev_status), int(timeout_ns),
                                            _stream(stream, dev_status.device)),
            "bca_selftest_wait_timeout")
+
+
+def selftest_exp2(x, stream=None):
+    """(software 2^x, hardware ex2.approx) of a float32 CUDA tensor x."""
+    import torch
+    yp, ym = torch.empty_like(x), torch.empty_like(x)
+    _check(lib().bca_selftest_exp2(_ptr(x), _ptr(yp), _ptr(ym), x.numel(),
+                                   _stream(stream, x.device)), "bca_selftest_exp2")
+    return yp, ym

@@ -39,13 +39,43 @@ constexpr int kBN = 128;  // keys per KV tile
 constexpr int kStages = 4;
 constexpr int kTileBytes = kBM * kHeadDim * 2;  // 32 KiB bf16 tile
 constexpr int kHalfBytes = kTileBytes / 2;      // one 64-column swizzled box
+constexpr int kTile8Bytes = kBN * kHeadDim;     // 16 KiB e4m3 tile
 constexpr int kAttnThreads = 384;
 constexpr int kWarpProducer = 8;
 constexpr int kWarpMma = 9;
+constexpr int kWarpConv0 = 10;  // warps 10 and 11 convert e4m3 cache tiles
+constexpr int kConvThreads = 64;
+// Register split: launched at kLaunchRegs per thread (384 x 168 = 64512), the two
+// softmax warpgroups take kSoftmaxRegs and warpgroup 2 (producer, MMA, converter)
+// keeps kOtherRegs: 128 * (2 * 216 + 72) = 64512.  The host checks the compiled
+// register count against this before launching.
+constexpr uint32_t kLaunchRegs = 168;
+constexpr uint32_t kSoftmaxRegs = 216;
+constexpr uint32_t kOtherRegs = 72;
+static_assert(128 * (2 * kSoftmaxRegs + kOtherRegs) <= kAttnThreads * kLaunchRegs,
+              "register split exceeds the launch allocation");
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
+constexpr int kPolyPairs = 3;  // of every 8 column pairs, exponentiated on the FMA pipe
 constexpr int kNoLimit = 1 << 30;
 
 enum : int { kModePrefill = 0, kModeStep = 1 };
+
+// Pipeline trace of one CTA (builds with BCA_TRACE only): clock64() stamps of the
+// roles' events per KV tile, trace[j * kTraceEvents + event], for j < kTraceTiles.
+constexpr int kTraceEvents = 32;
+constexpr int kTraceTiles = 64;
+#ifdef BCA_TRACE
+#define BCA_TRACE_AT(p, j, ev)                                                          \
+  do {                                                                                  \
+    if ((p).trace && static_cast<int>(blockIdx.x) == (p).trace_cta && (j) < kTraceTiles && \
+        (j) >= 0)                                                                       \
+      (p).trace[(j) * kTraceEvents + (ev)] = clock64();                                 \
+  } while (0)
+#else
+#define BCA_TRACE_AT(p, j, ev) \
+  do {                         \
+  } while (0)
+#endif
 
 template <int MAXR>
 struct AttnParams {
@@ -53,9 +83,13 @@ struct AttnParams {
   CUtensorMap tm_k;  // own keys, same geometry
   CUtensorMap tm_v;
   CUtensorMap tm_kc[MAXR];  // cache K of request r: dims (128, n_tokens, H), box (64, 128, 1)
+                            // (e4m3: box (128, 128, 1) into the staging buffers)
   CUtensorMap tm_vc[MAXR];
   __nv_bfloat16* o;
+  int32_t o_rows;  // rows of the Q/O tensors (bounds of the epilogue stores)
   int32_t* dev_status;
+  unsigned long long* trace;  // BCA_TRACE builds: [kTraceTiles][kTraceEvents] cycle stamps
+  int32_t trace_cta;
   unsigned long long timeout_ns;
   int32_t heads;
   int32_t mode;
@@ -70,6 +104,12 @@ struct AttnParams {
   int32_t q_start[MAXR];
   int32_t q_len[MAXR];
   int32_t n_cache[MAXR];
+  // e4m3 cache tensors (step mode): codes are converted to bf16 in shared memory;
+  // the K scale multiplies the scores of cache keys, the V scale their P.
+  int32_t k_fp8;
+  int32_t v_fp8;
+  const float* k_scale[MAXR];
+  const float* v_scale[MAXR];
 };
 
 // Shared memory map (offsets from a 1024-byte aligned base).
@@ -77,7 +117,8 @@ struct Smem {
   static constexpr int kQ0 = 0;
   static constexpr int kQ1 = kTileBytes;
   static constexpr int kRing = 2 * kTileBytes;
-  static constexpr int kBars = kRing + kStages * kTileBytes;
+  static constexpr int kStage8 = kRing + kStages * kTileBytes;  // 2 x 16 KiB e4m3 tiles
+  static constexpr int kBars = kStage8 + 2 * kTile8Bytes;
   // barrier indices
   static constexpr int bQFull = 0;                 // 2
   static constexpr int bKvFull = 2;                // kStages
@@ -86,7 +127,10 @@ struct Smem {
   static constexpr int bPFull = 4 + 2 * kStages;   // 2
   static constexpr int bOFull = 6 + 2 * kStages;   // 2
   static constexpr int bDone = 8 + 2 * kStages;    // 1
-  static constexpr int kNumBars = 9 + 2 * kStages;
+  static constexpr int bStgFull = 9 + 2 * kStages;   // 2
+  static constexpr int bStgEmpty = 11 + 2 * kStages; // 2
+  static constexpr int bConv = 13 + 2 * kStages;     // 1 (64 converter arrivals per tile)
+  static constexpr int kNumBars = 14 + 2 * kStages;
   static constexpr int kTmemSlot = kBars + 8 * kNumBars;
   static constexpr int kAbort = kTmemSlot + 4;
   static constexpr int kBytes = kAbort + 4;
@@ -174,14 +218,38 @@ __device__ __forceinline__ void kv_tile_extent(const AttnParams<MAXR>& p, const 
   }
 }
 
-__device__ __forceinline__ void raise_abort(volatile int* abort, int32_t* dev_status) {
+// On a failed wait: raise the CTA's abort flag and report the timeout.  Builds with
+// BCA_DEVICE_CHECKS report 1000 + `site` instead (first report wins) so that the
+// wait that gave up can be identified.
+__device__ __forceinline__ void raise_abort(volatile int* abort, int32_t* dev_status,
+                                            int site = 0) {
   *abort = 1;
+#ifdef BCA_DEVICE_CHECKS
+  if (dev_status) atomicCAS(dev_status, 0, 1000 + site);
+#else
+  (void)site;
   if (dev_status) atomicExch(dev_status, static_cast<int32_t>(BCA_ERR_DEVICE_TIMEOUT));
+#endif
 }
+
+// Self-checks of checked builds: a failed check records 2000 + code and the caller
+// skips the access.  Compiled out otherwise.
+#ifdef BCA_DEVICE_CHECKS
+#define BCA_CHECK(dev_status, cond, code)                                        \
+  ((cond) ? true : ((dev_status) ? (atomicCAS((dev_status), 0, 2000 + (code)), false) : false))
+#else
+#define BCA_CHECK(dev_status, cond, code) true
+#endif
 
 // ---------------------------------------------------------------------------
 // Producer: one thread.
 // ---------------------------------------------------------------------------
+template <int MAXR>
+__device__ __forceinline__ bool tile_is_fp8(const AttnParams<MAXR>& p, const Unit& u, int j,
+                                            int kv) {
+  return p.mode == kModeStep && j < u.n_cache_tiles && (kv ? p.v_fp8 : p.k_fp8) != 0;
+}
+
 template <int MAXR>
 __device__ void producer_role(const AttnParams<MAXR>& p, const Unit& u, uint32_t sbase,
                               uint32_t bars, volatile int* abort) {
@@ -195,19 +263,37 @@ __device__ void producer_role(const AttnParams<MAXR>& p, const Unit& u, uint32_t
     tma_load_3d(dst, &p.tm_q, bar(Smem::bQFull + w), 0, u.h, z);
     tma_load_3d(dst + kHalfBytes, &p.tm_q, bar(Smem::bQFull + w), 64, u.h, z);
   }
-  int it = 0;
+  int it = 0, fi = 0;  // item (K_0, V_0, K_1, ...) and e4m3 item counters
   bool ok = true;
   for (int j = 0; j < u.n_total && ok; ++j) {
     for (int kv = 0; kv < 2; ++kv, ++it) {
+      if (tile_is_fp8(p, u, j, kv)) {
+        // e4m3 cache tile -> staging buffer; the converter warps fill the ring slot.
+        const int ss = fi & 1;
+        const uint32_t ph = static_cast<uint32_t>(fi >> 1) & 1u;
+        if (!mbar_wait_bounded(bar(Smem::bStgEmpty + ss), ph ^ 1u, abort, p.timeout_ns)) {
+          raise_abort(abort, p.dev_status, 11);
+          ok = false;
+          break;
+        }
+        const uint32_t fb = bar(Smem::bStgFull + ss);
+        mbar_arrive_expect_tx(fb, kTile8Bytes);
+        if (BCA_CHECK(p.dev_status, u.req < p.n_req && j * kBN < p.n_cache[u.req] && u.h < p.heads, 1))
+          tma_load_3d(sbase + Smem::kStage8 + ss * kTile8Bytes,
+                      kv ? &p.tm_vc[u.req] : &p.tm_kc[u.req], fb, 0, j * kBN, u.h);
+        ++fi;
+        continue;
+      }
       const int st = it % kStages;
       const uint32_t ph = static_cast<uint32_t>(it / kStages) & 1u;
       if (!mbar_wait_bounded(bar(Smem::bKvEmpty + st), ph ^ 1u, abort, p.timeout_ns)) {
-        raise_abort(abort, p.dev_status);
+        raise_abort(abort, p.dev_status, 12);
         ok = false;
         break;
       }
       const uint32_t dst = sbase + Smem::kRing + st * kTileBytes;
       const uint32_t fb = bar(Smem::bKvFull + st);
+      BCA_TRACE_AT(p, j, 23 + kv);
       mbar_arrive_expect_tx(fb, kTileBytes);
       if (p.mode == kModeStep && j < u.n_cache_tiles) {
         const CUtensorMap* m = kv ? &p.tm_vc[u.req] : &p.tm_kc[u.req];
@@ -223,10 +309,93 @@ __device__ void producer_role(const AttnParams<MAXR>& p, const Unit& u, uint32_t
     }
   }
   if (!ok) {
-    // Drain: wait (bounded) for the loads this thread still has in flight.
+    // Drain: wait (time-bounded only) for copies this thread may still have in flight.
+    constexpr unsigned long long kDrainNs = 20000000ull;
     for (int i = max(0, it - kStages); i < it; ++i)
       mbar_wait_bounded(bar(Smem::bKvFull + i % kStages), static_cast<uint32_t>(i / kStages) & 1u,
-                        abort, p.timeout_ns);
+                        nullptr, kDrainNs);
+    for (int i = max(0, fi - 2); i < fi; ++i)
+      mbar_wait_bounded(bar(Smem::bStgFull + (i & 1)), static_cast<uint32_t>(i >> 1) & 1u, nullptr,
+                        kDrainNs);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Converter: warps 10-11 (64 threads) turn staged e4m3 cache tiles into the bf16
+// 128-byte-swizzled layout the MMA reads (e4m3 -> f16 -> bf16 is exact).
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t e4m3x2_to_bf16x2(uint32_t two) {
+  uint32_t h;
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h) : "h"(static_cast<uint16_t>(two & 0xFFFFu)));
+  float lo, hi;
+  asm("cvt.f32.f16 %0, %1;" : "=f"(lo) : "h"(static_cast<uint16_t>(h & 0xFFFFu)));
+  asm("cvt.f32.f16 %0, %1;" : "=f"(hi) : "h"(static_cast<uint16_t>(h >> 16)));
+  return pack_bf16x2(lo, hi);
+}
+
+template <int MAXR>
+__device__ void converter_role(const AttnParams<MAXR>& p, const Unit& u, uint32_t sbase,
+                               uint32_t bars, volatile int* abort) {
+  auto bar = [&](int i) { return bars + 8u * static_cast<uint32_t>(i); };
+  const int c = threadIdx.x - kWarpConv0 * 32;  // 0..63
+  int it = 0, fi = 0;
+  for (int j = 0; j < u.n_cache_tiles && j < u.n_total; ++j) {
+    for (int kv = 0; kv < 2; ++kv, ++it) {
+      if (!tile_is_fp8(p, u, j, kv)) continue;
+      const int ss = fi & 1;
+      const int st = it % kStages;
+      const bool got =
+          mbar_wait_bounded(bar(Smem::bStgFull + ss), static_cast<uint32_t>(fi >> 1) & 1u, abort,
+                            p.timeout_ns) &&
+          mbar_wait_bounded(bar(Smem::bKvEmpty + st),
+                            (static_cast<uint32_t>(it / kStages) & 1u) ^ 1u, abort, p.timeout_ns);
+      if (!got) {
+        raise_abort(abort, p.dev_status, 21);
+        return;
+      }
+      const uint32_t src = sbase + Smem::kStage8 + ss * kTile8Bytes;
+      const uint32_t dst = sbase + Smem::kRing + st * kTileBytes;
+#pragma unroll 4
+      for (int k = 0; k < 16; ++k) {
+        const int gid = k * kConvThreads + c;
+        const int row = gid >> 3, ch = gid & 7;
+        if (!BCA_CHECK(p.dev_status, row < kBN && src + row * 128 + 128 <= sbase + Smem::kBars &&
+                                         dst + kTileBytes <= sbase + Smem::kStage8, 2))
+          continue;
+        uint32_t w0, w1, w2, w3;
+        asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                     : "=r"(w0), "=r"(w1), "=r"(w2), "=r"(w3)
+                     : "r"(src + row * 128 + ((ch ^ (row & 7)) << 4)));
+        const uint32_t o0 = e4m3x2_to_bf16x2(w0), o1 = e4m3x2_to_bf16x2(w0 >> 16);
+        const uint32_t o2 = e4m3x2_to_bf16x2(w1), o3 = e4m3x2_to_bf16x2(w1 >> 16);
+        const uint32_t o4 = e4m3x2_to_bf16x2(w2), o5 = e4m3x2_to_bf16x2(w2 >> 16);
+        const uint32_t o6 = e4m3x2_to_bf16x2(w3), o7 = e4m3x2_to_bf16x2(w3 >> 16);
+        const int k0 = 2 * (ch & 3);
+        const uint32_t base = dst + (ch >> 2) * kHalfBytes + row * 128;
+        asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(
+                         base + ((k0 ^ (row & 7)) << 4)),
+                     "r"(o0), "r"(o1), "r"(o2), "r"(o3)
+                     : "memory");
+        asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(
+                         base + (((k0 + 1) ^ (row & 7)) << 4)),
+                     "r"(o4), "r"(o5), "r"(o6), "r"(o7)
+                     : "memory");
+      }
+      fence_proxy_async_smem();
+      mbar_arrive(bar(Smem::bConv));
+      // Every converter thread waits for the whole tile: none may run ahead and
+      // arrive for the next tile while this phase is still open.
+      if (!mbar_wait_bounded(bar(Smem::bConv), static_cast<uint32_t>(fi) & 1u, abort,
+                             p.timeout_ns)) {
+        raise_abort(abort, p.dev_status, 22);
+        return;
+      }
+      if (c == 0) {
+        mbar_arrive(bar(Smem::bKvFull + st));
+        mbar_arrive(bar(Smem::bStgEmpty + ss));
+      }
+      ++fi;
+    }
   }
 }
 
@@ -236,62 +405,80 @@ __device__ void producer_role(const AttnParams<MAXR>& p, const Unit& u, uint32_t
 template <int MAXR>
 __device__ void mma_role(const AttnParams<MAXR>& p, const Unit& u, uint32_t sbase, uint32_t bars,
                          uint32_t tmem, volatile int* abort) {
+  // Executed by the whole warp so that every value below is warp-uniform (kept in
+  // uniform registers); one elected lane issues each tcgen05 instruction.
   auto bar = [&](int i) { return bars + 8u * static_cast<uint32_t>(i); };
   constexpr uint32_t kIdescS = idesc_bf16_f32(kBM, kBN, false);      // Q K^T: K-major B
   constexpr uint32_t kIdescO = idesc_bf16_f32(kBM, kHeadDim, true);  // P V: MN-major B
   bool ok = true;
   auto wait = [&](int b, uint32_t parity) {
-    if (ok && !mbar_wait_bounded(bar(b), parity, abort, p.timeout_ns)) {
-      raise_abort(abort, p.dev_status);
-      ok = false;
+    if (ok) {
+      const bool got = mbar_wait_bounded(bar(b), parity, abort, p.timeout_ns);
+      if (!__all_sync(0xffffffffu, got)) {
+        if (elect_one()) raise_abort(abort, p.dev_status, 30 + b);
+        ok = false;
+      }
     }
     return ok;
   };
   for (int w = 0; w < 2; ++w)
     if (u.rows[w] > 0) wait(Smem::bQFull + w, 0);
   tc_fence_after();
-  const uint32_t sq[2] = {sbase + Smem::kQ0, sbase + Smem::kQ1};
+  const uint64_t dq[2] = {sdesc_sw128(sbase + Smem::kQ0, 16, 1024),
+                          sdesc_sw128(sbase + Smem::kQ1, 16, 1024)};
   for (int j = 0; j <= u.n_total && ok; ++j) {
     const int itK = 2 * j, itV = 2 * (j - 1) + 1;
     const int stK = itK % kStages, stV = (itV + kStages) % kStages;
+    BCA_TRACE_AT(p, j, 21);
     if (j < u.n_total) wait(Smem::bKvFull + stK, static_cast<uint32_t>(itK / kStages) & 1u);
+    BCA_TRACE_AT(p, j, 22);
     if (j > 0) wait(Smem::bKvFull + stV, static_cast<uint32_t>(itV / kStages) & 1u);
     if (!ok) break;
+    BCA_TRACE_AT(p, j, 0);
     tc_fence_after();
-    const uint32_t kt = sbase + Smem::kRing + stK * kTileBytes;
-    const uint32_t vt = sbase + Smem::kRing + stV * kTileBytes;
+    const uint64_t dk = sdesc_sw128(sbase + Smem::kRing + stK * kTileBytes, 16, 1024);
+    const uint64_t dv = sdesc_sw128(sbase + Smem::kRing + stV * kTileBytes, kHalfBytes, 1024);
 #pragma unroll
     for (int w = 0; w < 2; ++w) {
       if (j > 0 && j - 1 < u.ntiles[w]) {
         // O_w += P_w(j-1) V_{j-1}; P must be consumed before S_w(j) overwrites it.
         if (!wait(Smem::bPFull + w, static_cast<uint32_t>(j - 1) & 1u)) break;
+        BCA_TRACE_AT(p, j, 1 + 2 * w);
         tc_fence_after();
+        if (elect_one()) {
 #pragma unroll
-        for (int s = 0; s < kBN / 16; ++s) {
-          const uint64_t bdesc = sdesc_sw128(vt + s * 2048, kHalfBytes, 1024);
-          mma_bf16_ts(tmem + col_o(w), tmem + col_s(w) + s * 8, bdesc, kIdescO,
-                      (j - 1 > 0 || s > 0) ? 1u : 0u);
+          for (int s = 0; s < kBN / 16; ++s)
+            mma_bf16_ts(tmem + col_o(w), tmem + col_s(w) + s * 8, dv + ((s * 2048) >> 4), kIdescO,
+                        (j - 1 > 0 || s > 0) ? 1u : 0u);
+          if (j - 1 == u.ntiles[w] - 1) mma_commit(bar(Smem::bOFull + w));
         }
-        if (j - 1 == u.ntiles[w] - 1) mma_commit(bar(Smem::bOFull + w));
+        __syncwarp();
       }
       if (j < u.ntiles[w]) {
         // S_w = Q_w K_j^T
+        if (elect_one()) {
 #pragma unroll
-        for (int s = 0; s < kHeadDim / 16; ++s) {
-          const uint32_t koff = (s / 4) * kHalfBytes + (s % 4) * 32;
-          mma_bf16_ss(tmem + col_s(w), sdesc_sw128(sq[w] + koff, 16, 1024),
-                      sdesc_sw128(kt + koff, 16, 1024), kIdescS, s > 0 ? 1u : 0u);
+          for (int s = 0; s < kHeadDim / 16; ++s) {
+            const uint32_t koff = ((s / 4) * kHalfBytes + (s % 4) * 32) >> 4;
+            mma_bf16_ss(tmem + col_s(w), dq[w] + koff, dk + koff, kIdescS, s > 0 ? 1u : 0u);
+          }
+          mma_commit(bar(Smem::bSFull + w));
         }
-        mma_commit(bar(Smem::bSFull + w));
+        __syncwarp();
+        BCA_TRACE_AT(p, j, 2 + 2 * w);
       }
     }
     if (!ok) break;
-    if (j < u.n_total) mma_commit(bar(Smem::bKvEmpty + stK));
-    if (j > 0) mma_commit(bar(Smem::bKvEmpty + stV));
+    if (elect_one()) {
+      if (j < u.n_total) mma_commit(bar(Smem::bKvEmpty + stK));
+      if (j > 0) mma_commit(bar(Smem::bKvEmpty + stV));
+    }
+    __syncwarp();
   }
   // Everything issued must be complete before TMEM is released.
-  mma_commit(bar(Smem::bDone));
-  mbar_wait_bounded(bar(Smem::bDone), 0, abort, p.timeout_ns);
+  if (elect_one()) mma_commit(bar(Smem::bDone));
+  __syncwarp();
+  mbar_wait_bounded(bar(Smem::bDone), 0, nullptr, p.timeout_ns);
 }
 
 // ---------------------------------------------------------------------------
@@ -313,35 +500,64 @@ __device__ void softmax_role(const AttnParams<MAXR>& p, const Unit& u, int w, ui
   const int grow = u.q_row0 + w * kBM + row;
   int lim = kNoLimit;
   if (p.mode == kModePrefill) lim = row < rows_w ? block_end(p, grow) : p.seq_len;
-  const float sl2 = p.scale_log2;
+  // e4m3 cache tiles: scores scale by k_scale (folded into the exp2 scale) and P by
+  // v_scale (folded into the exp2 bias; the row sum keeps the unscaled P).
+  float sl2_cache = p.scale_log2, lg_vs = 0.f, inv_vs = 1.f;
+  if (p.mode == kModeStep) {
+    if (!BCA_CHECK(p.dev_status, u.req < p.n_req && (!p.k_fp8 || p.k_scale[u.req]) &&
+                                     (!p.v_fp8 || p.v_scale[u.req]), 4))
+      return;
+    if (p.k_fp8) sl2_cache *= __ldg(p.k_scale[u.req] + u.h);
+    if (p.v_fp8) {
+      const float vs = __ldg(p.v_scale[u.req] + u.h);
+      lg_vs = __log2f(vs);
+      inv_vs = 1.0f / vs;
+    }
+  }
   const uint32_t b_s = bar(Smem::bSFull + w), b_p = bar(Smem::bPFull + w);
   float m_run = -INFINITY, l_run = 0.f;
   bool ok = true;
   for (int j = 0; j < ntiles_w; ++j) {
     const bool got = mbar_wait_bounded(b_s, static_cast<uint32_t>(j) & 1u, abort, p.timeout_ns);
     if (!__all_sync(0xffffffffu, got)) {
-      raise_abort(abort, p.dev_status);
+      raise_abort(abort, p.dev_status, 61);
       ok = false;
       break;
     }
     tc_fence_after();
+    const bool tr = row == 0;
+    const bool trw = lane == 0 && warp > 0;
+    if (tr) BCA_TRACE_AT(p, j, 5 + 5 * w);
     uint32_t r[128];
 #pragma unroll
     for (int c = 0; c < 4; ++c)
       tmem_ld_32x32b_x32(tS + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&r[32 * c]));
     tmem_wait_ld();
+    if (tr) BCA_TRACE_AT(p, j, 6 + 5 * w);
     int valid, key_base;
     kv_tile_extent(p, u, j, valid, key_base);
+    const bool cache_tile = p.mode == kModeStep && j < u.n_cache_tiles;
+    const float sl2 = cache_tile ? sl2_cache : p.scale_log2;
     const int nv = min(valid, lim - key_base);
     if (nv < kBN) {
 #pragma unroll
       for (int c = 0; c < 128; ++c)
         if (c >= nv) r[c] = __float_as_uint(-INFINITY);
     }
-    float mx = -INFINITY;
+    if (tr && w == 0) BCA_TRACE_AT(p, j, 25);
+    // Row max: 8 independent chains of three-input max, then a short tree.
+    float t[8];
 #pragma unroll
-    for (int c = 0; c < 128; ++c) mx = fmaxf(mx, __uint_as_float(r[c]));
+    for (int i = 0; i < 8; ++i) {
+      const float* x = reinterpret_cast<const float*>(&r[16 * i]);
+      float a = fmax3(x[0], x[1], x[2]);
+#pragma unroll
+      for (int e = 3; e < 15; e += 2) a = fmax3(a, x[e], x[e + 1]);
+      t[i] = fmaxf(a, x[15]);
+    }
+    const float mx = fmax3(fmax3(t[0], t[1], t[2]), fmax3(t[3], t[4], t[5]), fmaxf(t[6], t[7]));
     const float m_new = mx * sl2;
+    if (tr) BCA_TRACE_AT(p, j, 7 + 5 * w);
     const bool need = m_new > m_run + kRescaleThreshold;
     float f = 1.0f;
     if (need) {
@@ -349,16 +565,35 @@ __device__ void softmax_role(const AttnParams<MAXR>& p, const Unit& u, int w, ui
       l_run *= f;
       m_run = m_new;
     }
-    const float neg_m = -m_run;
-    float sum = 0.f;
+    const float neg_m = (cache_tile ? lg_vs : 0.f) - m_run;
+    // p = 2^(s * sl2 - m) on column pairs: packed fp32x2 FMA for the exponent,
+    // then MUFU ex2 for most pairs and the FMA-pipe polynomial for kPolyPairs of
+    // every 8 (balances the two pipes); P is packed to bf16 in place over S.
+    const uint64_t sl2x2 = f2_pack(sl2, sl2), negm2 = f2_pack(neg_m, neg_m);
+    uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
     for (int c = 0; c < 64; ++c) {
-      const float p0 = ex2_approx(fmaf(__uint_as_float(r[2 * c]), sl2, neg_m));
-      const float p1 = ex2_approx(fmaf(__uint_as_float(r[2 * c + 1]), sl2, neg_m));
-      sum += p0 + p1;
+      const uint64_t x = f2_fma(f2_pack(__uint_as_float(r[2 * c]), __uint_as_float(r[2 * c + 1])),
+                                sl2x2, negm2);
+      uint64_t pp;
+      if ((c & 7) >= 8 - kPolyPairs) {
+        pp = exp2_poly2(x);
+      } else {
+        float x0, x1;
+        f2_unpack(x, x0, x1);
+        pp = f2_pack(ex2_approx(x0), ex2_approx(x1));
+      }
+      acc[c & 3] = f2_add(acc[c & 3], pp);
+      float p0, p1;
+      f2_unpack(pp, p0, p1);
       r[c] = pack_bf16x2(p0, p1);
     }
-    l_run += sum;
+    float a0, a1, b0, b1;
+    f2_unpack(f2_add(acc[0], acc[1]), a0, a1);
+    f2_unpack(f2_add(acc[2], acc[3]), b0, b1);
+    const float tile_sum = (a0 + a1) + (b0 + b1);
+    l_run += cache_tile ? tile_sum * inv_vs : tile_sum;
+    if (tr) BCA_TRACE_AT(p, j, 8 + 5 * w);
     tmem_st_32x32b_x32(tS, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
     tmem_st_32x32b_x32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
     // O was last written by P(j-1) V_{j-1}, complete before S(j) was signalled; it
@@ -377,18 +612,21 @@ __device__ void softmax_role(const AttnParams<MAXR>& p, const Unit& u, int w, ui
     tmem_wait_st();
     tc_fence_before();
     mbar_arrive(b_p);
+    if (tr) BCA_TRACE_AT(p, j, 9 + 5 * w);
+    if (trw) BCA_TRACE_AT(p, j, 14 + 3 * w + warp);
   }
   if (!ok) return;
   {
     const bool got = mbar_wait_bounded(bar(Smem::bOFull + w), 0, abort, p.timeout_ns);
     if (!__all_sync(0xffffffffu, got)) {
-      raise_abort(abort, p.dev_status);
+      raise_abort(abort, p.dev_status, 62);
       return;
     }
   }
   tc_fence_after();
   const float inv = v_out_scale / l_run;
-  const bool store = row < rows_w;
+  const bool store = row < rows_w &&
+                     BCA_CHECK(p.dev_status, grow < p.o_rows && u.h < p.heads, 3);
   uint4* dst = reinterpret_cast<uint4*>(p.o + (static_cast<size_t>(grow) * p.heads + u.h) * kHeadDim);
 #pragma unroll
   for (int c = 0; c < 4; ++c) {
@@ -437,6 +675,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       mbar_init(bar(Smem::bKvEmpty + i), 1);
     }
     mbar_init(bar(Smem::bDone), 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bar(Smem::bStgFull + i), 1);
+      mbar_init(bar(Smem::bStgEmpty + i), 1);
+    }
+    mbar_init(bar(Smem::bConv), kConvThreads);
     *abort = 0;
     fence_barrier_init();
   }
@@ -455,12 +698,19 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   const uint32_t tmem = *tmem_slot;
 
   if (warp < 8) {
+    regs_increase<kSoftmaxRegs>();
     softmax_role(p, u, warp / 4, bars, tmem, abort, 1.0f);
+  } else {
+    regs_decrease<kOtherRegs>();
+  }
+  if (warp < 8) {
   } else if (warp == kWarpProducer) {
     if (lane == 0) producer_role(p, u, sbase, bars, abort);
   } else if (warp == kWarpMma) {
-    if (lane == 0) mma_role(p, u, sbase, bars, tmem, abort);
+    mma_role(p, u, sbase, bars, tmem, abort);
     __syncwarp();
+  } else if (p.mode == kModeStep && (p.k_fp8 || p.v_fp8)) {
+    converter_role(p, u, sbase, bars, abort);
   }
   tc_fence_before();
   __syncthreads();

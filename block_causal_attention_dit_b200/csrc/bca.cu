@@ -27,6 +27,8 @@ namespace {
 using bca::AttnParams;
 
 std::atomic<unsigned long long> g_timeout_ns{2000000000ull};
+std::atomic<unsigned long long*> g_trace{nullptr};
+std::atomic<int> g_trace_cta{0};
 
 // ---------------------------------------------------------------------------
 // Driver entry point for cuTensorMapEncodeTiled (no link-time libcuda dependency)
@@ -79,6 +81,13 @@ bool map_cache_bf16(CUtensorMap* m, const void* base, int n_tokens, int cap, int
   return make_map_3d(m, base, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 128,
                      static_cast<uint64_t>(std::max(n_tokens, 1)), static_cast<uint64_t>(heads),
                      128 * 2, static_cast<uint64_t>(cap) * 128 * 2, 64, 128, 1);
+}
+
+// [H, cap, 128] e4m3 cache: one 128-byte box row per token, 128 rows per box.
+bool map_cache_e4m3(CUtensorMap* m, const void* base, int n_tokens, int cap, int heads) {
+  return make_map_3d(m, base, CU_TENSOR_MAP_DATA_TYPE_UINT8, 128,
+                     static_cast<uint64_t>(std::max(n_tokens, 1)), static_cast<uint64_t>(heads),
+                     128, static_cast<uint64_t>(cap) * 128, 128, 128, 1);
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -149,6 +158,17 @@ bca_status launch_attn(const AttnParams<MAXR>& p, int n_units, cudaStream_t stre
   if (n_units <= 0) return BCA_OK;
   if (!ensure_smem_attr(bca::attn_fwd_kernel<MAXR>, bca::Smem::kDynamicBytes, attr_flags<MAXR>()))
     return BCA_ERR_CUDA;
+  // The kernel re-splits its launch registers between warpgroups (setmaxnreg); that
+  // only works if the compiled register count provides the pool the split assumes.
+  static std::once_flag regs_once;
+  static bool regs_ok = false;
+  std::call_once(regs_once, [] {
+    cudaFuncAttributes a{};
+    regs_ok = cudaFuncGetAttributes(&a, bca::attn_fwd_kernel<MAXR>) == cudaSuccess &&
+              static_cast<uint32_t>(a.numRegs) * bca::kAttnThreads >=
+                  128u * (2u * bca::kSoftmaxRegs + bca::kOtherRegs);
+  });
+  if (!regs_ok) return BCA_ERR_CUDA;
   bca::attn_fwd_kernel<MAXR>
       <<<n_units, bca::kAttnThreads, bca::Smem::kDynamicBytes, stream>>>(p);
   return cudaGetLastError() == cudaSuccess ? BCA_OK : BCA_ERR_CUDA;
@@ -227,6 +247,18 @@ void bca_set_wait_timeout_ns(uint64_t ns) {
   g_timeout_ns.store(std::max<uint64_t>(ns, 1000000ull));
 }
 
+bca_status bca_debug_set_trace(unsigned long long* dev_buffer, int32_t cta) {
+#ifdef BCA_TRACE
+  g_trace.store(dev_buffer);
+  g_trace_cta.store(cta);
+  return BCA_OK;
+#else
+  (void)dev_buffer;
+  (void)cta;
+  return BCA_ERR_UNSUPPORTED;
+#endif
+}
+
 size_t bca_kv_slot_bytes(int32_t cap, int32_t heads, int32_t hd, bca_kv_dtype dt) {
   if (cap < 0 || heads < 1 || hd < 1 || !dtype_valid(dt)) return 0;
   return slot_layout(cap, heads, hd, dt).total;
@@ -291,7 +323,10 @@ bca_status bca_prefill(const void* q, const void* k, const void* v, void* o, int
   p.tm_kc[0] = p.tm_k;  // unused in prefill mode
   p.tm_vc[0] = p.tm_v;
   p.o = static_cast<__nv_bfloat16*>(o);
+  p.o_rows = seq_len;
   p.dev_status = dev_status;
+  p.trace = g_trace.load();
+  p.trace_cta = g_trace_cta.load();
   p.timeout_ns = g_timeout_ns.load();
   p.heads = heads;
   p.mode = bca::kModePrefill;
@@ -337,8 +372,8 @@ bca_status bca_step_attend(const void* q_t, const void* k_t, const void* v_t, vo
       return BCA_ERR_INVALID_ARG;
     if (slots[r].dtype != slots[0].dtype) return BCA_ERR_UNSUPPORTED;
   }
-  if (slots[0].dtype != BCA_KV_BF16) return BCA_ERR_UNSUPPORTED;
   if (total == 0) return BCA_OK;
+  const int32_t dt = slots[0].dtype;
   if (!get_encode()) return BCA_ERR_CUDA;
 
   // Longest key sequence first (largest per-unit work scheduled first).
@@ -355,19 +390,30 @@ bca_status bca_step_attend(const void* q_t, const void* k_t, const void* v_t, vo
         !map_thd(&p.tm_v, v_t, total, heads))
       return BCA_ERR_CUDA;
     p.o = static_cast<__nv_bfloat16*>(o_t);
+    p.o_rows = total;
     p.dev_status = dev_status;
+    p.trace = g_trace.load();
+    p.trace_cta = g_trace_cta.load();
     p.timeout_ns = g_timeout_ns.load();
     p.heads = heads;
     p.mode = bca::kModeStep;
     p.scale_log2 = scale * 1.4426950408889634f;
     p.n_req = nr;
+    p.k_fp8 = k_is_fp8(dt) ? 1 : 0;
+    p.v_fp8 = v_is_fp8(dt) ? 1 : 0;
     int units = 0;
     for (int i = 0; i < nr; ++i) {
       const int r = order[i];
       const bca_kv_slot& sl = slots[r];
-      if (!map_cache_bf16(&p.tm_kc[i], sl.k, sl.n_tokens, sl.cap_tokens, heads) ||
-          !map_cache_bf16(&p.tm_vc[i], sl.v, sl.n_tokens, sl.cap_tokens, heads))
-        return BCA_ERR_CUDA;
+      const bool kok = k_is_fp8(dt)
+                           ? map_cache_e4m3(&p.tm_kc[i], sl.k, sl.n_tokens, sl.cap_tokens, heads)
+                           : map_cache_bf16(&p.tm_kc[i], sl.k, sl.n_tokens, sl.cap_tokens, heads);
+      const bool vok = v_is_fp8(dt)
+                           ? map_cache_e4m3(&p.tm_vc[i], sl.v, sl.n_tokens, sl.cap_tokens, heads)
+                           : map_cache_bf16(&p.tm_vc[i], sl.v, sl.n_tokens, sl.cap_tokens, heads);
+      if (!kok || !vok) return BCA_ERR_CUDA;
+      p.k_scale[i] = sl.k_scale;
+      p.v_scale[i] = sl.v_scale;
       p.q_start[i] = cu[r];
       p.q_len[i] = cu[r + 1] - cu[r];
       p.n_cache[i] = sl.n_tokens;
@@ -415,5 +461,34 @@ extern "C" bca_status bca_selftest_wait_timeout(int32_t* dev_status, uint64_t ti
   if (!dev_status) return BCA_ERR_INVALID_ARG;
   if (timeout_ns < 1000000ull || timeout_ns > 10000000000ull) return BCA_ERR_INVALID_ARG;
   selftest_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(dev_status, timeout_ns);
+  return cudaGetLastError() == cudaSuccess ? BCA_OK : BCA_ERR_CUDA;
+}
+
+// ---------------------------------------------------------------------------
+// Software exp2 self-check: the kernel's FMA-pipe 2^x next to the MUFU ex2.
+// ---------------------------------------------------------------------------
+namespace {
+__global__ void selftest_exp2_kernel(const float* x, float* y_poly, float* y_mufu, int n) {
+  const int i = 2 * (blockIdx.x * blockDim.x + threadIdx.x);
+  if (i >= n) return;
+  const float a = x[i], b = (i + 1 < n) ? x[i + 1] : 0.0f;
+  float p0, p1;
+  bca::f2_unpack(bca::exp2_poly2(bca::f2_pack(a, b)), p0, p1);
+  y_poly[i] = p0;
+  y_mufu[i] = bca::ex2_approx(a);
+  if (i + 1 < n) {
+    y_poly[i + 1] = p1;
+    y_mufu[i + 1] = bca::ex2_approx(b);
+  }
+}
+}  // namespace
+
+extern "C" bca_status bca_selftest_exp2(const float* x, float* y_poly, float* y_mufu, int32_t n,
+                                        void* stream) {
+  if (n < 0 || (n > 0 && (!x || !y_poly || !y_mufu))) return BCA_ERR_INVALID_ARG;
+  if (n == 0) return BCA_OK;
+  const int threads = 256, pairs = (n + 1) / 2;
+  selftest_exp2_kernel<<<(pairs + threads - 1) / threads, threads, 0,
+                         static_cast<cudaStream_t>(stream)>>>(x, y_poly, y_mufu, n);
   return cudaGetLastError() == cudaSuccess ? BCA_OK : BCA_ERR_CUDA;
 }

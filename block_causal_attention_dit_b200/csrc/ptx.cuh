@@ -27,6 +27,17 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
 
 __device__ __forceinline__ uint32_t lane_id() { return threadIdx.x & 31u; }
 
+// One lane of the (converged) warp returns true; the others false.
+__device__ __forceinline__ bool elect_one() {
+  uint32_t pred;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "elect.sync _|p, 0xffffffff;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(pred));
+  return pred != 0;
+}
+
 // ---------------------------------------------------------------------------
 // mbarrier
 // ---------------------------------------------------------------------------
@@ -67,8 +78,8 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 }
 
 // Bounded wait for the phase of `bar` with the given parity to complete.
-// Returns false if `timeout_ns` elapsed or another thread raised *abort first;
-// never spins without a bound.
+// Returns false if `timeout_ns` elapsed or another thread raised *abort first
+// (abort may be null: then only the time bound applies); never spins without a bound.
 __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
                                                   const volatile int* abort,
                                                   uint64_t timeout_ns) {
@@ -77,7 +88,7 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((it & 15u) == 0u) {
-      if (*abort) return false;
+      if (abort != nullptr && *abort) return false;
       if (globaltimer_ns() - t0 > timeout_ns) return false;
     }
   }
@@ -115,6 +126,16 @@ __device__ __forceinline__ void tmem_relinquish() {
 __device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
   asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
                : "memory");
+}
+
+// Per-warpgroup register budget (all warps of a warpgroup execute the same one).
+template <uint32_t N>
+__device__ __forceinline__ void regs_increase() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <uint32_t N>
+__device__ __forceinline__ void regs_decrease() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
 }
 
 __device__ __forceinline__ void tc_fence_before() {
@@ -221,11 +242,76 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
+// max(a, b, c) in one instruction (three-input max.f32, sm_100+).
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
 // Two fp32 -> packed bf16x2 (round to nearest even); `lo` lands in bits [0,16).
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   uint32_t r;
   asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
   return r;
+}
+
+// ---------------------------------------------------------------------------
+// Packed fp32x2 arithmetic (sm_100): two lanes of fp32 in one 64-bit register.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ uint64_t f2_sub(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+
+// 2^x for two lanes on the FMA pipe (keeps the MUFU free for the other lanes):
+//  * clamp x >= -127 (2^-127 and below, -inf included, come out as exactly 0);
+//  * range reduction: t = x + 1.5*2^23 rounds x to the integer n held in the low
+//    mantissa bits of t; f = x - n lies in [-1/2, 1/2];
+//  * 2^f by a degree-3 polynomial whose coefficients were fitted here by a Remez
+//    exchange for minimax relative error on [-1/2, 1/2] (max 7.5e-5);
+//  * 2^n built directly as float bits: (bits(t) << 23) + bits(1.0), which is +0.0
+//    for n = -127 (the low 9 bits of bits(1.5*2^23) are zero, so they shift out).
+// Valid for x <= 127 (callers pass x <= 8).
+__device__ __forceinline__ uint64_t exp2_poly2(uint64_t x) {
+  float x0, x1;
+  f2_unpack(x, x0, x1);
+  x = f2_pack(fmaxf(x0, -127.0f), fmaxf(x1, -127.0f));
+  const uint64_t kMagic = f2_pack(12582912.0f, 12582912.0f);
+  const uint64_t t = f2_add(x, kMagic);
+  const uint64_t f = f2_sub(x, f2_sub(t, kMagic));
+  uint64_t q = f2_fma(f, f2_pack(0.0551716685f, 0.0551716685f), f2_pack(0.242611125f, 0.242611125f));
+  q = f2_fma(f, q, f2_pack(0.693260968f, 0.693260968f));
+  q = f2_fma(f, q, f2_pack(0.999928057f, 0.999928057f));
+  float t0, t1;
+  f2_unpack(t, t0, t1);
+  const uint32_t s0 = (__float_as_uint(t0) << 23) + 0x3F800000u;
+  const uint32_t s1 = (__float_as_uint(t1) << 23) + 0x3F800000u;
+  return f2_mul(q, f2_pack(__uint_as_float(s0), __uint_as_float(s1)));
 }
 
 }  // namespace bca

@@ -169,6 +169,19 @@ void bca_set_wait_timeout_ns(uint64_t timeout_ns);
  * device timeout without hanging or faulting the GPU. */
 bca_status bca_selftest_wait_timeout(int32_t* dev_status, uint64_t timeout_ns, void* stream);
 
+/* Self-check of the software 2^x the attention kernels evaluate on the FMA pipe
+ * for part of each softmax row (range reduction to [-1/2, 1/2] plus a degree-3
+ * minimax polynomial; inputs <= -127 give exactly 0).  Writes it to y_poly and the
+ * hardware ex2.approx to y_mufu for the n device floats x[].  Diagnostic only. */
+bca_status bca_selftest_exp2(const float* x, float* y_poly, float* y_mufu, int32_t n,
+                             void* stream);
+
+/* Pipeline tracing (diagnostic; builds compiled with BCA_TRACE only, otherwise
+ * BCA_ERR_UNSUPPORTED): attention launches enqueued afterwards record clock64()
+ * stamps of CTA `cta`'s producer/MMA/softmax events into dev_buffer
+  * ([64 tiles][32 events] uint64, device, caller-owned); NULL turns it off. */
+bca_status bca_debug_set_trace(unsigned long long* dev_buffer, int32_t cta);
+
 /* Library version string. */
 const char* bca_version(void);
 

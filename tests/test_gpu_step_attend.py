@@ -127,3 +127,98 @@ def test_repeated_calls_are_deterministic(cuda_device):
     a, _ = run_batch([req], 2, cuda_device)
     b, _ = run_batch([req], 2, cuda_device)
     assert torch.equal(a, b)
+
+
+# ---------------------------------------------------------------------------
+# e4m3 prefix cache ("Prefix KV cache": "fp8_v" quantises V, "fp8" K and V).
+# Compared with the oracle reading the same cache bytes: rel-L2 <= 2e-2.
+# ---------------------------------------------------------------------------
+from _parity import REL_L2_FP8  # noqa: E402
+
+
+@pytest.mark.parametrize("mode", ["fp8", "fp8_v"])
+@pytest.mark.parametrize("T,P,H", [(256, 128, 4), (300, 129, 2), (77, 1000, 2), (129, 0, 2),
+                                   (1, 5, 1)])
+def test_fp8_cache_single_request(cuda_device, mode, T, P, H):
+    req = make_request(T, P, H, seed=3 * T + P, device=cuda_device, cap=P + 11, mode=mode)
+    o, _ = run_batch([req], H, cuda_device)
+    assert_parity(o, oracle_for(req), rel_l2=REL_L2_FP8, what=f"{mode} T={T} P={P}")
+
+
+@pytest.mark.parametrize("mode", ["fp8", "fp8_v"])
+def test_fp8_cache_ragged_batch(cuda_device, mode):
+    H = 2
+    shapes = [(300, 513), (77, 0), (256, 1), (130, 2000)]
+    reqs = [make_request(T, P, H, seed=200 + i, device=cuda_device, cap=P + 3, mode=mode)
+            for i, (T, P) in enumerate(shapes)]
+    o, cu = run_batch(reqs, H, cuda_device)
+    for i, r in enumerate(reqs):
+        assert_parity(o[cu[i]:cu[i + 1]], oracle_for(r), rel_l2=REL_L2_FP8, what=f"req {i}")
+
+
+def test_prefill_into_fp8_slot_then_cached_step(cuda_device):
+    H, blocks = 2, [100, 333, 200]
+    S, P = sum(blocks), sum(blocks[:-1])
+    q, k, v = (randn_bf16((S, H, 128), 300 + t, cuda_device) for t in range(3))
+    o = torch.empty_like(q)
+    slot = bca.KVSlot(P, H, "fp8")
+    bca.prefill(q, k, v, o, [0, 100, 433, S], SCALE, slot=slot, epoch=4)
+    torch.cuda.synchronize()
+    kc, ks = oracle.quantize_prefix(k.cpu(), P)
+    vc, vs = oracle.quantize_prefix(v.cpu(), P)
+    assert np.array_equal(slot.k_view().cpu().numpy(), kc)
+    assert np.array_equal(slot.v_view().cpu().numpy(), vc)
+    assert np.array_equal(slot.k_scale_view().cpu().numpy(), ks)
+    assert np.array_equal(slot.v_scale_view().cpu().numpy(), vs)
+    qt, kt, vt = q[P:], k[P:], v[P:]
+    ot = torch.empty_like(qt)
+    bca.step_attend(qt, kt, vt, ot, [0, S - P], [slot], SCALE)
+    torch.cuda.synchronize()
+    want = oracle.cached_step(qt, kt, vt, kc, vc, P, SCALE, k_kind=oracle.KIND_E4M3,
+                              v_kind=oracle.KIND_E4M3, k_scale=ks, v_scale=vs)
+    assert_parity(ot, want, rel_l2=REL_L2_FP8, what="fp8 slot from prefill")
+
+
+def test_serving_batch_sampled_rows(cuda_device):
+    """The step-batched serving workload: 8 requests with ragged prefixes (77..~17k
+    tokens), target 4096 each, H=32, e4m3 K and V cache; sampled target rows of
+    every request x all heads."""
+    wl = W.workload(4)
+    slots, qs, ks_, vs_ = [], [], [], []
+    for i, r in enumerate(wl.requests):
+        q0, k0, v0 = W.qkv(wl, 0, 0, i, cuda_device)
+        slot = bca.KVSlot(r.prefix, wl.heads, "fp8")
+        bca.prefill(q0, k0, v0, torch.empty_like(q0), r.offsets, wl.scale, slot=slot, epoch=1)
+        slots.append(slot)
+        del q0, k0, v0
+        q, k, v = W.qkv(wl, 0, 1, i, cuda_device)
+        qs.append(q), ks_.append(k), vs_.append(v)
+    q, k, v = torch.cat(qs), torch.cat(ks_), torch.cat(vs_)
+    o = torch.empty_like(q)
+    cu = np.concatenate([[0], np.cumsum([r.target for r in wl.requests])])
+    bca.step_attend(q, k, v, o, cu, slots, wl.scale)
+    torch.cuda.synchronize()
+    for i, r in enumerate(wl.requests):
+        rows = sample_rows(r.target, 12, seed=i, boundaries=(128, 256, 2048))
+        s = slots[i]
+        want = oracle.cached_step(qs[i], ks_[i], vs_[i], s.k_view().cpu(), s.v_view().cpu(),
+                                  r.prefix, wl.scale, k_kind=oracle.KIND_E4M3,
+                                  v_kind=oracle.KIND_E4M3,
+                                  k_scale=s.k_scale_view().cpu().numpy(),
+                                  v_scale=s.v_scale_view().cpu().numpy(), rows=rows)
+        got = o[cu[i]:cu[i + 1]][torch.from_numpy(rows).to(cuda_device)]
+        assert_parity(got, want, rel_l2=REL_L2_FP8, what=f"serving request {i}")
+
+
+@pytest.mark.parametrize("mode", ["fp8", "fp8_v", "bf16"])
+def test_repeated_batches_are_bitwise_identical(cuda_device, mode):
+    """Races between the producer, converter, MMA and softmax roles would show up as
+    run-to-run differences; the kernel is deterministic, so outputs must repeat."""
+    H = 4
+    shapes = [(512, 3000), (300, 129), (1024, 2500)]
+    reqs = [make_request(T, P, H, seed=400 + i, device=cuda_device, cap=P, mode=mode)
+            for i, (T, P) in enumerate(shapes)]
+    first, _ = run_batch(reqs, H, cuda_device)
+    for _ in range(4):
+        again, _ = run_batch(reqs, H, cuda_device)
+        assert torch.equal(first, again)
