@@ -163,6 +163,7 @@ class Runner:
                    for i, r in enumerate(reqs)]
             self.pool.append(tuple(torch.cat([x[j] for x in per]) for j in range(3)))
         self.o_step = torch.empty_like(self.pool[0][0])
+        self.workspace = bca.step_workspace(device)
         self.status = torch.zeros(1, dtype=torch.int32, device=device)
         self.epoch = 0
         self.flops_prefill = sum(prefill_flops(r, H) for r in reqs) * layers
@@ -171,7 +172,16 @@ class Runner:
         self.flops = self.flops_prefill + self.flops_steps
         kv_store_launches = 1 if wl.kv_dtype == "bf16" else 4
         self.launches_per_step = (layers * len(reqs) * (1 + kv_store_launches)
-                                  + layers * (wl.steps - 1))
+                                  + layers * (wl.steps - 1) * (1 + self.split_launches()))
+
+    def split_launches(self) -> int:
+        """1 if cached steps also launch the chunk-merge kernel (the last partial
+        round of units is split along the keys), else 0 -- mirrors the library's
+        schedule: units = sum_r H * ceil(T_r / 256) over the SMs."""
+        import torch
+        sms = torch.cuda.get_device_properties(self.device).multi_processor_count
+        units = sum(self.H * -(-r.target // 256) for r in self.wl.requests)
+        return int(units > sms and units % sms != 0 and sms // (units % sms) >= 2)
 
     def step(self, events=None):
         """One pass of the hot path.  events: optional list collecting
@@ -194,7 +204,7 @@ class Runner:
                         e1 = torch.cuda.Event(enable_timing=True)
                         e0.record()
                     bca.step_attend(q, k, v, self.o_step, self.cu, self.slots[l], wl.scale,
-                                    dev_status=self.status)
+                                    workspace=self.workspace, dev_status=self.status)
                     if events is not None:
                         e1.record()
                         events.append((e0, e1))
@@ -246,7 +256,7 @@ class E2ERunner:
                     k.copy_(hk, non_blocking=True)
                     v.copy_(hv, non_blocking=True)
                     bca.step_attend(q, k, v, r.o_step, r.cu, r.slots[l], wl.scale,
-                                    dev_status=r.status)
+                                    workspace=r.workspace, dev_status=r.status)
                     self.h_out_step.copy_(r.o_step, non_blocking=True)
 
 

@@ -24,7 +24,8 @@ import os
 
 __all__ = [
     "BcaError", "KVSlot", "KV_BF16", "KV_FP8_V", "KV_FP8_KV", "MAX_BLOCKS", "MAX_BATCH",
-    "lib", "prefill", "kv_store", "step_attend", "slot_bytes", "set_wait_timeout_ns",
+    "lib", "prefill", "kv_store", "step_attend", "step_workspace", "step_workspace_bytes",
+    "slot_bytes", "set_wait_timeout_ns",
     "selftest_wait_timeout", "selftest_exp2", "status_string", "version", "LIB_PATH",
 ]
 
@@ -86,7 +87,10 @@ def lib():
     L.bca_prefill.restype = ctypes.c_int
     L.bca_prefill.argtypes = [P, P, P, P, i32, P, i32, i32, i32, f32, SP, u32, P, P]
     L.bca_step_attend.restype = ctypes.c_int
-    L.bca_step_attend.argtypes = [P, P, P, P, P, SP, i32, i32, i32, f32, P, P]
+    L.bca_step_attend.argtypes = [P, P, P, P, P, SP, i32, i32, i32, f32, P, ctypes.c_size_t,
+                                  P, P]
+    L.bca_step_workspace_bytes.restype = ctypes.c_size_t
+    L.bca_step_workspace_bytes.argtypes = []
     L.bca_status_string.restype = ctypes.c_char_p
     L.bca_status_string.argtypes = [ctypes.c_int]
     L.bca_set_wait_timeout_ns.restype = None
@@ -224,14 +228,26 @@ def prefill(q, k, v, o, block_offsets, scale: float, slot: KVSlot | None = None,
            "bca_prefill")
 
 
-def step_attend(q_t, k_t, v_t, o_t, cu_target, slots, scale: float, dev_status=None,
-                stream=None):
+def step_workspace_bytes() -> int:
+    return int(lib().bca_step_workspace_bytes())
+
+
+def step_workspace(device="cuda"):
+    """A workspace for step_attend (uint8 CUDA tensor of step_workspace_bytes())."""
+    import torch
+    return torch.empty(max(step_workspace_bytes(), 256), dtype=torch.uint8, device=device)
+
+
+def step_attend(q_t, k_t, v_t, o_t, cu_target, slots, scale: float, workspace=None,
+                dev_status=None, stream=None):
     _, H, d = q_t.shape
     cu = _i32_array(cu_target)
     arr = (SlotStruct * len(slots))(*[s.struct for s in slots])
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check(lib().bca_step_attend(_ptr(q_t), _ptr(k_t), _ptr(v_t), _ptr(o_t), cu, arr,
-                                 len(slots), H, d, float(scale), _ptr(dev_status),
-                                 _stream(stream, q_t.device)), "bca_step_attend")
+                                 len(slots), H, d, float(scale), _ptr(workspace), ws_bytes,
+                                 _ptr(dev_status), _stream(stream, q_t.device)),
+           "bca_step_attend")
 
 
 def selftest_wait_timeout(dev_status, timeout_ns: int, stream=None):

@@ -10,11 +10,18 @@
 //    prefix K/V followed by their own K/V.  Step mode computes this for a ragged
 //    batch of requests at the same phase ("Online serving": step-level batching).
 //
-// Design (B200): one CTA owns a (request, head, pair of 128-row Q tiles) unit.
-//  * warp 8      : TMA producer -- Q tiles once, then K_j, V_j tiles into a
+// Design (B200).  A unit is (request, head, pair of 128-row Q tiles).  The kernel
+// is persistent: one CTA per SM walks a static list of work items (item = CTA
+// index + k * grid).  Items of the first rounds are whole units; the units of the
+// last, partial round are split along the key dimension into `split_k` chunks so
+// that every SM ends at about the same time -- a chunk writes its unnormalised O,
+// row max and row sum to a workspace and attn_combine_kernel merges the chunks.
+//  * warp 8      : TMA producer -- Q tiles of each item, then K_j, V_j tiles into a
 //                  4-stage ring of 32 KiB bf16 tiles (128-byte swizzle).
-//  * warp 9      : tcgen05 issuer -- S_w = Q_w K_j^T (both operands in smem) and
-//                  O_w += P_w V_j (P from TMEM, V in smem, MN-major), fp32 in TMEM.
+//  * warp 9      : tcgen05 issuer (whole warp, one elected lane issues) --
+//                  S_w = Q_w K_j^T (both operands in smem) and O_w += P_w V_j (P from
+//                  TMEM, V in smem, MN-major), fp32 accumulators in TMEM.
+//  * warps 10-11 : e4m3 cache tiles -> bf16 in shared memory (FP8 cache only).
 //  * warps 0..3  : softmax of Q tile 0, warps 4..7: Q tile 1.  One thread per row:
 //                  load S from TMEM, mask ragged / block-causal keys, online softmax
 //                  in the exp2 domain, write P (bf16) back over S in TMEM.  O is
@@ -47,32 +54,36 @@ constexpr int kWarpConv0 = 10;  // warps 10 and 11 convert e4m3 cache tiles
 constexpr int kConvThreads = 64;
 // Register split: launched at kLaunchRegs per thread (384 x 168 = 64512), the two
 // softmax warpgroups take kSoftmaxRegs and warpgroup 2 (producer, MMA, converter)
-// keeps kOtherRegs: 128 * (2 * 216 + 72) = 64512.  The host checks the compiled
+// keeps kOtherRegs: 128 * (2 * 208 + 88) = 64512.  The host checks the compiled
 // register count against this before launching.
 constexpr uint32_t kLaunchRegs = 168;
-constexpr uint32_t kSoftmaxRegs = 216;
-constexpr uint32_t kOtherRegs = 72;
+constexpr uint32_t kSoftmaxRegs = 208;
+constexpr uint32_t kOtherRegs = 88;
 static_assert(128 * (2 * kSoftmaxRegs + kOtherRegs) <= kAttnThreads * kLaunchRegs,
               "register split exceeds the launch allocation");
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
-constexpr int kPolyPairs = 3;  // of every 8 column pairs, exponentiated on the FMA pipe
+constexpr int kPolyPairs = 2;  // of every 8 column pairs, exponentiated on the FMA pipe
 constexpr int kNoLimit = 1 << 30;
+// Split-chunk workspace: per chunk, O [256 rows][128] fp32, then m[256], l[256].
+constexpr int kChunkRows = 2 * kBM;
+constexpr size_t kChunkBytes = static_cast<size_t>(kChunkRows) * (kHeadDim + 2) * 4;
 
 enum : int { kModePrefill = 0, kModeStep = 1 };
 
 // Pipeline trace of one CTA (builds with BCA_TRACE only): clock64() stamps of the
-// roles' events per KV tile, trace[j * kTraceEvents + event], for j < kTraceTiles.
+// roles' events per KV tile t, counted over all items of the CTA,
+// trace[t * kTraceEvents + ev].
 constexpr int kTraceEvents = 32;
-constexpr int kTraceTiles = 64;
+constexpr int kTraceTiles = 192;
 #ifdef BCA_TRACE
-#define BCA_TRACE_AT(p, j, ev)                                                          \
+#define BCA_TRACE_AT(p, t, ev)                                                          \
   do {                                                                                  \
-    if ((p).trace && static_cast<int>(blockIdx.x) == (p).trace_cta && (j) < kTraceTiles && \
-        (j) >= 0)                                                                       \
-      (p).trace[(j) * kTraceEvents + (ev)] = clock64();                                 \
+    if ((p).trace && static_cast<int>(blockIdx.x) == (p).trace_cta && (t) < kTraceTiles && \
+        (t) >= 0)                                                                       \
+      (p).trace[(t) * kTraceEvents + (ev)] = clock64();                                 \
   } while (0)
 #else
-#define BCA_TRACE_AT(p, j, ev) \
+#define BCA_TRACE_AT(p, t, ev) \
   do {                         \
   } while (0)
 #endif
@@ -94,6 +105,13 @@ struct AttnParams {
   int32_t heads;
   int32_t mode;
   float scale_log2;  // softmax scale * log2(e)
+  // work items: [0, full_items) are whole units; the next units are split into
+  // split_k chunks each (chunk c of a unit with n tiles covers tiles
+  // [c*n/k, (c+1)*n/k)), written to `workspace` and merged by attn_combine_kernel.
+  int32_t n_items;
+  int32_t full_items;
+  int32_t split_k;
+  float* workspace;
   // prefill
   int32_t seq_len;
   int32_t n_blocks;
@@ -120,17 +138,18 @@ struct Smem {
   static constexpr int kStage8 = kRing + kStages * kTileBytes;  // 2 x 16 KiB e4m3 tiles
   static constexpr int kBars = kStage8 + 2 * kTile8Bytes;
   // barrier indices
-  static constexpr int bQFull = 0;                 // 2
-  static constexpr int bKvFull = 2;                // kStages
-  static constexpr int bKvEmpty = 2 + kStages;     // kStages
-  static constexpr int bSFull = 2 + 2 * kStages;   // 2
-  static constexpr int bPFull = 4 + 2 * kStages;   // 2
-  static constexpr int bOFull = 6 + 2 * kStages;   // 2
-  static constexpr int bDone = 8 + 2 * kStages;    // 1
-  static constexpr int bStgFull = 9 + 2 * kStages;   // 2
-  static constexpr int bStgEmpty = 11 + 2 * kStages; // 2
-  static constexpr int bConv = 13 + 2 * kStages;     // 1 (64 converter arrivals per tile)
-  static constexpr int kNumBars = 14 + 2 * kStages;
+  static constexpr int bQFull = 0;                     // 2
+  static constexpr int bKvFull = 2;                    // kStages
+  static constexpr int bKvEmpty = 2 + kStages;         // kStages
+  static constexpr int bSFull = 2 + 2 * kStages;       // 2
+  static constexpr int bPFull = 4 + 2 * kStages;       // 2
+  static constexpr int bOFull = 6 + 2 * kStages;       // 2
+  static constexpr int bDone = 8 + 2 * kStages;        // 1
+  static constexpr int bStgFull = 9 + 2 * kStages;     // 2
+  static constexpr int bStgEmpty = 11 + 2 * kStages;   // 2
+  static constexpr int bConv = 13 + 2 * kStages;       // 1 (64 converter arrivals per tile)
+  static constexpr int bQEmpty = 14 + 2 * kStages;     // 1 (Q tiles of an item consumed)
+  static constexpr int kNumBars = 15 + 2 * kStages;
   static constexpr int kTmemSlot = kBars + 8 * kNumBars;
   static constexpr int kAbort = kTmemSlot + 4;
   static constexpr int kBytes = kAbort + 4;
@@ -141,14 +160,19 @@ struct Smem {
 __host__ __device__ constexpr uint32_t col_s(int w) { return w == 0 ? 0u : 128u; }
 __host__ __device__ constexpr uint32_t col_o(int w) { return w == 0 ? 256u : 384u; }
 
-struct Unit {
+// One work item with every per-unit value it needs held in registers.
+struct Item {
   int req;        // request slot in the params arrays (step mode)
   int h;          // head
   int q_row0;     // row of Q tile 0 in the Q/O tensors
   int rows[2];    // valid rows of each Q tile (<= 0: tile absent)
-  int ntiles[2];  // KV tiles each Q tile visits
-  int n_total;    // max(ntiles)
+  int jend[2];    // Q tile w visits KV tiles [j0, jend[w]) (jend <= j0: inactive)
+  int j0, j1;     // KV tile range of the item (j1 = max(jend))
+  int n_cache;    // cached keys (step mode)
   int n_cache_tiles;
+  int q_start;    // first packed row of the request (step mode)
+  int q_len;      // target rows of the request (step mode)
+  int partial;    // -1: whole unit; else workspace chunk index
 };
 
 template <int MAXR>
@@ -159,23 +183,36 @@ __device__ __forceinline__ int block_end(const AttnParams<MAXR>& p, int row) {
 }
 
 template <int MAXR>
-__device__ __forceinline__ Unit decode_unit(const AttnParams<MAXR>& p, int unit) {
-  Unit u;
+__device__ __forceinline__ Item decode_item(const AttnParams<MAXR>& p, int item) {
+  Item it;
+  int unit = item, chunk = 0, k = 1;
+  it.partial = -1;
+  if (item >= p.full_items) {
+    k = p.split_k;
+    const int q = item - p.full_items;
+    unit = p.full_items + q / k;
+    chunk = q % k;
+    it.partial = q;
+  }
+  int ntiles[2];
   if (p.mode == kModePrefill) {
     const int S = p.seq_len;
     const int nqp = (S + 2 * kBM - 1) / (2 * kBM);
-    u.req = 0;
-    u.h = unit / nqp;
+    it.req = 0;
+    it.h = unit / nqp;
     const int qp = nqp - 1 - unit % nqp;  // heaviest (latest) rows first within a head
-    u.q_row0 = qp * 2 * kBM;
-    u.n_cache_tiles = 0;
+    it.q_row0 = qp * 2 * kBM;
+    it.n_cache = 0;
+    it.n_cache_tiles = 0;
+    it.q_start = 0;
+    it.q_len = S;
 #pragma unroll
     for (int w = 0; w < 2; ++w) {
-      u.rows[w] = min(kBM, S - u.q_row0 - w * kBM);
-      u.ntiles[w] = 0;
-      if (u.rows[w] > 0) {
-        const int lim = block_end(p, u.q_row0 + w * kBM + u.rows[w] - 1);
-        u.ntiles[w] = (lim + kBN - 1) / kBN;
+      it.rows[w] = min(kBM, S - it.q_row0 - w * kBM);
+      ntiles[w] = 0;
+      if (it.rows[w] > 0) {
+        const int lim = block_end(p, it.q_row0 + w * kBM + it.rows[w] - 1);
+        ntiles[w] = (lim + kBN - 1) / kBN;
       }
     }
   } else {
@@ -184,37 +221,47 @@ __device__ __forceinline__ Unit decode_unit(const AttnParams<MAXR>& p, int unit)
     const int T = p.q_len[r];
     const int nqp = (T + 2 * kBM - 1) / (2 * kBM);
     const int local = unit - p.unit_start[r];
-    u.req = r;
-    u.h = local / nqp;
+    it.req = r;
+    it.h = local / nqp;
     const int qp = local % nqp;
-    u.q_row0 = p.q_start[r] + qp * 2 * kBM;
-    u.n_cache_tiles = (p.n_cache[r] + kBN - 1) / kBN;
-    const int nt = u.n_cache_tiles + (T + kBN - 1) / kBN;
+    it.q_start = p.q_start[r];
+    it.q_len = T;
+    it.q_row0 = it.q_start + qp * 2 * kBM;
+    it.n_cache = p.n_cache[r];
+    it.n_cache_tiles = (it.n_cache + kBN - 1) / kBN;
+    const int nt = it.n_cache_tiles + (T + kBN - 1) / kBN;
 #pragma unroll
     for (int w = 0; w < 2; ++w) {
-      u.rows[w] = min(kBM, T - qp * 2 * kBM - w * kBM);
-      u.ntiles[w] = u.rows[w] > 0 ? nt : 0;
+      it.rows[w] = min(kBM, T - qp * 2 * kBM - w * kBM);
+      ntiles[w] = it.rows[w] > 0 ? nt : 0;
     }
   }
-  u.n_total = max(u.ntiles[0], u.ntiles[1]);
-  return u;
+  const int n = max(ntiles[0], ntiles[1]);
+  it.j0 = chunk * n / k;
+  it.j1 = (chunk + 1) * n / k;
+#pragma unroll
+  for (int w = 0; w < 2; ++w) it.jend[w] = min(it.j1, ntiles[w]);
+  return it;
 }
 
-// Geometry of KV tile j of a unit: number of valid keys and index of its first
-// key in the row's key sequence (for the block-causal limit).
-template <int MAXR>
-__device__ __forceinline__ void kv_tile_extent(const AttnParams<MAXR>& p, const Unit& u, int j,
+__device__ __forceinline__ bool tile_active(const Item& it, int w) {
+  return (w ? it.rows[1] : it.rows[0]) > 0 && it.j0 < (w ? it.jend[1] : it.jend[0]);
+}
+
+// Geometry of KV tile j: number of valid keys and index of its first key in the
+// row's key sequence (for the block-causal limit).  Registers only.
+__device__ __forceinline__ void kv_tile_extent(bool prefill, const Item& it, int seq_len, int j,
                                                int& valid, int& key_base) {
-  if (p.mode == kModePrefill) {
+  if (prefill) {
     key_base = j * kBN;
-    valid = min(kBN, p.seq_len - key_base);
-  } else if (j < u.n_cache_tiles) {
+    valid = min(kBN, seq_len - key_base);
+  } else if (j < it.n_cache_tiles) {
     key_base = j * kBN;
-    valid = min(kBN, p.n_cache[u.req] - key_base);
+    valid = min(kBN, it.n_cache - key_base);
   } else {
-    const int jj = j - u.n_cache_tiles;
-    key_base = p.n_cache[u.req] + jj * kBN;
-    valid = min(kBN, p.q_len[u.req] - jj * kBN);
+    const int jj = j - it.n_cache_tiles;
+    key_base = it.n_cache + jj * kBN;
+    valid = min(kBN, it.q_len - jj * kBN);
   }
 }
 
@@ -235,80 +282,91 @@ __device__ __forceinline__ void raise_abort(volatile int* abort, int32_t* dev_st
 // Self-checks of checked builds: a failed check records 2000 + code and the caller
 // skips the access.  Compiled out otherwise.
 #ifdef BCA_DEVICE_CHECKS
-#define BCA_CHECK(dev_status, cond, code)                                        \
+#define BCA_CHECK(dev_status, cond, code) \
   ((cond) ? true : ((dev_status) ? (atomicCAS((dev_status), 0, 2000 + (code)), false) : false))
 #else
 #define BCA_CHECK(dev_status, cond, code) true
 #endif
 
+template <int MAXR>
+__device__ __forceinline__ bool tile_is_fp8(const AttnParams<MAXR>& p, const Item& it, int j,
+                                            int kv) {
+  return p.mode == kModeStep && j < it.n_cache_tiles && (kv ? p.v_fp8 : p.k_fp8) != 0;
+}
+
 // ---------------------------------------------------------------------------
 // Producer: one thread.
 // ---------------------------------------------------------------------------
 template <int MAXR>
-__device__ __forceinline__ bool tile_is_fp8(const AttnParams<MAXR>& p, const Unit& u, int j,
-                                            int kv) {
-  return p.mode == kModeStep && j < u.n_cache_tiles && (kv ? p.v_fp8 : p.k_fp8) != 0;
-}
-
-template <int MAXR>
-__device__ void producer_role(const AttnParams<MAXR>& p, const Unit& u, uint32_t sbase,
-                              uint32_t bars, volatile int* abort) {
+__device__ void producer_role(const AttnParams<MAXR>& p, uint32_t sbase, uint32_t bars,
+                              volatile int* abort) {
   auto bar = [&](int i) { return bars + 8u * static_cast<uint32_t>(i); };
-#pragma unroll
-  for (int w = 0; w < 2; ++w) {
-    if (u.rows[w] <= 0) continue;
-    const uint32_t dst = sbase + (w == 0 ? Smem::kQ0 : Smem::kQ1);
-    const int z = u.q_row0 + w * kBM;
-    mbar_arrive_expect_tx(bar(Smem::bQFull + w), kTileBytes);
-    tma_load_3d(dst, &p.tm_q, bar(Smem::bQFull + w), 0, u.h, z);
-    tma_load_3d(dst + kHalfBytes, &p.tm_q, bar(Smem::bQFull + w), 64, u.h, z);
-  }
-  int it = 0, fi = 0;  // item (K_0, V_0, K_1, ...) and e4m3 item counters
+  int it = 0, fi = 0, nq = 0;  // ring items, e4m3 items, items (Q loads) so far
   bool ok = true;
-  for (int j = 0; j < u.n_total && ok; ++j) {
-    for (int kv = 0; kv < 2; ++kv, ++it) {
-      if (tile_is_fp8(p, u, j, kv)) {
-        // e4m3 cache tile -> staging buffer; the converter warps fill the ring slot.
-        const int ss = fi & 1;
-        const uint32_t ph = static_cast<uint32_t>(fi >> 1) & 1u;
-        if (!mbar_wait_bounded(bar(Smem::bStgEmpty + ss), ph ^ 1u, abort, p.timeout_ns)) {
-          raise_abort(abort, p.dev_status, 11);
+  for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x, ++nq) {
+    const Item c = decode_item(p, item);
+    // Both Q tiles are always loaded (rows past the tensor read as zero), so every
+    // item completes one phase of each Q barrier.
+    if (!mbar_wait_bounded(bar(Smem::bQEmpty), (static_cast<uint32_t>(nq) & 1u) ^ 1u, abort,
+                           p.timeout_ns)) {
+      raise_abort(abort, p.dev_status, 10);
+      ok = false;
+      break;
+    }
+    BCA_TRACE_AT(p, it / 2, 27);
+#pragma unroll
+    for (int w = 0; w < 2; ++w) {
+      const uint32_t dst = sbase + (w == 0 ? Smem::kQ0 : Smem::kQ1);
+      const int z = c.q_row0 + w * kBM;
+      mbar_arrive_expect_tx(bar(Smem::bQFull + w), kTileBytes);
+      tma_load_3d(dst, &p.tm_q, bar(Smem::bQFull + w), 0, c.h, z);
+      tma_load_3d(dst + kHalfBytes, &p.tm_q, bar(Smem::bQFull + w), 64, c.h, z);
+    }
+    for (int j = c.j0; j < c.j1 && ok; ++j) {
+      for (int kv = 0; kv < 2; ++kv, ++it) {
+        if (tile_is_fp8(p, c, j, kv)) {
+          // e4m3 cache tile -> staging buffer; the converter warps fill the ring slot.
+          const int ss = fi & 1;
+          const uint32_t ph = static_cast<uint32_t>(fi >> 1) & 1u;
+          if (!mbar_wait_bounded(bar(Smem::bStgEmpty + ss), ph ^ 1u, abort, p.timeout_ns)) {
+            raise_abort(abort, p.dev_status, 11);
+            ok = false;
+            break;
+          }
+          const uint32_t fb = bar(Smem::bStgFull + ss);
+          mbar_arrive_expect_tx(fb, kTile8Bytes);
+          if (BCA_CHECK(p.dev_status, c.req < p.n_req && j * kBN < c.n_cache && c.h < p.heads, 1))
+            tma_load_3d(sbase + Smem::kStage8 + ss * kTile8Bytes,
+                        kv ? &p.tm_vc[c.req] : &p.tm_kc[c.req], fb, 0, j * kBN, c.h);
+          ++fi;
+          continue;
+        }
+        const int st = it % kStages;
+        const uint32_t ph = static_cast<uint32_t>(it / kStages) & 1u;
+        if (!mbar_wait_bounded(bar(Smem::bKvEmpty + st), ph ^ 1u, abort, p.timeout_ns)) {
+          raise_abort(abort, p.dev_status, 12);
           ok = false;
           break;
         }
-        const uint32_t fb = bar(Smem::bStgFull + ss);
-        mbar_arrive_expect_tx(fb, kTile8Bytes);
-        if (BCA_CHECK(p.dev_status, u.req < p.n_req && j * kBN < p.n_cache[u.req] && u.h < p.heads, 1))
-          tma_load_3d(sbase + Smem::kStage8 + ss * kTile8Bytes,
-                      kv ? &p.tm_vc[u.req] : &p.tm_kc[u.req], fb, 0, j * kBN, u.h);
-        ++fi;
-        continue;
-      }
-      const int st = it % kStages;
-      const uint32_t ph = static_cast<uint32_t>(it / kStages) & 1u;
-      if (!mbar_wait_bounded(bar(Smem::bKvEmpty + st), ph ^ 1u, abort, p.timeout_ns)) {
-        raise_abort(abort, p.dev_status, 12);
-        ok = false;
-        break;
-      }
-      const uint32_t dst = sbase + Smem::kRing + st * kTileBytes;
-      const uint32_t fb = bar(Smem::bKvFull + st);
-      BCA_TRACE_AT(p, j, 23 + kv);
-      mbar_arrive_expect_tx(fb, kTileBytes);
-      if (p.mode == kModeStep && j < u.n_cache_tiles) {
-        const CUtensorMap* m = kv ? &p.tm_vc[u.req] : &p.tm_kc[u.req];
-        tma_load_3d(dst, m, fb, 0, j * kBN, u.h);
-        tma_load_3d(dst + kHalfBytes, m, fb, 64, j * kBN, u.h);
-      } else {
-        const CUtensorMap* m = kv ? &p.tm_v : &p.tm_k;
-        const int z = p.mode == kModePrefill ? j * kBN
-                                             : p.q_start[u.req] + (j - u.n_cache_tiles) * kBN;
-        tma_load_3d(dst, m, fb, 0, u.h, z);
-        tma_load_3d(dst + kHalfBytes, m, fb, 64, u.h, z);
+        const uint32_t dst = sbase + Smem::kRing + st * kTileBytes;
+        const uint32_t fb = bar(Smem::bKvFull + st);
+        BCA_TRACE_AT(p, it / 2, 23 + kv);
+        mbar_arrive_expect_tx(fb, kTileBytes);
+        if (p.mode == kModeStep && j < c.n_cache_tiles) {
+          const CUtensorMap* m = kv ? &p.tm_vc[c.req] : &p.tm_kc[c.req];
+          tma_load_3d(dst, m, fb, 0, j * kBN, c.h);
+          tma_load_3d(dst + kHalfBytes, m, fb, 64, j * kBN, c.h);
+        } else {
+          const CUtensorMap* m = kv ? &p.tm_v : &p.tm_k;
+          const int z = p.mode == kModePrefill ? j * kBN
+                                               : c.q_start + (j - c.n_cache_tiles) * kBN;
+          tma_load_3d(dst, m, fb, 0, c.h, z);
+          tma_load_3d(dst + kHalfBytes, m, fb, 64, c.h, z);
+        }
       }
     }
   }
-  if (!ok) {
+  if (!ok || *abort) {
     // Drain: wait (time-bounded only) for copies this thread may still have in flight.
     constexpr unsigned long long kDrainNs = 20000000ull;
     for (int i = max(0, it - kStages); i < it; ++i)
@@ -317,6 +375,10 @@ __device__ void producer_role(const AttnParams<MAXR>& p, const Unit& u, uint32_t
     for (int i = max(0, fi - 2); i < fi; ++i)
       mbar_wait_bounded(bar(Smem::bStgFull + (i & 1)), static_cast<uint32_t>(i >> 1) & 1u, nullptr,
                         kDrainNs);
+    if (nq > 0)
+      for (int w = 0; w < 2; ++w)
+        mbar_wait_bounded(bar(Smem::bQFull + w), static_cast<uint32_t>(nq - 1) & 1u, nullptr,
+                          kDrainNs);
   }
 }
 
@@ -334,79 +396,80 @@ __device__ __forceinline__ uint32_t e4m3x2_to_bf16x2(uint32_t two) {
 }
 
 template <int MAXR>
-__device__ void converter_role(const AttnParams<MAXR>& p, const Unit& u, uint32_t sbase,
-                               uint32_t bars, volatile int* abort) {
+__device__ void converter_role(const AttnParams<MAXR>& p, uint32_t sbase, uint32_t bars,
+                               volatile int* abort) {
   auto bar = [&](int i) { return bars + 8u * static_cast<uint32_t>(i); };
   const int c = threadIdx.x - kWarpConv0 * 32;  // 0..63
   int it = 0, fi = 0;
-  for (int j = 0; j < u.n_cache_tiles && j < u.n_total; ++j) {
-    for (int kv = 0; kv < 2; ++kv, ++it) {
-      if (!tile_is_fp8(p, u, j, kv)) continue;
-      const int ss = fi & 1;
-      const int st = it % kStages;
-      const bool got =
-          mbar_wait_bounded(bar(Smem::bStgFull + ss), static_cast<uint32_t>(fi >> 1) & 1u, abort,
-                            p.timeout_ns) &&
-          mbar_wait_bounded(bar(Smem::bKvEmpty + st),
-                            (static_cast<uint32_t>(it / kStages) & 1u) ^ 1u, abort, p.timeout_ns);
-      if (!got) {
-        raise_abort(abort, p.dev_status, 21);
-        return;
-      }
-      const uint32_t src = sbase + Smem::kStage8 + ss * kTile8Bytes;
-      const uint32_t dst = sbase + Smem::kRing + st * kTileBytes;
+  for (int item = blockIdx.x; item < p.n_items; item += gridDim.x) {
+    const Item ci = decode_item(p, item);
+    for (int j = ci.j0; j < ci.j1; ++j) {
+      for (int kv = 0; kv < 2; ++kv, ++it) {
+        if (!tile_is_fp8(p, ci, j, kv)) continue;
+        const int ss = fi & 1;
+        const int st = it % kStages;
+        const bool got =
+            mbar_wait_bounded(bar(Smem::bStgFull + ss), static_cast<uint32_t>(fi >> 1) & 1u,
+                              abort, p.timeout_ns) &&
+            mbar_wait_bounded(bar(Smem::bKvEmpty + st),
+                              (static_cast<uint32_t>(it / kStages) & 1u) ^ 1u, abort, p.timeout_ns);
+        if (!got) {
+          raise_abort(abort, p.dev_status, 21);
+          return;
+        }
+        const uint32_t src = sbase + Smem::kStage8 + ss * kTile8Bytes;
+        const uint32_t dst = sbase + Smem::kRing + st * kTileBytes;
 #pragma unroll 4
-      for (int k = 0; k < 16; ++k) {
-        const int gid = k * kConvThreads + c;
-        const int row = gid >> 3, ch = gid & 7;
-        if (!BCA_CHECK(p.dev_status, row < kBN && src + row * 128 + 128 <= sbase + Smem::kBars &&
-                                         dst + kTileBytes <= sbase + Smem::kStage8, 2))
-          continue;
-        uint32_t w0, w1, w2, w3;
-        asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
-                     : "=r"(w0), "=r"(w1), "=r"(w2), "=r"(w3)
-                     : "r"(src + row * 128 + ((ch ^ (row & 7)) << 4)));
-        const uint32_t o0 = e4m3x2_to_bf16x2(w0), o1 = e4m3x2_to_bf16x2(w0 >> 16);
-        const uint32_t o2 = e4m3x2_to_bf16x2(w1), o3 = e4m3x2_to_bf16x2(w1 >> 16);
-        const uint32_t o4 = e4m3x2_to_bf16x2(w2), o5 = e4m3x2_to_bf16x2(w2 >> 16);
-        const uint32_t o6 = e4m3x2_to_bf16x2(w3), o7 = e4m3x2_to_bf16x2(w3 >> 16);
-        const int k0 = 2 * (ch & 3);
-        const uint32_t base = dst + (ch >> 2) * kHalfBytes + row * 128;
-        asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(
-                         base + ((k0 ^ (row & 7)) << 4)),
-                     "r"(o0), "r"(o1), "r"(o2), "r"(o3)
-                     : "memory");
-        asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(
-                         base + (((k0 + 1) ^ (row & 7)) << 4)),
-                     "r"(o4), "r"(o5), "r"(o6), "r"(o7)
-                     : "memory");
+        for (int k = 0; k < 16; ++k) {
+          const int gid = k * kConvThreads + c;
+          const int row = gid >> 3, ch = gid & 7;
+          if (!BCA_CHECK(p.dev_status, row < kBN && src + row * 128 + 128 <= sbase + Smem::kBars &&
+                                           dst + kTileBytes <= sbase + Smem::kStage8, 2))
+            continue;
+          uint32_t w0, w1, w2, w3;
+          asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                       : "=r"(w0), "=r"(w1), "=r"(w2), "=r"(w3)
+                       : "r"(src + row * 128 + ((ch ^ (row & 7)) << 4)));
+          const uint32_t o0 = e4m3x2_to_bf16x2(w0), o1 = e4m3x2_to_bf16x2(w0 >> 16);
+          const uint32_t o2 = e4m3x2_to_bf16x2(w1), o3 = e4m3x2_to_bf16x2(w1 >> 16);
+          const uint32_t o4 = e4m3x2_to_bf16x2(w2), o5 = e4m3x2_to_bf16x2(w2 >> 16);
+          const uint32_t o6 = e4m3x2_to_bf16x2(w3), o7 = e4m3x2_to_bf16x2(w3 >> 16);
+          const int k0 = 2 * (ch & 3);
+          const uint32_t base = dst + (ch >> 2) * kHalfBytes + row * 128;
+          asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(
+                           base + ((k0 ^ (row & 7)) << 4)),
+                       "r"(o0), "r"(o1), "r"(o2), "r"(o3)
+                       : "memory");
+          asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(
+                           base + (((k0 + 1) ^ (row & 7)) << 4)),
+                       "r"(o4), "r"(o5), "r"(o6), "r"(o7)
+                       : "memory");
+        }
+        fence_proxy_async_smem();
+        mbar_arrive(bar(Smem::bConv));
+        // Every converter thread waits for the whole tile: none may run ahead and
+        // arrive for the next tile while this phase is still open.
+        if (!mbar_wait_bounded(bar(Smem::bConv), static_cast<uint32_t>(fi) & 1u, abort,
+                               p.timeout_ns)) {
+          raise_abort(abort, p.dev_status, 22);
+          return;
+        }
+        if (c == 0) {
+          mbar_arrive(bar(Smem::bKvFull + st));
+          mbar_arrive(bar(Smem::bStgEmpty + ss));
+        }
+        ++fi;
       }
-      fence_proxy_async_smem();
-      mbar_arrive(bar(Smem::bConv));
-      // Every converter thread waits for the whole tile: none may run ahead and
-      // arrive for the next tile while this phase is still open.
-      if (!mbar_wait_bounded(bar(Smem::bConv), static_cast<uint32_t>(fi) & 1u, abort,
-                             p.timeout_ns)) {
-        raise_abort(abort, p.dev_status, 22);
-        return;
-      }
-      if (c == 0) {
-        mbar_arrive(bar(Smem::bKvFull + st));
-        mbar_arrive(bar(Smem::bStgEmpty + ss));
-      }
-      ++fi;
     }
   }
 }
 
 // ---------------------------------------------------------------------------
-// MMA issuer: one thread.
+// MMA issuer: the whole warp (values stay warp-uniform); one elected lane issues.
 // ---------------------------------------------------------------------------
 template <int MAXR>
-__device__ void mma_role(const AttnParams<MAXR>& p, const Unit& u, uint32_t sbase, uint32_t bars,
-                         uint32_t tmem, volatile int* abort) {
-  // Executed by the whole warp so that every value below is warp-uniform (kept in
-  // uniform registers); one elected lane issues each tcgen05 instruction.
+__device__ void mma_role(const AttnParams<MAXR>& p, uint32_t sbase, uint32_t bars, uint32_t tmem,
+                         volatile int* abort) {
   auto bar = [&](int i) { return bars + 8u * static_cast<uint32_t>(i); };
   constexpr uint32_t kIdescS = idesc_bf16_f32(kBM, kBN, false);      // Q K^T: K-major B
   constexpr uint32_t kIdescO = idesc_bf16_f32(kBM, kHeadDim, true);  // P V: MN-major B
@@ -421,59 +484,74 @@ __device__ void mma_role(const AttnParams<MAXR>& p, const Unit& u, uint32_t sbas
     }
     return ok;
   };
-  for (int w = 0; w < 2; ++w)
-    if (u.rows[w] > 0) wait(Smem::bQFull + w, 0);
-  tc_fence_after();
   const uint64_t dq[2] = {sdesc_sw128(sbase + Smem::kQ0, 16, 1024),
                           sdesc_sw128(sbase + Smem::kQ1, 16, 1024)};
-  for (int j = 0; j <= u.n_total && ok; ++j) {
-    const int itK = 2 * j, itV = 2 * (j - 1) + 1;
-    const int stK = itK % kStages, stV = (itV + kStages) % kStages;
-    BCA_TRACE_AT(p, j, 21);
-    if (j < u.n_total) wait(Smem::bKvFull + stK, static_cast<uint32_t>(itK / kStages) & 1u);
-    BCA_TRACE_AT(p, j, 22);
-    if (j > 0) wait(Smem::bKvFull + stV, static_cast<uint32_t>(itV / kStages) & 1u);
+  int it = 0, nq = 0;   // ring items consumed, items
+  int npv[2] = {0, 0};  // P tiles consumed per Q tile (p_full phases)
+  for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x, ++nq) {
+    const Item c = decode_item(p, item);
+    const bool act0 = tile_active(c, 0), act1 = tile_active(c, 1);
+    wait(Smem::bQFull + 0, static_cast<uint32_t>(nq) & 1u);
+    wait(Smem::bQFull + 1, static_cast<uint32_t>(nq) & 1u);
     if (!ok) break;
-    BCA_TRACE_AT(p, j, 0);
     tc_fence_after();
-    const uint64_t dk = sdesc_sw128(sbase + Smem::kRing + stK * kTileBytes, 16, 1024);
-    const uint64_t dv = sdesc_sw128(sbase + Smem::kRing + stV * kTileBytes, kHalfBytes, 1024);
+    const int it0 = it;
+    BCA_TRACE_AT(p, it0 / 2, 26);
+    for (int j = c.j0; j <= c.j1 && ok; ++j) {
+      const int itK = it0 + 2 * (j - c.j0), itV = itK - 1;
+      const int stK = itK % kStages, stV = (itV + kStages) % kStages;
+      BCA_TRACE_AT(p, it0 / 2 + (j - c.j0), 21);
+      if (j < c.j1) wait(Smem::bKvFull + stK, static_cast<uint32_t>(itK / kStages) & 1u);
+      BCA_TRACE_AT(p, it0 / 2 + (j - c.j0), 22);
+      if (j > c.j0) wait(Smem::bKvFull + stV, static_cast<uint32_t>(itV / kStages) & 1u);
+      if (!ok) break;
+      BCA_TRACE_AT(p, it0 / 2 + (j - c.j0), 0);
+      tc_fence_after();
+      const uint64_t dk = sdesc_sw128(sbase + Smem::kRing + stK * kTileBytes, 16, 1024);
+      const uint64_t dv = sdesc_sw128(sbase + Smem::kRing + stV * kTileBytes, kHalfBytes, 1024);
 #pragma unroll
-    for (int w = 0; w < 2; ++w) {
-      if (j > 0 && j - 1 < u.ntiles[w]) {
-        // O_w += P_w(j-1) V_{j-1}; P must be consumed before S_w(j) overwrites it.
-        if (!wait(Smem::bPFull + w, static_cast<uint32_t>(j - 1) & 1u)) break;
-        BCA_TRACE_AT(p, j, 1 + 2 * w);
-        tc_fence_after();
-        if (elect_one()) {
+      for (int w = 0; w < 2; ++w) {
+        if (!(w ? act1 : act0)) continue;
+        const int jend = w ? c.jend[1] : c.jend[0];
+        if (j > c.j0 && j - 1 < jend) {
+          // O_w += P_w(j-1) V_{j-1}; P must be consumed before S_w(j) overwrites it.
+          if (!wait(Smem::bPFull + w, static_cast<uint32_t>(npv[w]) & 1u)) break;
+          ++npv[w];
+          BCA_TRACE_AT(p, it0 / 2 + (j - c.j0), 1 + 2 * w);
+          tc_fence_after();
+          if (elect_one()) {
 #pragma unroll
-          for (int s = 0; s < kBN / 16; ++s)
-            mma_bf16_ts(tmem + col_o(w), tmem + col_s(w) + s * 8, dv + ((s * 2048) >> 4), kIdescO,
-                        (j - 1 > 0 || s > 0) ? 1u : 0u);
-          if (j - 1 == u.ntiles[w] - 1) mma_commit(bar(Smem::bOFull + w));
-        }
-        __syncwarp();
-      }
-      if (j < u.ntiles[w]) {
-        // S_w = Q_w K_j^T
-        if (elect_one()) {
-#pragma unroll
-          for (int s = 0; s < kHeadDim / 16; ++s) {
-            const uint32_t koff = ((s / 4) * kHalfBytes + (s % 4) * 32) >> 4;
-            mma_bf16_ss(tmem + col_s(w), dq[w] + koff, dk + koff, kIdescS, s > 0 ? 1u : 0u);
+            for (int s = 0; s < kBN / 16; ++s)
+              mma_bf16_ts(tmem + col_o(w), tmem + col_s(w) + s * 8, dv + ((s * 2048) >> 4),
+                          kIdescO, (j - 1 > c.j0 || s > 0) ? 1u : 0u);
+            if (j == jend) mma_commit(bar(Smem::bOFull + w));
           }
-          mma_commit(bar(Smem::bSFull + w));
+          __syncwarp();
         }
-        __syncwarp();
-        BCA_TRACE_AT(p, j, 2 + 2 * w);
+        if (j < jend) {
+          // S_w = Q_w K_j^T
+          if (elect_one()) {
+#pragma unroll
+            for (int s = 0; s < kHeadDim / 16; ++s) {
+              const uint32_t koff = ((s / 4) * kHalfBytes + (s % 4) * 32) >> 4;
+              mma_bf16_ss(tmem + col_s(w), dq[w] + koff, dk + koff, kIdescS, s > 0 ? 1u : 0u);
+            }
+            mma_commit(bar(Smem::bSFull + w));
+          }
+          __syncwarp();
+          BCA_TRACE_AT(p, it0 / 2 + (j - c.j0), 2 + 2 * w);
+        }
       }
+      if (!ok) break;
+      if (elect_one()) {
+        if (j < c.j1) mma_commit(bar(Smem::bKvEmpty + stK));
+        if (j > c.j0) mma_commit(bar(Smem::bKvEmpty + stV));
+        // The last S MMA of the item has been issued: Q may be reloaded once it is done.
+        if (j == c.j1 - 1) mma_commit(bar(Smem::bQEmpty));
+      }
+      __syncwarp();
     }
-    if (!ok) break;
-    if (elect_one()) {
-      if (j < u.n_total) mma_commit(bar(Smem::bKvEmpty + stK));
-      if (j > 0) mma_commit(bar(Smem::bKvEmpty + stV));
-    }
-    __syncwarp();
+    it = it0 + 2 * (c.j1 - c.j0);
   }
   // Everything issued must be complete before TMEM is released.
   if (elect_one()) mma_commit(bar(Smem::bDone));
@@ -485,168 +563,205 @@ __device__ void mma_role(const AttnParams<MAXR>& p, const Unit& u, uint32_t sbas
 // Softmax + epilogue: 128 threads (one warpgroup) per Q tile, one row each.
 // ---------------------------------------------------------------------------
 template <int MAXR>
-__device__ void softmax_role(const AttnParams<MAXR>& p, const Unit& u, int w, uint32_t bars,
-                             uint32_t tmem, volatile int* abort, float v_out_scale) {
+__device__ void softmax_role(const AttnParams<MAXR>& p, int w, uint32_t bars, uint32_t tmem,
+                             volatile int* abort) {
   auto bar = [&](int i) { return bars + 8u * static_cast<uint32_t>(i); };
-  const int rows_w = w ? u.rows[1] : u.rows[0];
-  const int ntiles_w = w ? u.ntiles[1] : u.ntiles[0];
-  if (rows_w <= 0) return;
   const int warp = (threadIdx.x / 32) % 4;
   const int lane = threadIdx.x % 32;
   const int row = warp * 32 + lane;
   const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
   const uint32_t tS = tmem + lane_off + col_s(w);
   const uint32_t tO = tmem + lane_off + col_o(w);
-  const int grow = u.q_row0 + w * kBM + row;
-  int lim = kNoLimit;
-  if (p.mode == kModePrefill) lim = row < rows_w ? block_end(p, grow) : p.seq_len;
-  // e4m3 cache tiles: scores scale by k_scale (folded into the exp2 scale) and P by
-  // v_scale (folded into the exp2 bias; the row sum keeps the unscaled P).
-  float sl2_cache = p.scale_log2, lg_vs = 0.f, inv_vs = 1.f;
-  if (p.mode == kModeStep) {
-    if (!BCA_CHECK(p.dev_status, u.req < p.n_req && (!p.k_fp8 || p.k_scale[u.req]) &&
-                                     (!p.v_fp8 || p.v_scale[u.req]), 4))
-      return;
-    if (p.k_fp8) sl2_cache *= __ldg(p.k_scale[u.req] + u.h);
-    if (p.v_fp8) {
-      const float vs = __ldg(p.v_scale[u.req] + u.h);
-      lg_vs = __log2f(vs);
-      inv_vs = 1.0f / vs;
-    }
-  }
+  const bool prefill = p.mode == kModePrefill;
+  const int seq_len = p.seq_len;
   const uint32_t b_s = bar(Smem::bSFull + w), b_p = bar(Smem::bPFull + w);
-  float m_run = -INFINITY, l_run = 0.f;
-  bool ok = true;
-  for (int j = 0; j < ntiles_w; ++j) {
-    const bool got = mbar_wait_bounded(b_s, static_cast<uint32_t>(j) & 1u, abort, p.timeout_ns);
-    if (!__all_sync(0xffffffffu, got)) {
-      raise_abort(abort, p.dev_status, 61);
-      ok = false;
-      break;
+  const uint32_t b_o = bar(Smem::bOFull + w);
+  int ns = 0, no = 0;  // S tiles and O results consumed (barrier phases)
+  for (int item = blockIdx.x; item < p.n_items; item += gridDim.x) {
+    const Item c = decode_item(p, item);
+    if (!tile_active(c, w)) continue;
+    const int rows_w = w ? c.rows[1] : c.rows[0];
+    const int jend = w ? c.jend[1] : c.jend[0];
+    const int grow = c.q_row0 + w * kBM + row;
+    int lim = kNoLimit;
+    if (prefill) lim = row < rows_w ? block_end(p, grow) : seq_len;
+    // e4m3 cache tiles: scores scale by k_scale (folded into the exp2 scale) and P
+    // by v_scale (folded into the exp2 bias; the row sum keeps the unscaled P).
+    float sl2_cache = p.scale_log2, lg_vs = 0.f, inv_vs = 1.f;
+    if (!prefill) {
+      if (!BCA_CHECK(p.dev_status, c.req < p.n_req && (!p.k_fp8 || p.k_scale[c.req]) &&
+                                       (!p.v_fp8 || p.v_scale[c.req]), 4))
+        return;
+      if (p.k_fp8) sl2_cache *= __ldg(p.k_scale[c.req] + c.h);
+      if (p.v_fp8) {
+        const float vs = __ldg(p.v_scale[c.req] + c.h);
+        lg_vs = __log2f(vs);
+        inv_vs = 1.0f / vs;
+      }
+    }
+    const float sl2_base = p.scale_log2;
+    float m_run = -INFINITY, l_run = 0.f;
+    for (int j = c.j0; j < jend; ++j, ++ns) {
+      const bool got = mbar_wait_bounded(b_s, static_cast<uint32_t>(ns) & 1u, abort, p.timeout_ns);
+      if (!__all_sync(0xffffffffu, got)) {
+        raise_abort(abort, p.dev_status, 61);
+        return;
+      }
+      tc_fence_after();
+      const bool tr = row == 0;
+      const bool trw = lane == 0 && warp > 0;
+      if (tr) BCA_TRACE_AT(p, ns, 5 + 5 * w);
+      uint32_t r[128];
+#pragma unroll
+      for (int cc = 0; cc < 4; ++cc)
+        tmem_ld_32x32b_x32(tS + 32 * cc, *reinterpret_cast<uint32_t(*)[32]>(&r[32 * cc]));
+      tmem_wait_ld();
+      if (tr) BCA_TRACE_AT(p, ns, 6 + 5 * w);
+      int valid, key_base;
+      kv_tile_extent(prefill, c, seq_len, j, valid, key_base);
+      const bool cache_tile = !prefill && j < c.n_cache_tiles;
+      const float sl2 = cache_tile ? sl2_cache : sl2_base;
+      const int nv = min(valid, lim - key_base);
+      if (nv < kBN) {
+#pragma unroll
+        for (int cc = 0; cc < 128; ++cc)
+          if (cc >= nv) r[cc] = __float_as_uint(-INFINITY);
+      }
+      if (tr && w == 0) BCA_TRACE_AT(p, ns, 25);
+      // Row max: 8 independent chains of three-input max, then a short tree.
+      float t[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const float* x = reinterpret_cast<const float*>(&r[16 * i]);
+        float a = fmax3(x[0], x[1], x[2]);
+#pragma unroll
+        for (int e = 3; e < 15; e += 2) a = fmax3(a, x[e], x[e + 1]);
+        t[i] = fmaxf(a, x[15]);
+      }
+      const float mx = fmax3(fmax3(t[0], t[1], t[2]), fmax3(t[3], t[4], t[5]), fmaxf(t[6], t[7]));
+      const float m_new = mx * sl2;
+      if (tr) BCA_TRACE_AT(p, ns, 7 + 5 * w);
+      const bool need = m_new > m_run + kRescaleThreshold;
+      float f = 1.0f;
+      if (need) {
+        f = ex2_approx(m_run - m_new);  // 0 on the first tile (m_run = -inf)
+        l_run *= f;
+        m_run = m_new;
+      }
+      const float neg_m = (cache_tile ? lg_vs : 0.f) - m_run;
+      // p = 2^(s * sl2 - m) on column pairs: packed fp32x2 FMA for the exponent,
+      // then MUFU ex2 for most pairs and the FMA-pipe polynomial for kPolyPairs of
+      // every 8 (balances the two pipes); P is packed to bf16 in place over S.
+      const uint64_t sl2x2 = f2_pack(sl2, sl2), negm2 = f2_pack(neg_m, neg_m);
+      uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
+#pragma unroll
+      for (int cc = 0; cc < 64; ++cc) {
+        const uint64_t x =
+            f2_fma(f2_pack(__uint_as_float(r[2 * cc]), __uint_as_float(r[2 * cc + 1])), sl2x2,
+                   negm2);
+        uint64_t pp;
+        if ((cc & 7) >= 8 - kPolyPairs) {
+          pp = exp2_poly2(x);
+        } else {
+          float x0, x1;
+          f2_unpack(x, x0, x1);
+          pp = f2_pack(ex2_approx(x0), ex2_approx(x1));
+        }
+        acc[cc & 3] = f2_add(acc[cc & 3], pp);
+        float p0, p1;
+        f2_unpack(pp, p0, p1);
+        r[cc] = pack_bf16x2(p0, p1);
+      }
+      float a0, a1, b0, b1;
+      f2_unpack(f2_add(acc[0], acc[1]), a0, a1);
+      f2_unpack(f2_add(acc[2], acc[3]), b0, b1);
+      const float tile_sum = (a0 + a1) + (b0 + b1);
+      l_run += cache_tile ? tile_sum * inv_vs : tile_sum;
+      if (tr) BCA_TRACE_AT(p, ns, 8 + 5 * w);
+      tmem_st_32x32b_x32(tS, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
+      tmem_st_32x32b_x32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
+      // O was last written by P(j-1) V_{j-1}, complete before S(j) was signalled; it
+      // must be rescaled before P(j) V_j is issued (that waits for our arrival).
+      if (j > c.j0 && __any_sync(0xffffffffu, need)) {
+        const uint64_t f2 = f2_pack(f, f);
+#pragma unroll
+        for (int cc = 0; cc < 8; ++cc) {
+          uint32_t o[16];
+          tmem_ld_32x32b_x16(tO + 16 * cc, o);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 16; e += 2) {
+            float y0, y1;
+            f2_unpack(f2_mul(f2_pack(__uint_as_float(o[e]), __uint_as_float(o[e + 1])), f2), y0,
+                      y1);
+            o[e] = __float_as_uint(y0);
+            o[e + 1] = __float_as_uint(y1);
+          }
+          tmem_st_32x32b_x16(tO + 16 * cc, o);
+        }
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(b_p);
+      if (tr) BCA_TRACE_AT(p, ns, 9 + 5 * w);
+      if (trw) BCA_TRACE_AT(p, ns, 14 + 3 * w + warp);
+    }
+    // Epilogue: O of this item is complete once its last P V is.
+    {
+      const bool got = mbar_wait_bounded(b_o, static_cast<uint32_t>(no) & 1u, abort, p.timeout_ns);
+      ++no;
+      if (!__all_sync(0xffffffffu, got)) {
+        raise_abort(abort, p.dev_status, 62);
+        return;
+      }
     }
     tc_fence_after();
-    const bool tr = row == 0;
-    const bool trw = lane == 0 && warp > 0;
-    if (tr) BCA_TRACE_AT(p, j, 5 + 5 * w);
-    uint32_t r[128];
+    if (c.partial < 0) {
+      const float inv = 1.0f / l_run;
+      const bool store = row < rows_w &&
+                         BCA_CHECK(p.dev_status, grow < p.o_rows && c.h < p.heads, 3);
+      uint4* dst =
+          reinterpret_cast<uint4*>(p.o + (static_cast<size_t>(grow) * p.heads + c.h) * kHeadDim);
 #pragma unroll
-    for (int c = 0; c < 4; ++c)
-      tmem_ld_32x32b_x32(tS + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&r[32 * c]));
-    tmem_wait_ld();
-    if (tr) BCA_TRACE_AT(p, j, 6 + 5 * w);
-    int valid, key_base;
-    kv_tile_extent(p, u, j, valid, key_base);
-    const bool cache_tile = p.mode == kModeStep && j < u.n_cache_tiles;
-    const float sl2 = cache_tile ? sl2_cache : p.scale_log2;
-    const int nv = min(valid, lim - key_base);
-    if (nv < kBN) {
+      for (int cc = 0; cc < 4; ++cc) {
+        uint32_t o[32];
+        tmem_ld_32x32b_x32(tO + 32 * cc, o);
+        tmem_wait_ld();
+        uint32_t pk[16];
 #pragma unroll
-      for (int c = 0; c < 128; ++c)
-        if (c >= nv) r[c] = __float_as_uint(-INFINITY);
-    }
-    if (tr && w == 0) BCA_TRACE_AT(p, j, 25);
-    // Row max: 8 independent chains of three-input max, then a short tree.
-    float t[8];
+        for (int e = 0; e < 16; ++e)
+          pk[e] = pack_bf16x2(__uint_as_float(o[2 * e]) * inv, __uint_as_float(o[2 * e + 1]) * inv);
+        if (store) {
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const float* x = reinterpret_cast<const float*>(&r[16 * i]);
-      float a = fmax3(x[0], x[1], x[2]);
-#pragma unroll
-      for (int e = 3; e < 15; e += 2) a = fmax3(a, x[e], x[e + 1]);
-      t[i] = fmaxf(a, x[15]);
-    }
-    const float mx = fmax3(fmax3(t[0], t[1], t[2]), fmax3(t[3], t[4], t[5]), fmaxf(t[6], t[7]));
-    const float m_new = mx * sl2;
-    if (tr) BCA_TRACE_AT(p, j, 7 + 5 * w);
-    const bool need = m_new > m_run + kRescaleThreshold;
-    float f = 1.0f;
-    if (need) {
-      f = ex2_approx(m_run - m_new);  // 0 on the first tile (m_run = -inf)
-      l_run *= f;
-      m_run = m_new;
-    }
-    const float neg_m = (cache_tile ? lg_vs : 0.f) - m_run;
-    // p = 2^(s * sl2 - m) on column pairs: packed fp32x2 FMA for the exponent,
-    // then MUFU ex2 for most pairs and the FMA-pipe polynomial for kPolyPairs of
-    // every 8 (balances the two pipes); P is packed to bf16 in place over S.
-    const uint64_t sl2x2 = f2_pack(sl2, sl2), negm2 = f2_pack(neg_m, neg_m);
-    uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
-#pragma unroll
-    for (int c = 0; c < 64; ++c) {
-      const uint64_t x = f2_fma(f2_pack(__uint_as_float(r[2 * c]), __uint_as_float(r[2 * c + 1])),
-                                sl2x2, negm2);
-      uint64_t pp;
-      if ((c & 7) >= 8 - kPolyPairs) {
-        pp = exp2_poly2(x);
-      } else {
-        float x0, x1;
-        f2_unpack(x, x0, x1);
-        pp = f2_pack(ex2_approx(x0), ex2_approx(x1));
+          for (int e = 0; e < 4; ++e)
+            dst[4 * cc + e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+        }
       }
-      acc[c & 3] = f2_add(acc[c & 3], pp);
-      float p0, p1;
-      f2_unpack(pp, p0, p1);
-      r[c] = pack_bf16x2(p0, p1);
-    }
-    float a0, a1, b0, b1;
-    f2_unpack(f2_add(acc[0], acc[1]), a0, a1);
-    f2_unpack(f2_add(acc[2], acc[3]), b0, b1);
-    const float tile_sum = (a0 + a1) + (b0 + b1);
-    l_run += cache_tile ? tile_sum * inv_vs : tile_sum;
-    if (tr) BCA_TRACE_AT(p, j, 8 + 5 * w);
-    tmem_st_32x32b_x32(tS, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
-    tmem_st_32x32b_x32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
-    // O was last written by P(j-1) V_{j-1}, complete before S(j) was signalled; it
-    // must be rescaled before P(j) V_j is issued (that waits for our arrival).
-    if (j > 0 && __any_sync(0xffffffffu, need)) {
+    } else {
+      // Split chunk: unnormalised O (with this chunk's running max) plus m and l.
+      float* ws = p.workspace + static_cast<size_t>(c.partial) * (kChunkBytes / 4);
+      const int r2 = w * kBM + row;
+      float4* od = reinterpret_cast<float4*>(ws + static_cast<size_t>(r2) * kHeadDim);
 #pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        uint32_t o[16];
-        tmem_ld_32x32b_x16(tO + 16 * c, o);
+      for (int cc = 0; cc < 4; ++cc) {
+        uint32_t o[32];
+        tmem_ld_32x32b_x32(tO + 32 * cc, o);
         tmem_wait_ld();
 #pragma unroll
-        for (int e = 0; e < 16; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * f);
-        tmem_st_32x32b_x16(tO + 16 * c, o);
+        for (int e = 0; e < 8; ++e)
+          od[8 * cc + e] = make_float4(__uint_as_float(o[4 * e]), __uint_as_float(o[4 * e + 1]),
+                                       __uint_as_float(o[4 * e + 2]), __uint_as_float(o[4 * e + 3]));
       }
+      ws[kChunkRows * kHeadDim + r2] = m_run;
+      ws[kChunkRows * kHeadDim + kChunkRows + r2] = l_run;
     }
-    tmem_wait_st();
-    tc_fence_before();
-    mbar_arrive(b_p);
-    if (tr) BCA_TRACE_AT(p, j, 9 + 5 * w);
-    if (trw) BCA_TRACE_AT(p, j, 14 + 3 * w + warp);
-  }
-  if (!ok) return;
-  {
-    const bool got = mbar_wait_bounded(bar(Smem::bOFull + w), 0, abort, p.timeout_ns);
-    if (!__all_sync(0xffffffffu, got)) {
-      raise_abort(abort, p.dev_status, 62);
-      return;
-    }
-  }
-  tc_fence_after();
-  const float inv = v_out_scale / l_run;
-  const bool store = row < rows_w &&
-                     BCA_CHECK(p.dev_status, grow < p.o_rows && u.h < p.heads, 3);
-  uint4* dst = reinterpret_cast<uint4*>(p.o + (static_cast<size_t>(grow) * p.heads + u.h) * kHeadDim);
-#pragma unroll
-  for (int c = 0; c < 4; ++c) {
-    uint32_t o[32];
-    tmem_ld_32x32b_x32(tO + 32 * c, o);
-    tmem_wait_ld();
-    uint32_t pk[16];
-#pragma unroll
-    for (int e = 0; e < 16; ++e)
-      pk[e] = pack_bf16x2(__uint_as_float(o[2 * e]) * inv, __uint_as_float(o[2 * e + 1]) * inv);
-    if (store) {
-#pragma unroll
-      for (int e = 0; e < 4; ++e)
-        dst[4 * c + e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
-    }
+    // O of this item has been read: the next item's first P V (accumulate = 0) only
+    // runs after our next P arrival, which follows these TMEM loads in program order.
   }
 }
 
 // ---------------------------------------------------------------------------
-// The kernel
+// The kernel (persistent: one CTA per SM, static round-robin over work items)
 // ---------------------------------------------------------------------------
 template <int MAXR>
 __global__ void __launch_bounds__(kAttnThreads, 1)
@@ -660,7 +775,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Smem::kTmemSlot);
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
-  const Unit u = decode_unit(p, blockIdx.x);
 
   if (threadIdx.x == 0) {
     auto bar = [&](int i) { return bars + 8u * static_cast<uint32_t>(i); };
@@ -669,17 +783,16 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       mbar_init(bar(Smem::bSFull + i), 1);
       mbar_init(bar(Smem::bPFull + i), 128);
       mbar_init(bar(Smem::bOFull + i), 1);
+      mbar_init(bar(Smem::bStgFull + i), 1);
+      mbar_init(bar(Smem::bStgEmpty + i), 1);
     }
     for (int i = 0; i < kStages; ++i) {
       mbar_init(bar(Smem::bKvFull + i), 1);
       mbar_init(bar(Smem::bKvEmpty + i), 1);
     }
     mbar_init(bar(Smem::bDone), 1);
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(bar(Smem::bStgFull + i), 1);
-      mbar_init(bar(Smem::bStgEmpty + i), 1);
-    }
     mbar_init(bar(Smem::bConv), kConvThreads);
+    mbar_init(bar(Smem::bQEmpty), 1);
     *abort = 0;
     fence_barrier_init();
   }
@@ -699,24 +812,85 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 
   if (warp < 8) {
     regs_increase<kSoftmaxRegs>();
-    softmax_role(p, u, warp / 4, bars, tmem, abort, 1.0f);
+    softmax_role(p, warp / 4, bars, tmem, abort);
   } else {
     regs_decrease<kOtherRegs>();
-  }
-  if (warp < 8) {
-  } else if (warp == kWarpProducer) {
-    if (lane == 0) producer_role(p, u, sbase, bars, abort);
-  } else if (warp == kWarpMma) {
-    mma_role(p, u, sbase, bars, tmem, abort);
-    __syncwarp();
-  } else if (p.mode == kModeStep && (p.k_fp8 || p.v_fp8)) {
-    converter_role(p, u, sbase, bars, abort);
+    if (warp == kWarpProducer) {
+      if (lane == 0) producer_role(p, sbase, bars, abort);
+    } else if (warp == kWarpMma) {
+      mma_role(p, sbase, bars, tmem, abort);
+      __syncwarp();
+    } else if (p.mode == kModeStep && (p.k_fp8 || p.v_fp8)) {
+      converter_role(p, sbase, bars, abort);
+    }
   }
   tc_fence_before();
   __syncthreads();
   if (warp == kWarpMma) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Merge the split chunks of a unit: O = sum_c 2^(m_c - M) O_c / sum_c 2^(m_c - M) l_c.
+// One thread per (split unit, row); the grid covers n_split_units * 256 rows.
+// ---------------------------------------------------------------------------
+constexpr int kMaxSplit = 8;
+
+template <int MAXR>
+__global__ void __launch_bounds__(256)
+    attn_combine_kernel(const __grid_constant__ AttnParams<MAXR> p, int n_split_units) {
+  const int gid = blockIdx.x * blockDim.x + threadIdx.x;
+  const int su = gid / kChunkRows, r2 = gid % kChunkRows;
+  if (su >= n_split_units) return;
+  const int k = p.split_k;
+  const Item c = decode_item(p, p.full_items + su * k);  // chunk 0 of the unit
+  const int w = r2 / kBM, row = r2 % kBM;
+  const int rows_w = w ? c.rows[1] : c.rows[0];
+  if (row >= rows_w || k < 1 || k > kMaxSplit) return;
+  const int grow = c.q_row0 + w * kBM + row;
+  if (!BCA_CHECK(p.dev_status, grow < p.o_rows && c.h < p.heads, 5)) return;
+  constexpr size_t kStride = kChunkBytes / 4;
+  const float* ws0 = p.workspace + static_cast<size_t>(su) * k * kStride;
+  float M = -INFINITY;
+  for (int ci = 0; ci < k; ++ci) M = fmaxf(M, ws0[ci * kStride + kChunkRows * kHeadDim + r2]);
+  float wgt[kMaxSplit];
+  float L = 0.f;
+#pragma unroll
+  for (int ci = 0; ci < kMaxSplit; ++ci) {
+    wgt[ci] = 0.f;
+    if (ci < k) {
+      const float m = ws0[ci * kStride + kChunkRows * kHeadDim + r2];
+      const float l = ws0[ci * kStride + kChunkRows * kHeadDim + kChunkRows + r2];
+      wgt[ci] = ex2_approx(m - M);
+      L += wgt[ci] * l;
+    }
+  }
+  const float inv = 1.0f / L;
+  uint4* dst = reinterpret_cast<uint4*>(p.o + (static_cast<size_t>(grow) * p.heads + c.h) * kHeadDim);
+#pragma unroll 1
+  for (int e = 0; e < kHeadDim; e += 8) {
+    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int ci = 0; ci < kMaxSplit; ++ci) {
+      if (ci >= k) break;
+      const float4* src = reinterpret_cast<const float4*>(
+          ws0 + ci * kStride + static_cast<size_t>(r2) * kHeadDim + e);
+      const float4 a = src[0], b = src[1];
+      acc[0] += wgt[ci] * a.x;
+      acc[1] += wgt[ci] * a.y;
+      acc[2] += wgt[ci] * a.z;
+      acc[3] += wgt[ci] * a.w;
+      acc[4] += wgt[ci] * b.x;
+      acc[5] += wgt[ci] * b.y;
+      acc[6] += wgt[ci] * b.z;
+      acc[7] += wgt[ci] * b.w;
+    }
+    dst[e / 8] = make_uint4(pack_bf16x2(acc[0] * inv, acc[1] * inv),
+                            pack_bf16x2(acc[2] * inv, acc[3] * inv),
+                            pack_bf16x2(acc[4] * inv, acc[5] * inv),
+                            pack_bf16x2(acc[6] * inv, acc[7] * inv));
   }
 }
 

@@ -153,9 +153,45 @@ std::vector<char>& attr_flags() {
   return g_attr_attn64;
 }
 
+int sm_count() {
+  static std::mutex mu;
+  static std::vector<int> counts;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  std::lock_guard<std::mutex> lk(mu);
+  if (counts.size() <= static_cast<size_t>(dev)) counts.resize(dev + 1, 0);
+  if (!counts[dev] &&
+      cudaDeviceGetAttribute(&counts[dev], cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    counts[dev] = 0;
+  return counts[dev];
+}
+
+// Work-item schedule of the persistent kernel.  `unit_tiles(u)` gives the KV tiles
+// of unit u (units are in scheduling order, heaviest first).  With a workspace, the
+// units of the last partial round are split along the keys into k chunks so that
+// all CTAs finish together: k = grid / leftover units, limited by the workspace,
+// kMaxSplit and the smallest split unit's tile count.
+template <int MAXR, typename TilesFn>
+int plan_items(AttnParams<MAXR>& p, int units, int grid, size_t ws_chunks, TilesFn unit_tiles) {
+  p.full_items = units;
+  p.n_items = units;
+  p.split_k = 1;
+  if (ws_chunks == 0 || units <= grid) return 0;
+  const int rounds = units / grid, rem = units - rounds * grid;
+  if (rem == 0) return 0;
+  int k = std::min<int>(grid / rem, bca::kMaxSplit);
+  k = std::min<int>(k, static_cast<int>(ws_chunks / static_cast<size_t>(rem)));
+  for (int u = rounds * grid; u < units && k >= 2; ++u) k = std::min(k, unit_tiles(u));
+  if (k < 2) return 0;
+  p.full_items = rounds * grid;
+  p.split_k = k;
+  p.n_items = rounds * grid + rem * k;
+  return rem;
+}
+
 template <int MAXR>
-bca_status launch_attn(const AttnParams<MAXR>& p, int n_units, cudaStream_t stream) {
-  if (n_units <= 0) return BCA_OK;
+bca_status launch_attn(const AttnParams<MAXR>& p, int n_split_units, cudaStream_t stream) {
+  if (p.n_items <= 0) return BCA_OK;
   if (!ensure_smem_attr(bca::attn_fwd_kernel<MAXR>, bca::Smem::kDynamicBytes, attr_flags<MAXR>()))
     return BCA_ERR_CUDA;
   // The kernel re-splits its launch registers between warpgroups (setmaxnreg); that
@@ -169,9 +205,18 @@ bca_status launch_attn(const AttnParams<MAXR>& p, int n_units, cudaStream_t stre
                   128u * (2u * bca::kSoftmaxRegs + bca::kOtherRegs);
   });
   if (!regs_ok) return BCA_ERR_CUDA;
-  bca::attn_fwd_kernel<MAXR>
-      <<<n_units, bca::kAttnThreads, bca::Smem::kDynamicBytes, stream>>>(p);
-  return cudaGetLastError() == cudaSuccess ? BCA_OK : BCA_ERR_CUDA;
+  const int sms = sm_count();
+  if (sms <= 0) return BCA_ERR_CUDA;
+  const int grid = std::min(sms, p.n_items);
+  bca::attn_fwd_kernel<MAXR><<<grid, bca::kAttnThreads, bca::Smem::kDynamicBytes, stream>>>(p);
+  if (cudaGetLastError() != cudaSuccess) return BCA_ERR_CUDA;
+  if (n_split_units > 0) {
+    const int threads = 256, rows = n_split_units * bca::kChunkRows;
+    bca::attn_combine_kernel<MAXR><<<(rows + threads - 1) / threads, threads, 0, stream>>>(
+        p, n_split_units);
+    if (cudaGetLastError() != cudaSuccess) return BCA_ERR_CUDA;
+  }
+  return BCA_OK;
 }
 
 // Enqueue the store passes for one slot (no host-side slot updates).
@@ -336,7 +381,8 @@ bca_status bca_prefill(const void* q, const void* k, const void* v, void* o, int
   for (int b = 0; b <= n_blocks; ++b) p.block_off[b] = off[b];
   const int nqp = (seq_len + 2 * bca::kBM - 1) / (2 * bca::kBM);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  bca_status st = launch_attn(p, nqp * heads, s);
+  plan_items(p, nqp * heads, 1, 0, [](int) { return 1; });  // prefill: whole units only
+  bca_status st = launch_attn(p, 0, s);
   if (st != BCA_OK) return st;
   if (slot) {
     st = enqueue_kv_store(k, v, n_prefix, static_cast<int64_t>(heads) * 128, slot, dev_status, s);
@@ -347,10 +393,17 @@ bca_status bca_prefill(const void* q, const void* k, const void* v, void* o, int
   return BCA_OK;
 }
 
+size_t bca_step_workspace_bytes(void) {
+  const int sms = sm_count();
+  return sms > 0 ? static_cast<size_t>(sms) * bca::kChunkBytes : 0;
+}
+
 bca_status bca_step_attend(const void* q_t, const void* k_t, const void* v_t, void* o_t,
                            const int32_t* cu, const bca_kv_slot* slots, int32_t n_req,
-                           int32_t heads, int32_t head_dim, float scale, int32_t* dev_status,
-                           void* stream) {
+                           int32_t heads, int32_t head_dim, float scale, void* workspace,
+                           size_t workspace_bytes, int32_t* dev_status, void* stream) {
+  if (workspace && (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return BCA_ERR_INVALID_ARG;
+  const size_t ws_chunks = workspace ? workspace_bytes / bca::kChunkBytes : 0;
   if (!cu || !slots) return BCA_ERR_INVALID_ARG;
   if (head_dim != 128) return BCA_ERR_UNSUPPORTED;
   if (heads < 1 || heads > 256 || n_req < 1 || n_req > BCA_MAX_BATCH) return BCA_ERR_INVALID_ARG;
@@ -421,7 +474,15 @@ bca_status bca_step_attend(const void* q_t, const void* k_t, const void* v_t, vo
       units += heads * ((p.q_len[i] + 2 * bca::kBM - 1) / (2 * bca::kBM));
     }
     p.unit_start[nr] = units;
-    return launch_attn(p, units, static_cast<cudaStream_t>(stream));
+    p.workspace = static_cast<float*>(workspace);
+    const int sms = sm_count();
+    if (sms <= 0) return BCA_ERR_CUDA;
+    const int n_split = plan_items(p, units, sms, ws_chunks, [&](int unit) {
+      int i = 0;
+      while (i + 1 < nr && unit >= p.unit_start[i + 1]) ++i;
+      return (p.n_cache[i] + bca::kBN - 1) / bca::kBN + (p.q_len[i] + bca::kBN - 1) / bca::kBN;
+    });
+    return launch_attn(p, n_split, static_cast<cudaStream_t>(stream));
   };
   if (nr <= 1) {
     AttnParams<1> p;

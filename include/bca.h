@@ -23,8 +23,9 @@
  *    token rows heads*head_dim elements apart unless a stride is given.
  *  - Cache layout: per (request, layer) slot, K and V each [heads, cap_tokens,
  *    head_dim]; bf16, or OFP8 E4M3 codes (1 byte) with one fp32 scale per head.
- *  - All device memory is owned by the caller.  The library allocates no device
- *    memory; it keeps only host-side state (a driver entry point).
+ *  - All device memory is owned by the caller (including the optional
+ *    bca_step_attend workspace).  The library allocates no device memory; it keeps
+ *    only host-side state (a driver entry point, per-device attributes).
  *  - Calls enqueue work on `stream` and return at once.  Argument and state
  *    errors are reported synchronously, before anything is launched, and then
  *    nothing is written.  A failed launch returns BCA_ERR_CUDA.
@@ -148,13 +149,23 @@ bca_status bca_prefill(const void* q, const void* k, const void* v, void* o, int
  *   slots            : HOST array of n_req slots; each filled (epoch != 0) with
  *                      num_heads == heads, head_dim == 128, and all the same dtype.
  *   n_req            : 1..BCA_MAX_BATCH.
+ *   workspace,
+ *   workspace_bytes  : optional device scratch (256-byte aligned, caller-owned;
+ *                      NULL = none); see bca_step_workspace_bytes.  Its contents
+ *                      are overwritten; calls sharing a workspace must not overlap.
  * For e4m3 tensors the per-head scales are folded in: K's into the softmax scale,
- * V's into the output normalisation.  A request with T_r == 0 is skipped.
+ * V's into the P of the cached keys.  A request with T_r == 0 is skipped.
  * Errors: BCA_ERR_STATE for an empty slot, BCA_ERR_UNSUPPORTED for mixed dtypes. */
 bca_status bca_step_attend(const void* q_t, const void* k_t, const void* v_t, void* o_t,
                            const int32_t* cu_target, const bca_kv_slot* slots, int32_t n_req,
-                           int32_t heads, int32_t head_dim, float scale, int32_t* dev_status,
-                           void* stream);
+                           int32_t heads, int32_t head_dim, float scale, void* workspace,
+                           size_t workspace_bytes, int32_t* dev_status, void* stream);
+
+/* Bytes of the optional bca_step_attend workspace that lets the kernel split the
+ * last partial round of work along the keys (so that every SM finishes at the same
+ * time) for the current device: one chunk of 256 rows x (128 + 2) fp32 per SM.
+ * Without it (workspace NULL or too small for any chunk) nothing is split. */
+size_t bca_step_workspace_bytes(void);
 
 /* Human-readable name of a status code (static storage). */
 const char* bca_status_string(bca_status status);

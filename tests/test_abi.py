@@ -120,7 +120,8 @@ def test_step_attend_argument_errors(L):
     arr = (bca.SlotStruct * 2)(s0, s1)
     call = lambda **kw: L.bca_step_attend(FAKE, FAKE, FAKE, FAKE, kw.get("cu", cu),
                                           kw.get("arr", arr), kw.get("n", 2), kw.get("H", 2),
-                                          kw.get("d", 128), kw.get("scale", 0.1), None, None)
+                                          kw.get("d", 128), kw.get("scale", 0.1),
+                                          kw.get("ws", None), kw.get("ws_bytes", 0), None, None)
     assert call(d=96) == 2
     assert call(n=0) == 1
     assert call(n=65) == 1
@@ -133,6 +134,7 @@ def test_step_attend_argument_errors(L):
     assert call(arr=mixed) == 2
     over = _slot(L, cap=64, n=65)
     assert call(arr=(bca.SlotStruct * 2)(s0, over)) == 1
+    assert call(ws=ctypes.c_void_p((1 << 24) + 16), ws_bytes=1 << 20) == 1  # misaligned workspace
 
 
 def test_selftest_wait_rejects_bad_bounds(L):

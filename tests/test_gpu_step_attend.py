@@ -43,14 +43,15 @@ def oracle_for(req, rows=None):
                               v_scale=s.v_scale_view().cpu().numpy(), rows=rows)
 
 
-def run_batch(reqs, H, device):
+def run_batch(reqs, H, device, workspace=None):
     q = torch.cat([r["q"] for r in reqs])
     k = torch.cat([r["k"] for r in reqs])
     v = torch.cat([r["v"] for r in reqs])
     o = torch.full_like(q, float("nan"))
     cu = np.concatenate([[0], np.cumsum([r["T"] for r in reqs])])
     status = torch.zeros(1, dtype=torch.int32, device=device)
-    bca.step_attend(q, k, v, o, cu, [r["slot"] for r in reqs], SCALE, dev_status=status)
+    bca.step_attend(q, k, v, o, cu, [r["slot"] for r in reqs], SCALE, workspace=workspace,
+                    dev_status=status)
     torch.cuda.synchronize()
     assert int(status.item()) == 0
     return o, cu
@@ -222,3 +223,49 @@ def test_repeated_batches_are_bitwise_identical(cuda_device, mode):
     for _ in range(4):
         again, _ = run_batch(reqs, H, cuda_device)
         assert torch.equal(first, again)
+
+
+# ---------------------------------------------------------------------------
+# Split last round: with a workspace, units of the last partial round are split
+# along the keys and merged by a second kernel.
+# ---------------------------------------------------------------------------
+def test_split_tail_matches_oracle_and_unsplit(cuda_device):
+    """H=32, T=4096, P=512 gives 512 units on 148 SMs: 68 leftover units are split."""
+    H = 32
+    req = make_request(4096, 512, H, seed=900, device=cuda_device)
+    ws = bca.step_workspace(cuda_device)
+    assert bca.step_workspace_bytes() > 0
+    a, _ = run_batch([req], H, cuda_device, workspace=ws)
+    b, _ = run_batch([req], H, cuda_device)
+    rows = sample_rows(4096, 160, seed=9, boundaries=range(256, 4096, 256))
+    want = oracle_for(req, rows=rows)
+    idx = torch.from_numpy(rows).to(cuda_device)
+    assert_parity(a[idx], want, what="split")
+    assert_parity(b[idx], want, what="unsplit")
+    # the unsplit rows of both runs are computed identically
+    diff = (a.float() - b.float()).abs().amax(dim=(1, 2))
+    assert float(diff.max()) < 2e-2
+
+
+@pytest.mark.parametrize("mode", ["bf16", "fp8"])
+def test_split_tail_ragged_batch(cuda_device, mode):
+    H = 16
+    shapes = [(4096, 3000), (2048, 100), (1000, 700)]
+    reqs = [make_request(T, P, H, seed=950 + i, device=cuda_device, cap=P, mode=mode)
+            for i, (T, P) in enumerate(shapes)]
+    ws = bca.step_workspace(cuda_device)
+    o, cu = run_batch(reqs, H, cuda_device, workspace=ws)
+    tol = REL_L2_FP8 if mode != "bf16" else 5e-3
+    for i, r in enumerate(reqs):
+        rows = sample_rows(r["T"], 64, seed=i)
+        got = o[cu[i]:cu[i + 1]][torch.from_numpy(rows).to(cuda_device)]
+        assert_parity(got, oracle_for(r, rows=rows), rel_l2=tol, what=f"req {i}")
+
+
+def test_workspace_too_small_means_no_split(cuda_device):
+    H = 32
+    req = make_request(4096, 512, H, seed=901, device=cuda_device)
+    tiny = torch.empty(1024, dtype=torch.uint8, device=cuda_device)
+    o, _ = run_batch([req], H, cuda_device, workspace=tiny)
+    rows = sample_rows(4096, 64, seed=3)
+    assert_parity(o[torch.from_numpy(rows).to(cuda_device)], oracle_for(req, rows=rows))
