@@ -54,15 +54,36 @@ constexpr int kWarpConv0 = 10;  // warps 10 and 11 convert e4m3 cache tiles
 constexpr int kConvThreads = 64;
 // Register split: launched at kLaunchRegs per thread (384 x 168 = 64512), the two
 // softmax warpgroups take kSoftmaxRegs and warpgroup 2 (producer, MMA, converter)
-// keeps kOtherRegs: 128 * (2 * 208 + 88) = 64512.  The host checks the compiled
+// keeps kOtherRegs: 128 * (2 * 200 + 104) = 64512.  The host checks the compiled
 // register count against this before launching.
 constexpr uint32_t kLaunchRegs = 168;
-constexpr uint32_t kSoftmaxRegs = 208;
-constexpr uint32_t kOtherRegs = 88;
+constexpr uint32_t kSoftmaxRegs = 200;
+constexpr uint32_t kOtherRegs = 104;
 static_assert(128 * (2 * kSoftmaxRegs + kOtherRegs) <= kAttnThreads * kLaunchRegs,
               "register split exceeds the launch allocation");
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
-constexpr int kPolyPairs = 2;  // of every 8 column pairs, exponentiated on the FMA pipe
+#ifndef BCA_POLY_PAIRS
+#define BCA_POLY_PAIRS 0
+#endif
+// Of every 8 column pairs, kPolyPairs are exponentiated on the FMA pipe by the
+// software exp2 (the rest by MUFU ex2).  Measured on B200 for the T2I cached step:
+// 0 -> 1104, 1 -> 1080, 2 -> 1061, 3 -> 1037, 4 -> 1029 TFLOP/s (the softmax is
+// issue-bound, not MUFU-bound), so the default is 0.
+constexpr int kPolyPairs = BCA_POLY_PAIRS;
+// P is handed from the softmax to the MMA in kPHalves parts (1: whole tile; 2: two
+// halves of 64 keys, so P V can start on the first half while the second is made).
+#ifndef BCA_P_HALVES
+#define BCA_P_HALVES 1
+#endif
+constexpr int kPHalves = BCA_P_HALVES;
+// Exponentials of the softmax: 0 = MUFU ex2 (fp32) for most pairs plus the FMA-pipe
+// polynomial for kPolyPairs of every 8; 1 = MUFU ex2 in f16x2 (two per instruction)
+// for every pair.
+#ifndef BCA_EXP_F16
+#define BCA_EXP_F16 0
+#endif
+constexpr bool kExpF16 = BCA_EXP_F16 != 0;
+static_assert(kPHalves == 1 || kPHalves == 2, "kPHalves must be 1 or 2");
 constexpr int kNoLimit = 1 << 30;
 // Split-chunk workspace: per chunk, O [256 rows][128] fp32, then m[256], l[256].
 constexpr int kChunkRows = 2 * kBM;
@@ -142,14 +163,14 @@ struct Smem {
   static constexpr int bKvFull = 2;                    // kStages
   static constexpr int bKvEmpty = 2 + kStages;         // kStages
   static constexpr int bSFull = 2 + 2 * kStages;       // 2
-  static constexpr int bPFull = 4 + 2 * kStages;       // 2
-  static constexpr int bOFull = 6 + 2 * kStages;       // 2
-  static constexpr int bDone = 8 + 2 * kStages;        // 1
-  static constexpr int bStgFull = 9 + 2 * kStages;     // 2
-  static constexpr int bStgEmpty = 11 + 2 * kStages;   // 2
-  static constexpr int bConv = 13 + 2 * kStages;       // 1 (64 converter arrivals per tile)
-  static constexpr int bQEmpty = 14 + 2 * kStages;     // 1 (Q tiles of an item consumed)
-  static constexpr int kNumBars = 15 + 2 * kStages;
+  static constexpr int bPFull = 4 + 2 * kStages;       // 4: [w][half] (128 arrivals each)
+  static constexpr int bOFull = 8 + 2 * kStages;       // 2
+  static constexpr int bDone = 10 + 2 * kStages;       // 1
+  static constexpr int bStgFull = 11 + 2 * kStages;    // 2
+  static constexpr int bStgEmpty = 13 + 2 * kStages;   // 2
+  static constexpr int bConv = 15 + 2 * kStages;       // 1 (64 converter arrivals per tile)
+  static constexpr int bQEmpty = 16 + 2 * kStages;     // 2 (Q tile w of an item consumed)
+  static constexpr int kNumBars = 18 + 2 * kStages;
   static constexpr int kTmemSlot = kBars + 8 * kNumBars;
   static constexpr int kAbort = kTmemSlot + 4;
   static constexpr int kBytes = kAbort + 4;
@@ -306,21 +327,32 @@ __device__ void producer_role(const AttnParams<MAXR>& p, uint32_t sbase, uint32_
   for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x, ++nq) {
     const Item c = decode_item(p, item);
     // Both Q tiles are always loaded (rows past the tensor read as zero), so every
-    // item completes one phase of each Q barrier.
-    if (!mbar_wait_bounded(bar(Smem::bQEmpty), (static_cast<uint32_t>(nq) & 1u) ^ 1u, abort,
-                           p.timeout_ns)) {
-      raise_abort(abort, p.dev_status, 10);
-      ok = false;
-      break;
-    }
+    // item completes one phase of each Q barrier.  Tile w is reloaded as soon as
+    // the previous item's last S_w MMA is done with it.
     BCA_TRACE_AT(p, it / 2, 27);
 #pragma unroll
     for (int w = 0; w < 2; ++w) {
+      if (!mbar_wait_bounded(bar(Smem::bQEmpty + w), (static_cast<uint32_t>(nq) & 1u) ^ 1u, abort,
+                             p.timeout_ns)) {
+        raise_abort(abort, p.dev_status, 10);
+        ok = false;
+        break;
+      }
       const uint32_t dst = sbase + (w == 0 ? Smem::kQ0 : Smem::kQ1);
       const int z = c.q_row0 + w * kBM;
       mbar_arrive_expect_tx(bar(Smem::bQFull + w), kTileBytes);
       tma_load_3d(dst, &p.tm_q, bar(Smem::bQFull + w), 0, c.h, z);
       tma_load_3d(dst + kHalfBytes, &p.tm_q, bar(Smem::bQFull + w), 64, c.h, z);
+    }
+    if (!ok) break;
+    if (item + static_cast<int>(gridDim.x) < p.n_items) {
+      // Warm L2 with the next item's Q while this item runs.
+      const Item nx = decode_item(p, item + gridDim.x);
+#pragma unroll
+      for (int w = 0; w < 2; ++w) {
+        tma_prefetch_l2_3d(&p.tm_q, 0, nx.h, nx.q_row0 + w * kBM);
+        tma_prefetch_l2_3d(&p.tm_q, 64, nx.h, nx.q_row0 + w * kBM);
+      }
     }
     for (int j = c.j0; j < c.j1 && ok; ++j) {
       for (int kv = 0; kv < 2; ++kv, ++it) {
@@ -470,6 +502,10 @@ __device__ void converter_role(const AttnParams<MAXR>& p, uint32_t sbase, uint32
 template <int MAXR>
 __device__ void mma_role(const AttnParams<MAXR>& p, uint32_t sbase, uint32_t bars, uint32_t tmem,
                          volatile int* abort) {
+  // The items of this CTA are one stream of KV tiles.  Iteration t issues, per Q tile
+  // w, O_w += P_w(t-1) V(t-1) (in two K=64 halves, as the softmax hands P over in
+  // halves) and then S_w(t) = Q_w K(t)^T -- also across item boundaries, so the last
+  // tile of an item overlaps the first tile of the next.
   auto bar = [&](int i) { return bars + 8u * static_cast<uint32_t>(i); };
   constexpr uint32_t kIdescS = idesc_bf16_f32(kBM, kBN, false);      // Q K^T: K-major B
   constexpr uint32_t kIdescO = idesc_bf16_f32(kBM, kHeadDim, true);  // P V: MN-major B
@@ -486,50 +522,59 @@ __device__ void mma_role(const AttnParams<MAXR>& p, uint32_t sbase, uint32_t bar
   };
   const uint64_t dq[2] = {sdesc_sw128(sbase + Smem::kQ0, 16, 1024),
                           sdesc_sw128(sbase + Smem::kQ1, 16, 1024)};
-  int it = 0, nq = 0;   // ring items consumed, items
-  int npv[2] = {0, 0};  // P tiles consumed per Q tile (p_full phases)
+  int npv[2] = {0, 0};  // P tiles consumed per Q tile (P barrier phases)
+  int nq = 0;           // items started (Q barrier phases)
+  // The previous tile (its P V is issued in the next iteration).
+  bool has_prev = false, prev_pv[2] = {false, false}, prev_last[2] = {false, false};
+  bool prev_first[2] = {false, false};
+  int prev_stV = 0;
+  int t = 0;  // tiles of this CTA so far (ring items 2t, 2t+1)
+  auto issue_pv = [&](int w, int stV, bool first_of_item, bool last_of_item) {
+    const uint64_t dv = sdesc_sw128(sbase + Smem::kRing + stV * kTileBytes, kHalfBytes, 1024);
+    constexpr int kPer = (kBN / 16) / kPHalves;  // MMAs (K = 16 keys) per part of P
+#pragma unroll
+    for (int half = 0; half < kPHalves; ++half) {
+      if (!wait(Smem::bPFull + 2 * w + half, static_cast<uint32_t>(npv[w]) & 1u)) return;
+      tc_fence_after();
+      if (elect_one()) {
+#pragma unroll
+        for (int s = kPer * half; s < kPer * half + kPer; ++s)
+          mma_bf16_ts(tmem + col_o(w), tmem + col_s(w) + s * 8, dv + ((s * 2048) >> 4), kIdescO,
+                      (!first_of_item || s > 0) ? 1u : 0u);
+        if (half == kPHalves - 1 && last_of_item) mma_commit(bar(Smem::bOFull + w));
+      }
+      __syncwarp();
+    }
+    ++npv[w];
+  };
   for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x, ++nq) {
     const Item c = decode_item(p, item);
-    const bool act0 = tile_active(c, 0), act1 = tile_active(c, 1);
-    wait(Smem::bQFull + 0, static_cast<uint32_t>(nq) & 1u);
-    wait(Smem::bQFull + 1, static_cast<uint32_t>(nq) & 1u);
-    if (!ok) break;
-    tc_fence_after();
-    const int it0 = it;
-    BCA_TRACE_AT(p, it0 / 2, 26);
-    for (int j = c.j0; j <= c.j1 && ok; ++j) {
-      const int itK = it0 + 2 * (j - c.j0), itV = itK - 1;
-      const int stK = itK % kStages, stV = (itV + kStages) % kStages;
-      BCA_TRACE_AT(p, it0 / 2 + (j - c.j0), 21);
-      if (j < c.j1) wait(Smem::bKvFull + stK, static_cast<uint32_t>(itK / kStages) & 1u);
-      BCA_TRACE_AT(p, it0 / 2 + (j - c.j0), 22);
-      if (j > c.j0) wait(Smem::bKvFull + stV, static_cast<uint32_t>(itV / kStages) & 1u);
+    const bool act[2] = {tile_active(c, 0), tile_active(c, 1)};
+    for (int j = c.j0; j < c.j1 && ok; ++j, ++t) {
+      const int itK = 2 * t, itV = 2 * t - 1;
+      const int stK = itK % kStages;
+      BCA_TRACE_AT(p, t, 21);
+      wait(Smem::bKvFull + stK, static_cast<uint32_t>(itK / kStages) & 1u);
+      BCA_TRACE_AT(p, t, 22);
+      if (has_prev) wait(Smem::bKvFull + prev_stV, static_cast<uint32_t>(itV / kStages) & 1u);
+      if (j == c.j0) {
+        wait(Smem::bQFull + 0, static_cast<uint32_t>(nq) & 1u);
+        wait(Smem::bQFull + 1, static_cast<uint32_t>(nq) & 1u);
+        BCA_TRACE_AT(p, t, 26);
+      }
       if (!ok) break;
-      BCA_TRACE_AT(p, it0 / 2 + (j - c.j0), 0);
+      BCA_TRACE_AT(p, t, 0);
       tc_fence_after();
       const uint64_t dk = sdesc_sw128(sbase + Smem::kRing + stK * kTileBytes, 16, 1024);
-      const uint64_t dv = sdesc_sw128(sbase + Smem::kRing + stV * kTileBytes, kHalfBytes, 1024);
 #pragma unroll
       for (int w = 0; w < 2; ++w) {
-        if (!(w ? act1 : act0)) continue;
-        const int jend = w ? c.jend[1] : c.jend[0];
-        if (j > c.j0 && j - 1 < jend) {
-          // O_w += P_w(j-1) V_{j-1}; P must be consumed before S_w(j) overwrites it.
-          if (!wait(Smem::bPFull + w, static_cast<uint32_t>(npv[w]) & 1u)) break;
-          ++npv[w];
-          BCA_TRACE_AT(p, it0 / 2 + (j - c.j0), 1 + 2 * w);
-          tc_fence_after();
-          if (elect_one()) {
-#pragma unroll
-            for (int s = 0; s < kBN / 16; ++s)
-              mma_bf16_ts(tmem + col_o(w), tmem + col_s(w) + s * 8, dv + ((s * 2048) >> 4),
-                          kIdescO, (j - 1 > c.j0 || s > 0) ? 1u : 0u);
-            if (j == jend) mma_commit(bar(Smem::bOFull + w));
-          }
-          __syncwarp();
+        if (has_prev && prev_pv[w]) {
+          issue_pv(w, prev_stV, prev_first[w], prev_last[w]);
+          if (!ok) break;
+          BCA_TRACE_AT(p, t, 1 + 2 * w);
         }
-        if (j < jend) {
-          // S_w = Q_w K_j^T
+        const int jend = w ? c.jend[1] : c.jend[0];
+        if (act[w] && j < jend) {
           if (elect_one()) {
 #pragma unroll
             for (int s = 0; s < kHeadDim / 16; ++s) {
@@ -537,21 +582,41 @@ __device__ void mma_role(const AttnParams<MAXR>& p, uint32_t sbase, uint32_t bar
               mma_bf16_ss(tmem + col_s(w), dq[w] + koff, dk + koff, kIdescS, s > 0 ? 1u : 0u);
             }
             mma_commit(bar(Smem::bSFull + w));
+            // Last S_w of the item: Q tile w may be reloaded once this MMA is done.
+            if (j == jend - 1) mma_commit(bar(Smem::bQEmpty + w));
           }
           __syncwarp();
-          BCA_TRACE_AT(p, it0 / 2 + (j - c.j0), 2 + 2 * w);
+          BCA_TRACE_AT(p, t, 2 + 2 * w);
         }
       }
       if (!ok) break;
       if (elect_one()) {
-        if (j < c.j1) mma_commit(bar(Smem::bKvEmpty + stK));
-        if (j > c.j0) mma_commit(bar(Smem::bKvEmpty + stV));
-        // The last S MMA of the item has been issued: Q may be reloaded once it is done.
-        if (j == c.j1 - 1) mma_commit(bar(Smem::bQEmpty));
+        mma_commit(bar(Smem::bKvEmpty + stK));
+        if (has_prev) mma_commit(bar(Smem::bKvEmpty + prev_stV));
       }
       __syncwarp();
+      has_prev = true;
+      prev_stV = (2 * t + 1) % kStages;
+#pragma unroll
+      for (int w = 0; w < 2; ++w) {
+        const int jend = w ? c.jend[1] : c.jend[0];
+        prev_pv[w] = act[w] && j < jend;
+        prev_first[w] = j == c.j0;
+        prev_last[w] = j == jend - 1;
+      }
     }
-    it = it0 + 2 * (c.j1 - c.j0);
+  }
+  if (ok && has_prev) {
+    // The last tile's P V.
+    wait(Smem::bKvFull + prev_stV, static_cast<uint32_t>(2 * t - 1) / kStages & 1u);
+    if (ok) {
+      tc_fence_after();
+#pragma unroll
+      for (int w = 0; w < 2; ++w)
+        if (prev_pv[w] && ok) issue_pv(w, prev_stV, prev_first[w], prev_last[w]);
+      if (ok && elect_one()) mma_commit(bar(Smem::bKvEmpty + prev_stV));
+      __syncwarp();
+    }
   }
   // Everything issued must be complete before TMEM is released.
   if (elect_one()) mma_commit(bar(Smem::bDone));
@@ -574,7 +639,7 @@ __device__ void softmax_role(const AttnParams<MAXR>& p, int w, uint32_t bars, ui
   const uint32_t tO = tmem + lane_off + col_o(w);
   const bool prefill = p.mode == kModePrefill;
   const int seq_len = p.seq_len;
-  const uint32_t b_s = bar(Smem::bSFull + w), b_p = bar(Smem::bPFull + w);
+  const uint32_t b_s = bar(Smem::bSFull + w);
   const uint32_t b_o = bar(Smem::bOFull + w);
   int ns = 0, no = 0;  // S tiles and O results consumed (barrier phases)
   for (int item = blockIdx.x; item < p.n_items; item += gridDim.x) {
@@ -649,39 +714,8 @@ __device__ void softmax_role(const AttnParams<MAXR>& p, int w, uint32_t bars, ui
         m_run = m_new;
       }
       const float neg_m = (cache_tile ? lg_vs : 0.f) - m_run;
-      // p = 2^(s * sl2 - m) on column pairs: packed fp32x2 FMA for the exponent,
-      // then MUFU ex2 for most pairs and the FMA-pipe polynomial for kPolyPairs of
-      // every 8 (balances the two pipes); P is packed to bf16 in place over S.
-      const uint64_t sl2x2 = f2_pack(sl2, sl2), negm2 = f2_pack(neg_m, neg_m);
-      uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
-#pragma unroll
-      for (int cc = 0; cc < 64; ++cc) {
-        const uint64_t x =
-            f2_fma(f2_pack(__uint_as_float(r[2 * cc]), __uint_as_float(r[2 * cc + 1])), sl2x2,
-                   negm2);
-        uint64_t pp;
-        if ((cc & 7) >= 8 - kPolyPairs) {
-          pp = exp2_poly2(x);
-        } else {
-          float x0, x1;
-          f2_unpack(x, x0, x1);
-          pp = f2_pack(ex2_approx(x0), ex2_approx(x1));
-        }
-        acc[cc & 3] = f2_add(acc[cc & 3], pp);
-        float p0, p1;
-        f2_unpack(pp, p0, p1);
-        r[cc] = pack_bf16x2(p0, p1);
-      }
-      float a0, a1, b0, b1;
-      f2_unpack(f2_add(acc[0], acc[1]), a0, a1);
-      f2_unpack(f2_add(acc[2], acc[3]), b0, b1);
-      const float tile_sum = (a0 + a1) + (b0 + b1);
-      l_run += cache_tile ? tile_sum * inv_vs : tile_sum;
-      if (tr) BCA_TRACE_AT(p, ns, 8 + 5 * w);
-      tmem_st_32x32b_x32(tS, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
-      tmem_st_32x32b_x32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
-      // O was last written by P(j-1) V_{j-1}, complete before S(j) was signalled; it
-      // must be rescaled before P(j) V_j is issued (that waits for our arrival).
+      // O was last written by P(j-1) V(j-1), complete before S(j) was signalled; it
+      // is rescaled before the first half of P(j) is handed over (P(j) V(j) waits).
       if (j > c.j0 && __any_sync(0xffffffffu, need)) {
         const uint64_t f2 = f2_pack(f, f);
 #pragma unroll
@@ -700,9 +734,47 @@ __device__ void softmax_role(const AttnParams<MAXR>& p, int w, uint32_t bars, ui
           tmem_st_32x32b_x16(tO + 16 * cc, o);
         }
       }
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(b_p);
+      // p = 2^(s * sl2 - m) on column pairs: packed fp32x2 FMA for the exponent,
+      // then MUFU ex2 for most pairs and the FMA-pipe polynomial for kPolyPairs of
+      // every 8 (balances the two pipes); P is packed to bf16 in place over S and
+      // handed to the MMA in two halves of 64 keys.
+      const uint64_t sl2x2 = f2_pack(sl2, sl2), negm2 = f2_pack(neg_m, neg_m);
+      uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+#pragma unroll
+        for (int cc = 32 * half; cc < 32 * half + 32; ++cc) {
+          const uint64_t x =
+              f2_fma(f2_pack(__uint_as_float(r[2 * cc]), __uint_as_float(r[2 * cc + 1])), sl2x2,
+                     negm2);
+          uint64_t pp;
+          if (kExpF16) {
+            pp = exp2_f16x2(x);
+          } else if ((cc & 7) >= 8 - kPolyPairs) {
+            pp = exp2_poly2(x);
+          } else {
+            float x0, x1;
+            f2_unpack(x, x0, x1);
+            pp = f2_pack(ex2_approx(x0), ex2_approx(x1));
+          }
+          acc[cc & 3] = f2_add(acc[cc & 3], pp);
+          float p0, p1;
+          f2_unpack(pp, p0, p1);
+          r[cc] = pack_bf16x2(p0, p1);
+        }
+        tmem_st_32x32b_x32(tS + 32 * half, *reinterpret_cast<uint32_t(*)[32]>(&r[32 * half]));
+        if (kPHalves == 2 || half == 1) {
+          tmem_wait_st();
+          tc_fence_before();
+          mbar_arrive(bar(Smem::bPFull + 2 * w + (kPHalves == 2 ? half : 0)));
+        }
+      }
+      float a0, a1, b0, b1;
+      f2_unpack(f2_add(acc[0], acc[1]), a0, a1);
+      f2_unpack(f2_add(acc[2], acc[3]), b0, b1);
+      const float tile_sum = (a0 + a1) + (b0 + b1);
+      l_run += cache_tile ? tile_sum * inv_vs : tile_sum;
+      if (tr) BCA_TRACE_AT(p, ns, 8 + 5 * w);
       if (tr) BCA_TRACE_AT(p, ns, 9 + 5 * w);
       if (trw) BCA_TRACE_AT(p, ns, 14 + 3 * w + warp);
     }
@@ -775,13 +847,18 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Smem::kTmemSlot);
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
+#ifdef BCA_TRACE
+  const long long t_start = clock64();
+#endif
 
   if (threadIdx.x == 0) {
     auto bar = [&](int i) { return bars + 8u * static_cast<uint32_t>(i); };
     for (int i = 0; i < 2; ++i) {
       mbar_init(bar(Smem::bQFull + i), 1);
+      mbar_init(bar(Smem::bQEmpty + i), 1);
       mbar_init(bar(Smem::bSFull + i), 1);
-      mbar_init(bar(Smem::bPFull + i), 128);
+      mbar_init(bar(Smem::bPFull + 2 * i), 128);
+      mbar_init(bar(Smem::bPFull + 2 * i + 1), 128);
       mbar_init(bar(Smem::bOFull + i), 1);
       mbar_init(bar(Smem::bStgFull + i), 1);
       mbar_init(bar(Smem::bStgEmpty + i), 1);
@@ -792,7 +869,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     }
     mbar_init(bar(Smem::bDone), 1);
     mbar_init(bar(Smem::bConv), kConvThreads);
-    mbar_init(bar(Smem::bQEmpty), 1);
     *abort = 0;
     fence_barrier_init();
   }
@@ -830,6 +906,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
+#ifdef BCA_TRACE
+  // Whole-CTA cycle count (cheap; independent of the per-tile trace).
+  if (threadIdx.x == 0 && p.trace && blockIdx.x < 1024)
+    p.trace[kTraceTiles * kTraceEvents + blockIdx.x] = clock64() - t_start;
+#endif
 }
 
 // ---------------------------------------------------------------------------

@@ -190,7 +190,8 @@ bca_status bca_selftest_exp2(const float* x, float* y_poly, float* y_mufu, int32
 /* Pipeline tracing (diagnostic; builds compiled with BCA_TRACE only, otherwise
  * BCA_ERR_UNSUPPORTED): attention launches enqueued afterwards record clock64()
  * stamps of CTA `cta`'s producer/MMA/softmax events into dev_buffer
-  * ([64 tiles][32 events] uint64, device, caller-owned); NULL turns it off. */
+ * ([192 tiles][32 events] uint64, device, caller-owned; cta < 0: none), followed by
+ * each CTA's total cycles (one uint64 per CTA, up to 1024 CTAs); NULL turns it off. */
 bca_status bca_debug_set_trace(unsigned long long* dev_buffer, int32_t cta);
 
 /* Library version string. */
