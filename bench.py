@@ -140,7 +140,7 @@ class Runner:
         self.cu = [0]
         for r in reqs:
             self.cu.append(self.cu[-1] + r.target)
-        seed_base = 1000 * rank
+        seed_base = rank_seed_base(rank)
         # per-layer prefill inputs (one per request) and per-layer cache slots
         self.pre = [[W.qkv(wl, l, 0, i, device) for i in range(len(reqs))] for l in range(layers)]
         if rank:
@@ -260,6 +260,28 @@ class E2ERunner:
                     self.h_out_step.copy_(r.o_step, non_blocking=True)
 
 
+def rank_seed_base(rank: int) -> int:
+    """Replicas: rank r draws its own requests (seed offset 1000*r); rank 0 uses the
+    workload's published seeds."""
+    return 1000 * rank
+
+
+def max_over_ranks(value: float, device=None) -> float:
+    """The slowest rank's time (all ranks take part; identity without a group)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(work_per_rank: float, n_ranks: int, steps: int, max_ms: float) -> float:
+    """Aggregate throughput: the work all ranks did over the slowest rank's time."""
+    return work_per_rank * n_ranks * steps / (max_ms / 1e3)
+
+
 def timed(fn, steps: int, warmup: int, dist_on: bool):
     import torch
     import torch.distributed as dist
@@ -278,9 +300,7 @@ def timed(fn, steps: int, warmup: int, dist_on: bool):
     torch.cuda.synchronize()
     ms = e0.elapsed_time(e1)
     if dist_on:
-        t = torch.tensor([ms], dtype=torch.float64, device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+        ms = max_over_ranks(ms, device="cuda")
         dist.barrier()
     return ms
 
@@ -392,7 +412,7 @@ def main():
     avg_step_ms = sum(step_ms) / len(step_ms)
     ms_per_step = ms / args.steps
     flops_total = runner.flops * n_gpus
-    value = flops_total * args.steps / (ms / 1e3) / 1e12
+    value = whole_job_rate(runner.flops, n_gpus, args.steps, ms) / 1e12
 
     peaks, peak_src = load_peaks()
     achieved = runner.flops_step_call / (avg_step_ms / 1e3) / 1e12
