@@ -593,6 +593,12 @@ __device__ void mma_role(const AttnParams<MAXR>& p, uint32_t sbase, uint32_t bar
       if (elect_one()) {
         mma_commit(bar(Smem::bKvEmpty + stK));
         if (has_prev) mma_commit(bar(Smem::bKvEmpty + prev_stV));
+        // A Q tile without rows in this item was loaded but is never read: release
+        // it at once (the producer reloads every Q tile for every item).
+        if (j == c.j0) {
+          if (!act[0]) mma_commit(bar(Smem::bQEmpty + 0));
+          if (!act[1]) mma_commit(bar(Smem::bQEmpty + 1));
+        }
       }
       __syncwarp();
       has_prev = true;
@@ -915,15 +921,18 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 
 // ---------------------------------------------------------------------------
 // Merge the split chunks of a unit: O = sum_c 2^(m_c - M) O_c / sum_c 2^(m_c - M) l_c.
-// One thread per (split unit, row); the grid covers n_split_units * 256 rows.
+// One warp per (split unit, row), one float4 of the row per lane: every chunk row is
+// read as one coalesced 512-byte segment.  8 rows per 256-thread block.
 // ---------------------------------------------------------------------------
 constexpr int kMaxSplit = 8;
+constexpr int kCombineRowsPerBlock = 8;
 
 template <int MAXR>
 __global__ void __launch_bounds__(256)
     attn_combine_kernel(const __grid_constant__ AttnParams<MAXR> p, int n_split_units) {
-  const int gid = blockIdx.x * blockDim.x + threadIdx.x;
-  const int su = gid / kChunkRows, r2 = gid % kChunkRows;
+  const int gw = blockIdx.x * kCombineRowsPerBlock + static_cast<int>(threadIdx.x / 32);
+  const int lane = threadIdx.x % 32;
+  const int su = gw / kChunkRows, r2 = gw % kChunkRows;
   if (su >= n_split_units) return;
   const int k = p.split_k;
   const Item c = decode_item(p, p.full_items + su * k);  // chunk 0 of the unit
@@ -936,43 +945,22 @@ __global__ void __launch_bounds__(256)
   const float* ws0 = p.workspace + static_cast<size_t>(su) * k * kStride;
   float M = -INFINITY;
   for (int ci = 0; ci < k; ++ci) M = fmaxf(M, ws0[ci * kStride + kChunkRows * kHeadDim + r2]);
-  float wgt[kMaxSplit];
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
   float L = 0.f;
-#pragma unroll
-  for (int ci = 0; ci < kMaxSplit; ++ci) {
-    wgt[ci] = 0.f;
-    if (ci < k) {
-      const float m = ws0[ci * kStride + kChunkRows * kHeadDim + r2];
-      const float l = ws0[ci * kStride + kChunkRows * kHeadDim + kChunkRows + r2];
-      wgt[ci] = ex2_approx(m - M);
-      L += wgt[ci] * l;
-    }
+  for (int ci = 0; ci < k; ++ci) {
+    const float* chunk = ws0 + ci * kStride;
+    const float wgt = ex2_approx(chunk[kChunkRows * kHeadDim + r2] - M);
+    L += wgt * chunk[kChunkRows * kHeadDim + kChunkRows + r2];
+    const float4 a =
+        reinterpret_cast<const float4*>(chunk + static_cast<size_t>(r2) * kHeadDim)[lane];
+    acc.x += wgt * a.x;
+    acc.y += wgt * a.y;
+    acc.z += wgt * a.z;
+    acc.w += wgt * a.w;
   }
   const float inv = 1.0f / L;
-  uint4* dst = reinterpret_cast<uint4*>(p.o + (static_cast<size_t>(grow) * p.heads + c.h) * kHeadDim);
-#pragma unroll 1
-  for (int e = 0; e < kHeadDim; e += 8) {
-    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-    for (int ci = 0; ci < kMaxSplit; ++ci) {
-      if (ci >= k) break;
-      const float4* src = reinterpret_cast<const float4*>(
-          ws0 + ci * kStride + static_cast<size_t>(r2) * kHeadDim + e);
-      const float4 a = src[0], b = src[1];
-      acc[0] += wgt[ci] * a.x;
-      acc[1] += wgt[ci] * a.y;
-      acc[2] += wgt[ci] * a.z;
-      acc[3] += wgt[ci] * a.w;
-      acc[4] += wgt[ci] * b.x;
-      acc[5] += wgt[ci] * b.y;
-      acc[6] += wgt[ci] * b.z;
-      acc[7] += wgt[ci] * b.w;
-    }
-    dst[e / 8] = make_uint4(pack_bf16x2(acc[0] * inv, acc[1] * inv),
-                            pack_bf16x2(acc[2] * inv, acc[3] * inv),
-                            pack_bf16x2(acc[4] * inv, acc[5] * inv),
-                            pack_bf16x2(acc[6] * inv, acc[7] * inv));
-  }
+  uint2* dst = reinterpret_cast<uint2*>(p.o + (static_cast<size_t>(grow) * p.heads + c.h) * kHeadDim);
+  dst[lane] = make_uint2(pack_bf16x2(acc.x * inv, acc.y * inv), pack_bf16x2(acc.z * inv, acc.w * inv));
 }
 
 }  // namespace bca

@@ -211,8 +211,9 @@ bca_status launch_attn(const AttnParams<MAXR>& p, int n_split_units, cudaStream_
   bca::attn_fwd_kernel<MAXR><<<grid, bca::kAttnThreads, bca::Smem::kDynamicBytes, stream>>>(p);
   if (cudaGetLastError() != cudaSuccess) return BCA_ERR_CUDA;
   if (n_split_units > 0) {
-    const int threads = 256, rows = n_split_units * bca::kChunkRows;
-    bca::attn_combine_kernel<MAXR><<<(rows + threads - 1) / threads, threads, 0, stream>>>(
+    const int rows = n_split_units * bca::kChunkRows;
+    const int blocks = (rows + bca::kCombineRowsPerBlock - 1) / bca::kCombineRowsPerBlock;
+    bca::attn_combine_kernel<MAXR><<<blocks, 32 * bca::kCombineRowsPerBlock, 0, stream>>>(
         p, n_split_units);
     if (cudaGetLastError() != cudaSuccess) return BCA_ERR_CUDA;
   }
@@ -553,3 +554,4 @@ extern "C" bca_status bca_selftest_exp2(const float* x, float* y_poly, float* y_
                          static_cast<cudaStream_t>(stream)>>>(x, y_poly, y_mufu, n);
   return cudaGetLastError() == cudaSuccess ? BCA_OK : BCA_ERR_CUDA;
 }
+

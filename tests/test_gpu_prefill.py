@@ -93,3 +93,14 @@ def test_full_size_sampled_rows(cuda_device, wl_index):
     rows = sample_rows(req.seq_len, 48, seed=wl_index, boundaries=req.offsets[1:-1])
     want = oracle.prefill(q, k, v, req.offsets, wl.scale, rows=rows)
     assert_parity(o[torch.from_numpy(rows).to(cuda_device)], want, what=wl.name)
+
+
+def test_many_items_per_cta_with_half_empty_q_pairs(cuda_device):
+    """S = 384: the second pair of every head has one 128-row tile and an empty one;
+    H = 256 gives 512 work items, several per CTA, so Q buffers are reused across
+    items that have an absent tile."""
+    blocks, H = [100, 284], 256
+    q, k, v, o = run(blocks, H, 31, cuda_device)
+    rows = sample_rows(384, 48, seed=5, boundaries=(100, 128, 256))
+    want = oracle.prefill(q, k, v, offsets(blocks), SCALE, rows=rows)
+    assert_parity(o[torch.from_numpy(rows).to(cuda_device)], want, what="half-empty pairs")

@@ -269,3 +269,19 @@ def test_workspace_too_small_means_no_split(cuda_device):
     o, _ = run_batch([req], H, cuda_device, workspace=tiny)
     rows = sample_rows(4096, 64, seed=3)
     assert_parity(o[torch.from_numpy(rows).to(cuda_device)], oracle_for(req, rows=rows))
+
+
+@pytest.mark.parametrize("mode", ["bf16", "fp8"])
+def test_many_items_per_cta_with_half_empty_q_pairs(cuda_device, mode):
+    """T = 128 per request: every unit has an empty second Q tile; H = 256 and two
+    requests give 512 items, several per CTA (with and without the split round)."""
+    H = 256
+    reqs = [make_request(128, 200, H, seed=980 + i, device=cuda_device, mode=mode)
+            for i in range(2)]
+    tol = REL_L2_FP8 if mode != "bf16" else 5e-3
+    for ws in (None, bca.step_workspace(cuda_device)):
+        o, cu = run_batch(reqs, H, cuda_device, workspace=ws)
+        for i, r in enumerate(reqs):
+            rows = sample_rows(128, 24, seed=i)
+            got = o[cu[i]:cu[i + 1]][torch.from_numpy(rows).to(cuda_device)]
+            assert_parity(got, oracle_for(r, rows=rows), rel_l2=tol, what=f"req {i}")
