@@ -555,3 +555,50 @@ extern "C" bca_status bca_selftest_exp2(const float* x, float* y_poly, float* y_
   return cudaGetLastError() == cudaSuccess ? BCA_OK : BCA_ERR_CUDA;
 }
 
+// ---------------------------------------------------------------------------
+// bca_step_attend_noalloc: the cached step for callers that cannot allocate device
+// memory.  Its split-chunk scratch is a file-scope device array instead of a
+// caller-provided workspace; the GPU holds the array for as long as the library is
+// loaded.
+// ---------------------------------------------------------------------------
+namespace {
+// Capacity in split chunks (256 rows x (128 + 2) fp32 each): 160 x 133,120 B
+// = 21.3 MB.  A split schedule uses at most one chunk per SM.
+constexpr size_t kNoAllocChunks = 160;
+constexpr size_t kNoAllocBytes = kNoAllocChunks * bca::kChunkBytes;
+static __device__ __align__(256) float g_noalloc_scratch[kNoAllocBytes / sizeof(float)];
+
+// Device address of g_noalloc_scratch on the current device.  Host code must not
+// use the symbol itself (that is a host-side stand-in, not a device address); the
+// address is looked up once per device, with that device current, and cached.
+bool noalloc_scratch_ptr(void** out) {
+  static std::mutex mu;
+  static std::vector<void*> ptrs;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return false;
+  std::lock_guard<std::mutex> lk(mu);
+  if (ptrs.size() <= static_cast<size_t>(dev)) ptrs.resize(dev + 1, nullptr);
+  if (!ptrs[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return false;
+    ptrs[dev] = p;
+  }
+  *out = ptrs[dev];
+  return true;
+}
+}  // namespace
+
+extern "C" bca_status bca_step_attend_noalloc(const void* q_t, const void* k_t, const void* v_t,
+                                              void* o_t, const int32_t* cu_target,
+                                              const bca_kv_slot* slots, int32_t n_req,
+                                              int32_t heads, int32_t head_dim, float scale,
+                                              int32_t* dev_status, void* stream) {
+  // The largest split schedule needs one chunk per SM.
+  const int sms = sm_count();
+  if (sms <= 0) return BCA_ERR_CUDA;
+  if (static_cast<size_t>(sms) > kNoAllocChunks) return BCA_ERR_CAPACITY;
+  void* scratch = nullptr;
+  if (!noalloc_scratch_ptr(&scratch)) return BCA_ERR_CUDA;
+  return bca_step_attend(q_t, k_t, v_t, o_t, cu_target, slots, n_req, heads, head_dim, scale,
+                         scratch, kNoAllocBytes, dev_status, stream);
+}

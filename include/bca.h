@@ -167,6 +167,27 @@ bca_status bca_step_attend(const void* q_t, const void* k_t, const void* v_t, vo
  * Without it (workspace NULL or too small for any chunk) nothing is split. */
 size_t bca_step_workspace_bytes(void);
 
+/* bca_step_attend for callers that cannot allocate device memory -- for example a
+ * serving process whose device memory is owned by another allocator, or one that
+ * reserves its whole memory budget at start-up and allows no allocation after it.
+ * The pages have no counterpart to this call; it is a library convenience.
+ * Same arguments and results as bca_step_attend without the workspace: the split
+ * chunks go to a scratch array that lives in the library itself (a file-scope
+ * device array of 160 chunks = 21.3 MB, held on every GPU that loads the library
+ * until the process exits).  The call allocates nothing.
+ *  - The first call on a device looks up the array's device address (once per
+ *    device, with that device current); make that first call before any stream
+ *    capture.
+ *  - Every call shares the one array and it keeps the previous call's contents.
+ *    Nothing in it needs to start at zero: each call writes every chunk it reads.
+ *    Calls that overlap on the GPU (other streams, other threads) race on it.
+ *  - Errors: as bca_step_attend; BCA_ERR_CAPACITY if the device has more SMs than
+ *    the array has chunks (a split schedule can use one chunk per SM). */
+bca_status bca_step_attend_noalloc(const void* q_t, const void* k_t, const void* v_t, void* o_t,
+                                   const int32_t* cu_target, const bca_kv_slot* slots,
+                                   int32_t n_req, int32_t heads, int32_t head_dim, float scale,
+                                   int32_t* dev_status, void* stream);
+
 /* Human-readable name of a status code (static storage). */
 const char* bca_status_string(bca_status status);
 
