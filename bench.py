@@ -212,52 +212,98 @@ class Runner:
 
 class E2ERunner:
     """The same step through the public calls with pinned host buffers: each call's
-    inputs are copied host->device and its output read back inside the timing."""
+    inputs are copied host->device and its output read back inside the timing.
+
+    Pipelined the way a serving loop would run it: host->device copies on one
+    stream, the library calls on the compute stream, device->host copies on a third,
+    with two device buffer sets so that the copies of neighbouring calls overlap the
+    kernels (and each other, on the two copy directions)."""
 
     def __init__(self, runner, host_sets: int = 2):
         import torch
+        self.torch = torch
         self.r = runner
         wl = runner.wl
         pin = lambda t: t.cpu().pin_memory()
-        self.h_pre = [[tuple(pin(x) for x in runner.pre[l % runner.layers][i])
-                       for i in range(len(wl.requests))] for l in range(host_sets)]
+        n = len(wl.requests)
+        self.h_pre = [[tuple(pin(x) for x in runner.pre[l % runner.layers][i]) for i in range(n)]
+                      for l in range(host_sets)]
         self.h_pool = [tuple(pin(x) for x in runner.pool[p]) for p in range(host_sets)]
-        self.d_pre = [tuple(torch.empty_like(x) for x in runner.pre[0][i])
-                      for i in range(len(wl.requests))]
-        self.d_step = tuple(torch.empty_like(x) for x in runner.pool[0])
-        self.h_out_pre = [torch.empty(x[0].shape, dtype=x[0].dtype).pin_memory()
-                          for x in self.d_pre]
-        self.h_out_step = torch.empty(self.d_step[0].shape, dtype=self.d_step[0].dtype).pin_memory()
+        self.d_pre = [[tuple(torch.empty_like(x) for x in runner.pre[0][i]) for i in range(n)]
+                      for _ in range(2)]
+        self.d_step = [tuple(torch.empty_like(x) for x in runner.pool[0]) for _ in range(2)]
+        self.o_pre = [[torch.empty_like(runner.pre[0][i][0]) for i in range(n)] for _ in range(2)]
+        self.o_step = [torch.empty_like(runner.pool[0][0]) for _ in range(2)]
+        self.h_out_pre = [[torch.empty(x.shape, dtype=x.dtype).pin_memory() for x in o]
+                          for o in self.o_pre]
+        self.h_out_step = [torch.empty(x.shape, dtype=x.dtype).pin_memory() for x in self.o_step]
+        self.s_h2d = torch.cuda.Stream()
+        self.s_d2h = torch.cuda.Stream()
+        self.ev = {k: [torch.cuda.Event(), torch.cuda.Event()] for k in ("h2d", "comp", "d2h")}
+        self.started = [False, False]
         layers, steps = runner.layers, wl.steps
-        self.h2d = (layers * sum(3 * x[0].numel() * 2 for x in self.d_pre)
-                    + layers * (steps - 1) * 3 * self.d_step[0].numel() * 2)
-        self.d2h = (layers * sum(x[0].numel() * 2 for x in self.d_pre)
-                    + layers * (steps - 1) * self.d_step[0].numel() * 2)
+        self.h2d = (layers * sum(3 * x[0].numel() * 2 for x in runner.pre[0])
+                    + layers * (steps - 1) * 3 * runner.pool[0][0].numel() * 2)
+        self.d2h = (layers * sum(x[0].numel() * 2 for x in runner.pre[0])
+                    + layers * (steps - 1) * runner.pool[0][0].numel() * 2)
+
+    def _call(self, b, host_in, dev_in, launch, dev_out, host_out):
+        torch, ev = self.torch, self.ev
+        comp = torch.cuda.current_stream()
+        if self.started[b]:
+            self.s_h2d.wait_event(ev["comp"][b])  # inputs of buffer set b are free
+        with torch.cuda.stream(self.s_h2d):
+            for d, h in zip(dev_in, host_in):
+                d.copy_(h, non_blocking=True)
+            ev["h2d"][b].record()
+        comp.wait_event(ev["h2d"][b])
+        if self.started[b]:
+            comp.wait_event(ev["d2h"][b])  # output of buffer set b has been read back
+        launch()
+        ev["comp"][b].record()
+        self.s_d2h.wait_event(ev["comp"][b])
+        with torch.cuda.stream(self.s_d2h):
+            for h, d in zip(host_out, dev_out):
+                h.copy_(d, non_blocking=True)
+            ev["d2h"][b].record()
+        self.started[b] = True
 
     def step(self):
+        torch = self.torch
         bca, r, wl = self.r.bca, self.r, self.r.wl
         r.epoch += 1
+        comp = torch.cuda.current_stream()
+        start = torch.cuda.Event()
+        start.record()
+        self.s_h2d.wait_event(start)
+        b = 0
         for s in range(wl.steps):
             for l in range(r.layers):
                 if s == 0:
                     for i, req in enumerate(wl.requests):
-                        hq, hk, hv = self.h_pre[l % len(self.h_pre)][i]
-                        q, k, v = self.d_pre[i]
-                        q.copy_(hq, non_blocking=True)
-                        k.copy_(hk, non_blocking=True)
-                        v.copy_(hv, non_blocking=True)
-                        bca.prefill(q, k, v, r.o_pre[i], req.offsets, wl.scale,
-                                    slot=r.slots[l][i], epoch=r.epoch, dev_status=r.status)
-                        self.h_out_pre[i].copy_(r.o_pre[i], non_blocking=True)
+                        q, k, v = self.d_pre[b][i]
+                        o = self.o_pre[b][i]
+                        slot = r.slots[l][i]
+                        self._call(b, self.h_pre[l % len(self.h_pre)][i], (q, k, v),
+                                   lambda q=q, k=k, v=v, o=o, req=req, slot=slot: bca.prefill(
+                                       q, k, v, o, req.offsets, wl.scale, slot=slot,
+                                       epoch=r.epoch, dev_status=r.status),
+                                   (o,), (self.h_out_pre[b][i],))
+                        b ^= 1
                 else:
-                    hq, hk, hv = self.h_pool[(l + s) % len(self.h_pool)]
-                    q, k, v = self.d_step
-                    q.copy_(hq, non_blocking=True)
-                    k.copy_(hk, non_blocking=True)
-                    v.copy_(hv, non_blocking=True)
-                    bca.step_attend(q, k, v, r.o_step, r.cu, r.slots[l], wl.scale,
-                                    workspace=r.workspace, dev_status=r.status)
-                    self.h_out_step.copy_(r.o_step, non_blocking=True)
+                    q, k, v = self.d_step[b]
+                    o = self.o_step[b]
+                    slots = r.slots[l]
+                    self._call(b, self.h_pool[(l + s) % len(self.h_pool)], (q, k, v),
+                               lambda q=q, k=k, v=v, o=o, slots=slots: bca.step_attend(
+                                   q, k, v, o, r.cu, slots, wl.scale, workspace=r.workspace,
+                                   dev_status=r.status),
+                               (o,), (self.h_out_step[b],))
+                    b ^= 1
+        # join: the step ends when the last read-back has landed
+        end = torch.cuda.Event()
+        end.record(self.s_d2h)
+        comp.wait_event(end)
 
 
 def rank_seed_base(rank: int) -> int:

@@ -21,7 +21,8 @@ def L():
 
 
 def declared_functions():
-    text = open(HEADER).read()
+    with open(HEADER) as f:
+        text = f.read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
     names = re.findall(r"\b(bca_[a-z0-9_]+)\s*\(", text)
     return sorted(set(names))

@@ -24,7 +24,9 @@ def _all_bf16_finite():
 
 
 def test_golden_special_values():
-    for line in open(GOLDEN):
+    with open(GOLDEN) as f:
+        lines = f.readlines()
+    for line in lines:
         line = line.strip()
         if not line or line.startswith("#"):
             continue

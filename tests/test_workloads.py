@@ -9,7 +9,9 @@ GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "token_arithmetic.txt
 
 def _golden():
     vals = {}
-    for line in open(GOLDEN):
+    with open(GOLDEN) as f:
+        lines = f.readlines()
+    for line in lines:
         line = line.strip()
         if line and not line.startswith("#"):
             k, v = line.split()
