@@ -66,9 +66,9 @@ constexpr float kRescaleThreshold = 8.0f;  // log2 units
 #define BCA_POLY_PAIRS 0
 #endif
 // Of every 8 column pairs, kPolyPairs are exponentiated on the FMA pipe by the
-// software exp2 (the rest by MUFU ex2).  Measured on B200 for the T2I cached step:
-// 0 -> 1104, 1 -> 1080, 2 -> 1061, 3 -> 1037, 4 -> 1029 TFLOP/s (the softmax is
-// issue-bound, not MUFU-bound), so the default is 0.
+// software exp2 (the rest by MUFU ex2).  Measured on B200 for the T2I cached step
+// (kernel alone, TFLOP/s, two runs each in one process order): 0 -> 1145.7 / 1145.4,
+// 1 -> 1127.2 / 1126.5, 2 -> 1103.4; so the default is 0.
 constexpr int kPolyPairs = BCA_POLY_PAIRS;
 // P is handed from the softmax to the MMA in kPHalves parts (1: whole tile; 2: two
 // halves of 64 keys, so P V can start on the first half while the second is made).
