@@ -15,6 +15,11 @@ e2e    = the same through the Python/C-ABI calls with pinned HOST buffers: every
          the timed region.
 roofline: the dominant kernel (cached-step attention) against the measured
          dense bf16 tensor peak; cpu_baseline: the fp64 oracle on the host cores.
+qk_norm_rope = the Q/K RMS norm + rotary embedding call on the cached step's
+         target rows, GB/s against the measured HBM copy bandwidth.
+graph  = the same pass with each step's cached-step calls of all layers replayed
+         from one CUDA graph (bca_step_graph; one graph per assignment of input
+         buffers to layers); the prefill stays eager.
 
 Inputs: seeded synthetic bf16 N(0,1) (see block_causal_attention_dit_b200.workloads);
 per-layer prefill inputs; cached-step inputs cycle through a pool of distinct
@@ -55,6 +60,31 @@ def prefill_flops(req, H, d=128) -> float:
 
 def step_flops(req, H, d=128) -> float:
     return 4.0 * d * H * req.target * (req.prefix + req.target)
+
+
+# DRAM traffic of one cached-step attention launch (dram__bytes_read.sum +
+# dram__bytes_write.sum) from the ncu capture summarised in
+# profiles/attn_fwd_cached_step_t2i1024.md, valid only for the kernel sources it was
+# taken from (their sha256 below); any later change reports null instead.
+ATTN_TRAFFIC = {"bytes_per_launch": 109.33e6 + 13.79e6, "workload": 1,
+                "sources": {"block_causal_attention_dit_b200/csrc/attn_kernel.cuh":
+                            "a0dfc044881073dc60933061f04c88d7f946a50a3168e0483962686bca8a4e1d",
+                            "block_causal_attention_dit_b200/csrc/ptx.cuh":
+                            "0a502641c086d1c990ea14655d28721c277848084e0fb2dd1e0195c7b78ce88f"}}
+
+
+def measured_traffic(workload: int):
+    import hashlib
+    if workload != ATTN_TRAFFIC["workload"]:
+        return None
+    for rel, digest in ATTN_TRAFFIC["sources"].items():
+        try:
+            with open(os.path.join(ROOT, rel), "rb") as f:
+                if hashlib.sha256(f.read()).hexdigest() != digest:
+                    return None
+        except OSError:
+            return None
+    return ATTN_TRAFFIC["bytes_per_launch"]
 
 
 def load_peaks():
@@ -166,6 +196,7 @@ class Runner:
         self.workspace = bca.step_workspace(device)
         self.status = torch.zeros(1, dtype=torch.int32, device=device)
         self.epoch = 0
+        self.graphs = {}
         self.flops_prefill = sum(prefill_flops(r, H) for r in reqs) * layers
         self.flops_step_call = sum(step_flops(r, H) for r in reqs)
         self.flops_steps = self.flops_step_call * layers * (wl.steps - 1)
@@ -208,6 +239,43 @@ class Runner:
                     if events is not None:
                         e1.record()
                         events.append((e0, e1))
+
+
+    def graph_for_step(self, s):
+        """The StepGraph (all layers' cached-step calls) of step s >= 1: one graph per
+        assignment of pool entries to layers, built on first use."""
+        wl = self.wl
+        key = tuple((l * (wl.steps - 1) + s - 1) % len(self.pool) for l in range(self.layers))
+        g = self.graphs.get(key)
+        if g is None:
+            g = self.bca.StepGraph([self.pool[i][0] for i in key], [self.pool[i][1] for i in key],
+                                   [self.pool[i][2] for i in key], [self.o_step] * self.layers,
+                                   self.cu, self.slots, wl.scale, workspace=self.workspace,
+                                   dev_status=self.status)
+            self.graphs[key] = g
+        return g
+
+    def graph_step(self, events=None):
+        """The same pass with every cached step replayed from its StepGraph (the
+        prefill stays eager, as in the pages' engine)."""
+        import torch
+        bca, wl = self.bca, self.wl
+        self.epoch += 1
+        for l in range(self.layers):
+            for i, r in enumerate(wl.requests):
+                q, k, v = self.pre[l][i]
+                bca.prefill(q, k, v, self.o_pre[i], r.offsets, wl.scale, slot=self.slots[l][i],
+                            epoch=self.epoch, dev_status=self.status)
+        for s in range(1, wl.steps):
+            g = self.graph_for_step(s)
+            if events is not None:
+                e0 = torch.cuda.Event(enable_timing=True)
+                e1 = torch.cuda.Event(enable_timing=True)
+                e0.record()
+            g.launch()
+            if events is not None:
+                e1.record()
+                events.append((e0, e1))
 
 
 class E2ERunner:
@@ -328,6 +396,42 @@ def whole_job_rate(work_per_rank: float, n_ranks: int, steps: int, max_ms: float
     return work_per_rank * n_ranks * steps / (max_ms / 1e3)
 
 
+def norm_rope_leg(device, peaks, rows: int, heads: int, calls: int = 20):
+    """bca_qk_norm_rope on the cached step's target Q and K ([rows, H, 128] each):
+    GB/s on the algorithmic bytes (Q, K read and written once, cos/sin tables read
+    once) against the measured HBM copy bandwidth.  Four input sets (larger than
+    L2 together) are cycled so no call finds its data in L2."""
+    import numpy as np
+    import torch
+    import block_causal_attention_dit_b200 as bca
+    from block_causal_attention_dit_b200 import workloads as W
+    sets = [tuple(W.randn_bf16((rows, heads, 128), 90000 + 2 * i + j, device) for j in range(2))
+            for i in range(4)]
+    rng = np.random.default_rng(0)
+    gq, gk = (torch.from_numpy(rng.uniform(0.5, 1.5, 128).astype(np.float32)).to(device)
+              for _ in range(2))
+    ang = np.arange(rows)[:, None] * 10000.0 ** (-np.arange(64) / 64.0)
+    cos_t = torch.from_numpy(np.cos(ang).astype(np.float32)).to(device)
+    sin_t = torch.from_numpy(np.sin(ang).astype(np.float32)).to(device)
+    run = lambda i: bca.qk_norm_rope(sets[i % 4][0], sets[i % 4][1], gq, gk, cos_t, sin_t, 1e-6)
+    for i in range(4):
+        run(i)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for i in range(calls):
+        run(i)
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / calls
+    nbytes = 2 * rows * heads * 128 * 2 * 2 + 2 * rows * 64 * 4 + 2 * 128 * 4
+    gbs = nbytes / (ms / 1e3) / 1e9
+    peak = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    return {"bound": "hbm", "rows": rows, "heads": heads, "us_per_call": ms * 1e3,
+            "algorithmic_bytes": nbytes, "achieved": gbs, "peak": peak, "unit": "GB/s",
+            "frac": gbs / peak, "l2": "4 input sets cycled (536 MB for the T2I shape)"}
+
+
 def timed(fn, steps: int, warmup: int, dist_on: bool):
     import torch
     import torch.distributed as dist
@@ -393,6 +497,10 @@ def main():
     ap.add_argument("--pool", type=int, default=8)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-norm", action="store_true",
+                    help="skip the Q/K norm + rotary embedding leg")
+    ap.add_argument("--no-graph", action="store_true",
+                    help="skip the leg that replays the cached steps from CUDA graphs")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     args = ap.parse_args()
 
@@ -469,7 +577,32 @@ def main():
                 "frac": achieved / peak_sus, "peak_kind": f"bf16 sustained ({peak_src})",
                 "frac_of_burst_peak": achieved / peak_burst, "peak_burst": peak_burst,
                 "flops_per_launch": runner.flops_step_call, "avg_launch_ms": avg_step_ms,
-                "traffic": None}
+                "traffic": measured_traffic(args.workload),
+                "traffic_unit": "bytes per launch (ncu dram read + write)"}
+
+    graph = None
+    if not args.no_graph:
+        # The same pass with the cached steps of all layers replayed from one CUDA
+        # graph per layout (bca_step_graph); outputs are bit-identical to eager.
+        for _ in range(args.warmup):
+            runner.graph_step()
+        torch.cuda.synchronize()
+        gev = []
+        g_ms = timed(lambda: runner.graph_step(gev), args.steps, 0, dist_on)
+        if int(runner.status.item()) != 0:
+            raise RuntimeError(f"device status {int(runner.status.item())} (graph leg)")
+        g_launch_ms = sum(a.elapsed_time(b) for a, b in gev) / len(gev)
+        nodes = [g.kernel_nodes for g in runner.graphs.values()]
+        graph = {"value": whole_job_rate(runner.flops, n_gpus, args.steps, g_ms) / 1e12,
+                 "unit": "TFLOP/s", "ms_per_40step_attn": g_ms / args.steps,
+                 "cached_step_tflops": runner.flops_step_call * layers / (g_launch_ms / 1e3) / 1e12,
+                 "eager_cached_step_tflops": achieved,
+                 "ms_per_graph_launch": g_launch_ms, "layers_per_graph": layers,
+                 "graphs": len(nodes), "kernel_nodes_per_graph": max(nodes)}
+
+    norm = None
+    if not args.no_norm:
+        norm = norm_rope_leg(device, peaks, sum(r.target for r in wl.requests), wl.heads)
 
     e2e = None
     if not args.no_e2e:
@@ -493,10 +626,13 @@ def main():
             "pct_of_bf16_peak": {"sustained": 100 * achieved / peak_sus,
                                  "burst": 100 * achieved / peak_burst, "source": peak_src},
             "prefill_and_store_ms_per_step": ms_per_step - sum(step_ms) / args.steps,
-            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "graph": graph,
+            "qk_norm_rope": norm,
             "gpu_launches": runner.launches_per_step * args.steps, "clocks": clocks}
     if rank == 0:
         print(json.dumps(line), flush=True)
+    for g in runner.graphs.values():
+        g.close()
     if dist_on:
         dist.barrier()
         dist.destroy_process_group()

@@ -11,6 +11,11 @@ three calls of the method mirror include/bca.h one to one:
   step_attend(q_t, k_t, v_t, o_t, cu_target, slots, scale)
       cached-step attention of packed target rows over [cache ; own K/V] for a
       ragged batch of requests at the same phase.
+  qk_norm_rope(q, k, gamma_q, gamma_k, cos_t, sin_t, eps)
+      Q/K RMS norm + rotary embedding of the rows entering attention (in place).
+  StepGraph(q_layers, k_layers, v_layers, o_layers, cu_target, slots_per_layer, scale)
+      the cached-step calls of every layer of one layout recorded as one CUDA graph;
+      .launch() replays them (bit-identical to the eager calls).
 
 This module only marshals arguments (device pointers, sizes, the current CUDA
 stream) into the C ABI: every step of the path runs in the library's kernels.
@@ -25,6 +30,7 @@ import os
 __all__ = [
     "BcaError", "KVSlot", "KV_BF16", "KV_FP8_V", "KV_FP8_KV", "MAX_BLOCKS", "MAX_BATCH",
     "lib", "prefill", "kv_store", "step_attend", "step_workspace", "step_workspace_bytes",
+    "StepGraph", "qk_norm_rope",
     "slot_bytes", "set_wait_timeout_ns",
     "selftest_wait_timeout", "selftest_exp2", "status_string", "version", "LIB_PATH",
 ]
@@ -49,6 +55,19 @@ class BcaError(RuntimeError):
     def __init__(self, status: int, where: str):
         self.status = int(status)
         super().__init__(f"{where}: {STATUS_NAMES.get(self.status, self.status)}")
+
+
+class StepGraphDesc(ctypes.Structure):
+    """Mirror of bca_step_graph_desc."""
+    _fields_ = [
+        ("n_layers", ctypes.c_int32),
+        ("q_t", ctypes.POINTER(ctypes.c_void_p)), ("k_t", ctypes.POINTER(ctypes.c_void_p)),
+        ("v_t", ctypes.POINTER(ctypes.c_void_p)), ("o_t", ctypes.POINTER(ctypes.c_void_p)),
+        ("slots", ctypes.c_void_p), ("cu_target", ctypes.POINTER(ctypes.c_int32)),
+        ("n_req", ctypes.c_int32), ("heads", ctypes.c_int32), ("head_dim", ctypes.c_int32),
+        ("scale", ctypes.c_float), ("workspace", ctypes.c_void_p),
+        ("workspace_bytes", ctypes.c_size_t), ("dev_status", ctypes.c_void_p),
+    ]
 
 
 class SlotStruct(ctypes.Structure):
@@ -101,6 +120,16 @@ def lib():
     L.bca_selftest_exp2.argtypes = [P, P, P, i32, P]
     L.bca_debug_set_trace.restype = ctypes.c_int
     L.bca_debug_set_trace.argtypes = [P, i32]
+    L.bca_qk_norm_rope.restype = ctypes.c_int
+    L.bca_qk_norm_rope.argtypes = [P, P, ctypes.c_int64, i32, i32, P, P, P, P, f32, P]
+    L.bca_step_graph_create.restype = ctypes.c_int
+    L.bca_step_graph_create.argtypes = [ctypes.POINTER(StepGraphDesc), ctypes.POINTER(P)]
+    L.bca_step_graph_launch.restype = ctypes.c_int
+    L.bca_step_graph_launch.argtypes = [P, P]
+    L.bca_step_graph_kernel_nodes.restype = i32
+    L.bca_step_graph_kernel_nodes.argtypes = [P]
+    L.bca_step_graph_destroy.restype = None
+    L.bca_step_graph_destroy.argtypes = [P]
     L.bca_version.restype = ctypes.c_char_p
     L.bca_version.argtypes = []
     _lib = L
@@ -248,6 +277,77 @@ def step_attend(q_t, k_t, v_t, o_t, cu_target, slots, scale: float, workspace=No
                                  len(slots), H, d, float(scale), _ptr(workspace), ws_bytes,
                                  _ptr(dev_status), _stream(stream, q_t.device)),
            "bca_step_attend")
+
+
+def qk_norm_rope(q, k, gamma_q, gamma_k, cos_t, sin_t, eps: float = 1e-6, stream=None):
+    """In place on q and/or k ([rows, H, 128] bf16 CUDA; either may be None):
+    RMS norm over the head dim with weights gamma_* ([128] fp32), then the rotary
+    embedding of channel pairs (2i, 2i+1) by the angles whose cos/sin are
+    cos_t[t, i], sin_t[t, i] ([rows, 64] fp32)."""
+    ref = q if q is not None else k
+    rows, H, d = ref.shape
+    _check(lib().bca_qk_norm_rope(_ptr(q), _ptr(k), rows, H, d, _ptr(gamma_q), _ptr(gamma_k),
+                                  _ptr(cos_t), _ptr(sin_t), float(eps),
+                                  _stream(stream, ref.device)), "bca_qk_norm_rope")
+
+
+class StepGraph:
+    """The cached-step attention of every layer of one layout as one CUDA graph.
+
+    q_layers..o_layers: per-layer packed target tensors [sum T_r, H, 128] (bf16,
+    CUDA); slots_per_layer: per-layer lists of KVSlot (one per request, in
+    cu_target order).  The buffers are read in place at every launch(): write new
+    contents into them between launches.  Keep them (and the slots) alive while the
+    graph exists; close() or garbage collection releases it."""
+
+    def __init__(self, q_layers, k_layers, v_layers, o_layers, cu_target, slots_per_layer,
+                 scale: float, workspace=None, dev_status=None):
+        n = len(q_layers)
+        assert n == len(k_layers) == len(v_layers) == len(o_layers) == len(slots_per_layer)
+        n_req = len(slots_per_layer[0])
+        assert all(len(sl) == n_req for sl in slots_per_layer)
+        _, H, d = q_layers[0].shape
+        self._keep = (list(q_layers), list(k_layers), list(v_layers), list(o_layers),
+                      [list(sl) for sl in slots_per_layer], workspace, dev_status)
+        ptrs = lambda ts: (ctypes.c_void_p * n)(*[t.data_ptr() for t in ts])
+        self._q, self._k, self._v, self._o = (ptrs(q_layers), ptrs(k_layers), ptrs(v_layers),
+                                              ptrs(o_layers))
+        self._slots = (SlotStruct * (n * n_req))(*[s.struct for sl in slots_per_layer for s in sl])
+        self._cu = _i32_array(cu_target)
+        desc = StepGraphDesc(
+            n, ctypes.cast(self._q, ctypes.POINTER(ctypes.c_void_p)),
+            ctypes.cast(self._k, ctypes.POINTER(ctypes.c_void_p)),
+            ctypes.cast(self._v, ctypes.POINTER(ctypes.c_void_p)),
+            ctypes.cast(self._o, ctypes.POINTER(ctypes.c_void_p)),
+            ctypes.cast(self._slots, ctypes.c_void_p), self._cu, n_req, H, d, float(scale),
+            None if workspace is None else workspace.data_ptr(),
+            0 if workspace is None else workspace.numel() * workspace.element_size(),
+            None if dev_status is None else dev_status.data_ptr())
+        self.device = q_layers[0].device
+        self._g = ctypes.c_void_p()
+        import torch
+        with torch.cuda.device(self.device):
+            _check(lib().bca_step_graph_create(ctypes.byref(desc), ctypes.byref(self._g)),
+                   "bca_step_graph_create")
+
+    @property
+    def kernel_nodes(self) -> int:
+        return int(lib().bca_step_graph_kernel_nodes(self._g))
+
+    def launch(self, stream=None):
+        _check(lib().bca_step_graph_launch(self._g, _stream(stream, self.device)),
+               "bca_step_graph_launch")
+
+    def close(self):
+        if getattr(self, "_g", None):
+            lib().bca_step_graph_destroy(self._g)
+            self._g = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
 
 
 def selftest_wait_timeout(dev_status, timeout_ns: int, stream=None):

@@ -4,6 +4,8 @@
 //   bca_prefill      step-1 block-causal attention (+ prefix K/V into a slot)
 //   bca_kv_store     prefix K/V cache layout, bf16 or OFP8 E4M3 with per-head scales
 //   bca_step_attend  cached-step target attention for a ragged same-phase batch
+// and around them: bca_qk_norm_rope (Q/K RMS norm + rotary embedding of the rows
+// entering attention) and bca_step_graph_* (all layers' cached steps as one graph).
 // Every step of the path runs in the kernels of attn_kernel.cuh and
 // kv_store_kernel.cuh; this file only checks arguments and enqueues them.
 #include <cuda.h>
@@ -21,6 +23,7 @@
 #include "../../include/bca.h"
 #include "attn_kernel.cuh"
 #include "kv_store_kernel.cuh"
+#include "qk_norm_rope_kernel.cuh"
 
 namespace {
 
@@ -189,11 +192,12 @@ int plan_items(AttnParams<MAXR>& p, int units, int grid, size_t ws_chunks, Tiles
   return rem;
 }
 
+// One-time (per device) kernel attributes; also run before a stream capture so that
+// no attribute call happens inside it.
 template <int MAXR>
-bca_status launch_attn(const AttnParams<MAXR>& p, int n_split_units, cudaStream_t stream) {
-  if (p.n_items <= 0) return BCA_OK;
+bool prepare_attn() {
   if (!ensure_smem_attr(bca::attn_fwd_kernel<MAXR>, bca::Smem::kDynamicBytes, attr_flags<MAXR>()))
-    return BCA_ERR_CUDA;
+    return false;
   // The kernel re-splits its launch registers between warpgroups (setmaxnreg); that
   // only works if the compiled register count provides the pool the split assumes.
   static std::once_flag regs_once;
@@ -204,7 +208,13 @@ bca_status launch_attn(const AttnParams<MAXR>& p, int n_split_units, cudaStream_
               static_cast<uint32_t>(a.numRegs) * bca::kAttnThreads >=
                   128u * (2u * bca::kSoftmaxRegs + bca::kOtherRegs);
   });
-  if (!regs_ok) return BCA_ERR_CUDA;
+  return regs_ok;
+}
+
+template <int MAXR>
+bca_status launch_attn(const AttnParams<MAXR>& p, int n_split_units, cudaStream_t stream) {
+  if (p.n_items <= 0) return BCA_OK;
+  if (!prepare_attn<MAXR>()) return BCA_ERR_CUDA;
   const int sms = sm_count();
   if (sms <= 0) return BCA_ERR_CUDA;
   const int grid = std::min(sms, p.n_items);
@@ -601,4 +611,124 @@ extern "C" bca_status bca_step_attend_noalloc(const void* q_t, const void* k_t, 
   if (!noalloc_scratch_ptr(&scratch)) return BCA_ERR_CUDA;
   return bca_step_attend(q_t, k_t, v_t, o_t, cu_target, slots, n_req, heads, head_dim, scale,
                          scratch, kNoAllocBytes, dev_status, stream);
+}
+
+// ---------------------------------------------------------------------------
+// Cached-step graphs: the launches of bca_step_attend for every layer of a fixed
+// layout, recorded once by stream capture and replayed with one graph launch.
+// ---------------------------------------------------------------------------
+struct bca_step_graph {
+  cudaGraph_t graph = nullptr;
+  cudaGraphExec_t exec = nullptr;
+  int device = -1;
+  int32_t kernel_nodes = 0;
+};
+
+extern "C" bca_status bca_step_graph_create(const bca_step_graph_desc* d, bca_step_graph** out) {
+  if (!d || !out) return BCA_ERR_INVALID_ARG;
+  *out = nullptr;
+  if (d->n_layers < 1 || d->n_layers > 4096 || !d->q_t || !d->k_t || !d->v_t || !d->o_t ||
+      !d->slots || !d->cu_target || d->n_req < 1 || d->n_req > BCA_MAX_BATCH)
+    return BCA_ERR_INVALID_ARG;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return BCA_ERR_CUDA;
+  if (!prepare_attn<1>() || !prepare_attn<8>() || !prepare_attn<64>() || sm_count() <= 0 ||
+      !get_encode())
+    return BCA_ERR_CUDA;
+  cudaStream_t cs = nullptr;
+  if (cudaStreamCreateWithFlags(&cs, cudaStreamNonBlocking) != cudaSuccess) return BCA_ERR_CUDA;
+  // Each layer's call checks its arguments before it records anything; the first
+  // failing layer ends the capture and its status is returned.
+  bca_status st = BCA_OK;
+  cudaGraph_t graph = nullptr;
+  if (cudaStreamBeginCapture(cs, cudaStreamCaptureModeThreadLocal) != cudaSuccess) {
+    st = BCA_ERR_CUDA;
+  } else {
+    for (int l = 0; l < d->n_layers && st == BCA_OK; ++l)
+      st = bca_step_attend(d->q_t[l], d->k_t[l], d->v_t[l], d->o_t[l], d->cu_target,
+                           d->slots + static_cast<size_t>(l) * d->n_req, d->n_req, d->heads,
+                           d->head_dim, d->scale, d->workspace, d->workspace_bytes,
+                           d->dev_status, cs);
+    if (cudaStreamEndCapture(cs, &graph) != cudaSuccess && st == BCA_OK) st = BCA_ERR_CUDA;
+  }
+  cudaStreamDestroy(cs);
+  auto* g = new bca_step_graph();
+  g->graph = graph;
+  g->device = dev;
+  if (st == BCA_OK && graph) {
+    size_t n = 0;
+    if (cudaGraphGetNodes(graph, nullptr, &n) != cudaSuccess) st = BCA_ERR_CUDA;
+    std::vector<cudaGraphNode_t> nodes(n);
+    if (st == BCA_OK && n > 0 && cudaGraphGetNodes(graph, nodes.data(), &n) != cudaSuccess)
+      st = BCA_ERR_CUDA;
+    for (size_t i = 0; st == BCA_OK && i < n; ++i) {
+      cudaGraphNodeType t;
+      if (cudaGraphNodeGetType(nodes[i], &t) != cudaSuccess) st = BCA_ERR_CUDA;
+      else if (t == cudaGraphNodeTypeKernel) ++g->kernel_nodes;
+    }
+    if (st == BCA_OK && n > 0 && cudaGraphInstantiate(&g->exec, graph, 0) != cudaSuccess)
+      st = BCA_ERR_CUDA;
+  } else if (st == BCA_OK) {
+    st = BCA_ERR_CUDA;
+  }
+  if (st != BCA_OK) {
+    bca_step_graph_destroy(g);
+    cudaGetLastError();  // clear a capture error so later calls see a clean state
+    return st;
+  }
+  *out = g;
+  return BCA_OK;
+}
+
+extern "C" bca_status bca_step_graph_launch(const bca_step_graph* g, void* stream) {
+  if (!g) return BCA_ERR_INVALID_ARG;
+  if (!g->exec) return BCA_OK;  // a layout without target rows records nothing
+  return cudaGraphLaunch(g->exec, static_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? BCA_OK
+             : BCA_ERR_CUDA;
+}
+
+extern "C" int32_t bca_step_graph_kernel_nodes(const bca_step_graph* g) {
+  return g ? g->kernel_nodes : 0;
+}
+
+extern "C" void bca_step_graph_destroy(bca_step_graph* g) {
+  if (!g) return;
+  if (g->exec) cudaGraphExecDestroy(g->exec);
+  if (g->graph) cudaGraphDestroy(g->graph);
+  delete g;
+}
+
+// ---------------------------------------------------------------------------
+// Q/K RMS norm + rotary embedding (in place)
+// ---------------------------------------------------------------------------
+extern "C" bca_status bca_qk_norm_rope(void* q, void* k, int64_t rows, int32_t heads,
+                                       int32_t head_dim, const float* gamma_q,
+                                       const float* gamma_k, const float* cos_t,
+                                       const float* sin_t, float eps, void* stream) {
+  if (head_dim != 128) return BCA_ERR_UNSUPPORTED;
+  if (rows < 0 || heads < 1 || heads > 256 || !(eps > 0.0f) || !std::isfinite(eps))
+    return BCA_ERR_INVALID_ARG;
+  if (rows == 0) return BCA_OK;
+  if (!q && !k) return BCA_ERR_INVALID_ARG;
+  if ((q && (!aligned16(q) || !gamma_q || !aligned16(gamma_q))) ||
+      (k && (!aligned16(k) || !gamma_k || !aligned16(gamma_k))) || !cos_t || !sin_t ||
+      !aligned16(cos_t) || !aligned16(sin_t))
+    return BCA_ERR_INVALID_ARG;
+  bca::QkNormRopeParams p{};
+  p.x[0] = static_cast<uint16_t*>(q);
+  p.x[1] = static_cast<uint16_t*>(k);
+  p.gamma[0] = gamma_q;
+  p.gamma[1] = gamma_k;
+  p.cos_t = cos_t;
+  p.sin_t = sin_t;
+  p.rows = rows;
+  p.heads = heads;
+  p.eps = eps;
+  const int sms = sm_count();
+  if (sms <= 0) return BCA_ERR_CUDA;
+  const int64_t want = (2 * rows + bca::kNormWarpsPerBlock - 1) / bca::kNormWarpsPerBlock;
+  const int blocks = static_cast<int>(std::min<int64_t>(want, static_cast<int64_t>(sms) * 8));
+  bca::qk_norm_rope_kernel<<<blocks, bca::kNormThreads, 0, static_cast<cudaStream_t>(stream)>>>(p);
+  return cudaGetLastError() == cudaSuccess ? BCA_OK : BCA_ERR_CUDA;
 }

@@ -188,6 +188,82 @@ bca_status bca_step_attend_noalloc(const void* q_t, const void* k_t, const void*
                                    int32_t n_req, int32_t heads, int32_t head_dim, float scale,
                                    int32_t* dev_status, void* stream);
 
+/* ---- Q/K normalisation + rotary embedding ------------------------------------
+ * "SGLang-Diffusion stöder Qwen-Image-2.1 på dag noll" (orcarouter.ai), section
+ * "Siffrorna, och vad de inte säger": a Q/K-norm change is among the steps around
+ * the DiT's attention.  The pages give no formula; the plain reading (RMS norm over
+ * the head dimension with one learned weight vector per tensor, then the rotary
+ * position embedding of consecutive channel pairs) is computed here, in one pass
+ * over each tensor, in place, for x in {q, k} ([rows, heads, 128] bf16):
+ *   r          = 1 / sqrt(mean_c x[t,h,c]^2 + eps)
+ *   y_c        = x[t,h,c] * r * gamma_x[c]
+ *   x'[t,h,2i]   = y_{2i} cos_t[t,i] - y_{2i+1} sin_t[t,i]
+ *   x'[t,h,2i+1] = y_{2i} sin_t[t,i] + y_{2i+1} cos_t[t,i]      (i < 64)
+ * in fp32 with one round-to-nearest-even to bf16.  The caller's cos/sin tables
+ * ([rows, 64] fp32, device) carry any position scheme (1-D or per-axis angles).
+ * Run it on the target rows before bca_step_attend (and on the whole sequence
+ * before bca_prefill).  q or k may be NULL (that tensor is left alone; not both).
+ * gamma_q / gamma_k: [128] fp32 device (the one for a NULL tensor is unused).
+ * Errors: BCA_ERR_UNSUPPORTED for head_dim != 128; BCA_ERR_INVALID_ARG for rows < 0,
+ * heads outside [1, 256], eps not finite and > 0, a NULL or non-16-byte-aligned
+ * pointer that is needed.  rows == 0 enqueues nothing (pointers unchecked). */
+bca_status bca_qk_norm_rope(void* q, void* k, int64_t rows, int32_t heads, int32_t head_dim,
+                            const float* gamma_q, const float* gamma_k, const float* cos_t,
+                            const float* sin_t, float eps, void* stream);
+
+/* ---- Cached-step graphs ----------------------------------------------------
+ * "Qwen-Image-2.1 + vLLM-Omni day-0", "vLLM-Omni's day-0 support" and "Serving
+ * architecture: the cross-step prefix KV cache": besides the prefix reuse, the
+ * step loop's kernel-launch cost is removed with CUDA graphs.  "Qwen/Qwen-Image-2.1"
+ * (recipes.vllm.ai), "CUDA graphs": fixed-shape denoising steps are captured, one
+ * entry per image layout (the pages' engine copies prefix K/V into static buffers
+ * first and runs quantised caches eagerly; here neither is needed).
+ *
+ * A step graph is the cached-step attention of n_layers layers for one layout: a
+ * fixed request set (cu_target), fixed activation buffers per layer and fixed
+ * cache slots per (layer, request).  bca_step_graph_create checks every layer's
+ * arguments exactly as bca_step_attend does and records, in layer order, the same
+ * kernel launches bca_step_attend would enqueue (each layer after the one before,
+ * since the layers share the workspace) into one CUDA graph; bca_step_graph_launch
+ * replays them all with one call.  At replay the kernels read the activation
+ * buffers and the slots' device memory in place: contents written into the same
+ * buffers between replays are used -- nothing is copied into static buffers -- and
+ * the outputs are bit-identical to the eager bca_step_attend calls on the same
+ * contents.  Pointers, row counts, slot shapes and n_tokens are fixed when the
+ * graph is created; another layout needs another graph.  bf16 and e4m3 caches are
+ * captured alike.  The graph object lives in host memory (the CUDA driver keeps
+ * its own copy of the recorded launches); the library allocates no device memory. */
+typedef struct bca_step_graph bca_step_graph; /* opaque */
+
+typedef struct {
+  int32_t n_layers;         /* >= 1 */
+  const void* const* q_t;   /* [n_layers] device pointers (host array), each as in */
+  const void* const* k_t;   /*   bca_step_attend: packed target rows [sum T_r, H, d] */
+  const void* const* v_t;
+  void* const* o_t;
+  const bca_kv_slot* slots; /* [n_layers * n_req] host array, layer-major (read at create) */
+  const int32_t* cu_target; /* [n_req + 1] host array, shared by the layers */
+  int32_t n_req, heads, head_dim;
+  float scale;
+  void* workspace;          /* as bca_step_attend (nullable), shared by the layers */
+  size_t workspace_bytes;
+  int32_t* dev_status;      /* nullable */
+} bca_step_graph_desc;
+
+/* Builds the graph on the current device.  Errors: BCA_ERR_INVALID_ARG for a NULL
+ * desc/graph or a bad array; otherwise the first failing layer's bca_step_attend
+ * status (nothing is created then); BCA_ERR_CUDA if capture or instantiation fails. */
+bca_status bca_step_graph_create(const bca_step_graph_desc* desc, bca_step_graph** graph);
+
+/* Enqueues one replay (all layers) on `stream` (of the graph's device). */
+bca_status bca_step_graph_launch(const bca_step_graph* graph, void* stream);
+
+/* Kernel launches one replay performs (attention + chunk-merge kernels). */
+int32_t bca_step_graph_kernel_nodes(const bca_step_graph* graph);
+
+/* Releases the graph (NULL is ignored).  No replay may be pending on the GPU. */
+void bca_step_graph_destroy(bca_step_graph* graph);
+
 /* Human-readable name of a status code (static storage). */
 const char* bca_status_string(bca_status status);
 

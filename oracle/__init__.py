@@ -13,7 +13,8 @@ torch bf16 / uint8 CPU tensors are accepted and viewed as such.
 Sources (cited by page title and section):
   "Qwen-Image-2.1 + vLLM-Omni day-0", "Serving architecture: the cross-step
   prefix KV cache"; "Qwen/Qwen-Image-2.1" (vLLM recipe), "Prefix KV cache";
-  OCP OFP8 specification, E4M3.
+  OCP OFP8 specification, E4M3; "SGLang-Diffusion stöder Qwen-Image-2.1 på dag
+  noll", "Siffrorna, och vad de inte säger" (the Q/K norm next to attention).
 """
 from __future__ import annotations
 
@@ -75,6 +76,10 @@ def _load():
         lib.bca_oracle_cached_step.argtypes = [P, P, P, i64, i64, i64, P, ctypes.c_int, P,
                                                P, ctypes.c_int, P, i64, i64, ctypes.c_double,
                                                P, i64, P, ctypes.c_int]
+        lib.bca_oracle_rms_norm.restype = None
+        lib.bca_oracle_rms_norm.argtypes = [P, i64, i64, P, ctypes.c_double, P]
+        lib.bca_oracle_rope.restype = None
+        lib.bca_oracle_rope.argtypes = [P, i64, i64, i64, P, P, P]
         lib.bca_oracle_max_threads.restype = ctypes.c_int
         lib.bca_oracle_max_threads.argtypes = []
         _lib = lib
@@ -196,3 +201,32 @@ def cached_step(q_t, k_t, v_t, k_cache, v_cache, P: int, scale: float, k_kind=KI
     if rc != 0:
         raise ValueError("oracle cached_step: bad arguments")
     return out
+
+
+def rms_norm(x, gamma, eps: float) -> np.ndarray:
+    """x: [..., d] bf16 (bits or tensor); gamma: [d] fp32.  fp64 result, same shape."""
+    xb = _bits16(x)
+    d = xb.shape[-1]
+    g = np.ascontiguousarray(gamma, dtype=np.float32)
+    assert g.shape == (d,)
+    y = np.empty(xb.shape, dtype=np.float64)
+    _load().bca_oracle_rms_norm(_ptr(xb), xb.size // d, d, _ptr(g), float(eps), _ptr(y))
+    return y
+
+
+def rope(y, cos_t, sin_t) -> np.ndarray:
+    """y: [rows, H, d] fp64; cos_t, sin_t: [rows, d/2] fp32.  Pair (2i, 2i+1) of row t
+    turned by the angle whose cos/sin are cos_t[t, i], sin_t[t, i]."""
+    y = np.ascontiguousarray(y, dtype=np.float64)
+    rows, H, d = y.shape
+    c = np.ascontiguousarray(cos_t, dtype=np.float32)
+    s = np.ascontiguousarray(sin_t, dtype=np.float32)
+    assert c.shape == (rows, d // 2) and s.shape == c.shape
+    out = np.empty_like(y)
+    _load().bca_oracle_rope(_ptr(y), rows, H, d, _ptr(c), _ptr(s), _ptr(out))
+    return out
+
+
+def qk_norm_rope(x, gamma, cos_t, sin_t, eps: float) -> np.ndarray:
+    """rope(rms_norm(x)) for x [rows, H, d] bf16: the exact (fp64) values."""
+    return rope(rms_norm(x, gamma, eps), cos_t, sin_t)

@@ -296,3 +296,45 @@ int bca_oracle_cached_step(const uint16_t* q_t, const uint16_t* k_t, const uint1
   }
   return 0;
 }
+
+/* ------------------------------------------------------------------------ */
+/* Q/K RMS norm and rotary embedding                                         */
+/* ------------------------------------------------------------------------ */
+/* "SGLang-Diffusion stöder Qwen-Image-2.1 på dag noll" (orcarouter.ai), section
+ * "Siffrorna, och vad de inte säger", names a Q/K-norm change next to the DiT's
+ * attention but gives no formula.  Reading taken: RMS norm over the head dimension
+ * with one weight vector per tensor, then the rotary embedding of consecutive
+ * channel pairs by caller-given angles (as cos/sin tables).  fp64 throughout; the
+ * fp32 weights and tables are widened exactly. */
+
+/* y[v, c] = x[v, c] / sqrt(mean_c' x[v, c']^2 + eps) * gamma[c], for n_vec vectors
+ * of d bf16 values each. */
+void bca_oracle_rms_norm(const uint16_t* x, int64_t n_vec, int64_t d, const float* gamma,
+                         double eps, double* y) {
+  for (int64_t v = 0; v < n_vec; ++v) {
+    double ss = 0.0;
+    for (int64_t c = 0; c < d; ++c) {
+      double e = bca_oracle_bf16_to_f64(x[v * d + c]);
+      ss += e * e;
+    }
+    double inv = 1.0 / sqrt(ss / (double)d + eps);
+    for (int64_t c = 0; c < d; ++c)
+      y[v * d + c] = bca_oracle_bf16_to_f64(x[v * d + c]) * inv * (double)gamma[c];
+  }
+}
+
+/* Rotate every pair (2i, 2i+1) of y [rows, H, d] by the angle of row t and pair i:
+ * out_{2i} = y_{2i} cos - y_{2i+1} sin, out_{2i+1} = y_{2i} sin + y_{2i+1} cos,
+ * with cos/sin [rows, d/2].  out may not alias y. */
+void bca_oracle_rope(const double* y, int64_t rows, int64_t H, int64_t d, const float* cos_t,
+                     const float* sin_t, double* out) {
+  for (int64_t t = 0; t < rows; ++t)
+    for (int64_t h = 0; h < H; ++h)
+      for (int64_t i = 0; i < d / 2; ++i) {
+        const double* a = y + (t * H + h) * d + 2 * i;
+        double* o = out + (t * H + h) * d + 2 * i;
+        double cs = (double)cos_t[t * (d / 2) + i], sn = (double)sin_t[t * (d / 2) + i];
+        o[0] = a[0] * cs - a[1] * sn;
+        o[1] = a[0] * sn + a[1] * cs;
+      }
+}

@@ -141,3 +141,49 @@ def test_step_attend_argument_errors(L):
 def test_selftest_wait_rejects_bad_bounds(L):
     assert L.bca_selftest_wait_timeout(None, 10_000_000, None) == 1
     assert L.bca_selftest_wait_timeout(FAKE, 10, None) == 1
+
+
+def test_step_graph_argument_errors(L):
+    """bca_step_graph_create rejects a malformed description before any CUDA call."""
+    cu = (ctypes.c_int32 * 2)(0, 128)
+    ptrs = (ctypes.c_void_p * 2)(FAKE.value, FAKE.value)
+    pp = ctypes.cast(ptrs, ctypes.POINTER(ctypes.c_void_p))
+    slots = (bca.SlotStruct * 2)(_slot(L), _slot(L))
+    good = dict(n_layers=2, q_t=pp, k_t=pp, v_t=pp, o_t=pp,
+                slots=ctypes.cast(slots, ctypes.c_void_p), cu_target=cu, n_req=1, heads=2,
+                head_dim=128, scale=0.1, workspace=None, workspace_bytes=0, dev_status=None)
+    out = ctypes.c_void_p()
+    create = lambda **kw: L.bca_step_graph_create(ctypes.byref(bca.StepGraphDesc(**dict(good, **kw))),
+                                                  ctypes.byref(out))
+    assert L.bca_step_graph_create(None, ctypes.byref(out)) == 1
+    assert L.bca_step_graph_create(ctypes.byref(bca.StepGraphDesc(**good)), None) == 1
+    assert create(n_layers=0) == 1
+    assert create(q_t=None) == 1
+    assert create(o_t=None) == 1
+    assert create(slots=None) == 1
+    assert create(cu_target=None) == 1
+    assert create(n_req=0) == 1
+    assert create(n_req=65) == 1
+    assert out.value is None
+    assert L.bca_step_graph_launch(None, None) == 1
+    assert L.bca_step_graph_kernel_nodes(None) == 0
+    L.bca_step_graph_destroy(None)
+
+
+def test_qk_norm_rope_argument_errors(L):
+    call = lambda **kw: L.bca_qk_norm_rope(kw.get("q", FAKE), kw.get("k", FAKE), kw.get("rows", 16),
+                                           kw.get("H", 2), kw.get("d", 128), kw.get("gq", FAKE),
+                                           kw.get("gk", FAKE), kw.get("c", FAKE), kw.get("s", FAKE),
+                                           kw.get("eps", 1e-6), None)
+    assert call(d=64) == 2
+    assert call(rows=-1) == 1
+    assert call(H=0) == 1
+    assert call(H=257) == 1
+    assert call(eps=0.0) == 1
+    assert call(eps=float("nan")) == 1
+    assert call(q=None, k=None) == 1
+    assert call(q=None, k=None, rows=0) == 0  # nothing to do
+    assert call(q=ctypes.c_void_p((1 << 24) + 8)) == 1  # misaligned
+    assert call(gq=None) == 1
+    assert call(k=None, gk=None, c=None) == 1
+    assert call(s=ctypes.c_void_p((1 << 24) + 4)) == 1
