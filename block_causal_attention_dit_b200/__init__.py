@@ -285,6 +285,8 @@ def qk_norm_rope(q, k, gamma_q, gamma_k, cos_t, sin_t, eps: float = 1e-6, stream
     embedding of channel pairs (2i, 2i+1) by the angles whose cos/sin are
     cos_t[t, i], sin_t[t, i] ([rows, 64] fp32)."""
     ref = q if q is not None else k
+    if ref is None:
+        raise BcaError(1, "bca_qk_norm_rope")
     rows, H, d = ref.shape
     _check(lib().bca_qk_norm_rope(_ptr(q), _ptr(k), rows, H, d, _ptr(gamma_q), _ptr(gamma_k),
                                   _ptr(cos_t), _ptr(sin_t), float(eps),

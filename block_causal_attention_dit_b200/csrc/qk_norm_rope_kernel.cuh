@@ -15,8 +15,8 @@
 // HBM-bound.  One warp per (tensor, row): the row's cos/sin (shared by its heads)
 // and the weights are loaded once; the two half-warps take alternate heads, 16
 // lanes per 256-byte head vector (16 bytes = 8 channels = 4 pairs each), and every
-// lane keeps kNormHeadsInFlight vectors' loads in flight before it reduces (a
-// 16-lane shuffle sum of squares per vector) and stores.  Warps take consecutive
+// lane issues kNormHeadsInFlight vectors' loads before it reduces (a 16-lane
+// shuffle sum of squares per vector) and stores.  Warps take consecutive
 // rows, so the loads of a warp cover whole 256-byte rows of the [rows, H, 128]
 // tensor.
 #pragma once
@@ -38,7 +38,12 @@ struct QkNormRopeParams {
 
 constexpr int kNormThreads = 256;
 constexpr int kNormWarpsPerBlock = kNormThreads / 32;
-constexpr int kNormHeadsInFlight = 4;  // per half-warp: 8 head vectors per warp in flight
+// Head vectors each half-warp loads before it reduces (2 per warp per slot).
+// Measured on B200, GB/s as a fraction of the HBM copy bandwidth, at 4096 / 32768
+// rows x 32 heads: 2 -> 0.76 / 0.93, 4 -> 0.68 / 0.87, 8 -> 0.59 / 0.75 (more
+// registers, fewer resident warps); a cp.async ring of 2-6 chunks per warp in
+// shared memory measured 0.63-0.77 / 0.72-0.86.
+constexpr int kNormHeadsInFlight = 2;
 
 __device__ __forceinline__ float lo_bf16(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float hi_bf16(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
