@@ -30,7 +30,7 @@ import os
 __all__ = [
     "BcaError", "KVSlot", "KV_BF16", "KV_FP8_V", "KV_FP8_KV", "MAX_BLOCKS", "MAX_BATCH",
     "lib", "prefill", "kv_store", "step_attend", "step_workspace", "step_workspace_bytes",
-    "StepGraph", "qk_norm_rope",
+    "StepGraph", "qk_norm_rope", "ulysses_pack", "ulysses_unpack",
     "slot_bytes", "set_wait_timeout_ns",
     "selftest_wait_timeout", "selftest_exp2", "status_string", "version", "LIB_PATH",
 ]
@@ -122,6 +122,9 @@ def lib():
     L.bca_debug_set_trace.argtypes = [P, i32]
     L.bca_qk_norm_rope.restype = ctypes.c_int
     L.bca_qk_norm_rope.argtypes = [P, P, ctypes.c_int64, i32, i32, P, P, P, P, f32, P]
+    for name in ("bca_ulysses_pack", "bca_ulysses_unpack"):
+        getattr(L, name).restype = ctypes.c_int
+        getattr(L, name).argtypes = [P, P, ctypes.c_int64, i32, i32, i32, P]
     L.bca_step_graph_create.restype = ctypes.c_int
     L.bca_step_graph_create.argtypes = [ctypes.POINTER(StepGraphDesc), ctypes.POINTER(P)]
     L.bca_step_graph_launch.restype = ctypes.c_int
@@ -291,6 +294,20 @@ def qk_norm_rope(q, k, gamma_q, gamma_k, cos_t, sin_t, eps: float = 1e-6, stream
     _check(lib().bca_qk_norm_rope(_ptr(q), _ptr(k), rows, H, d, _ptr(gamma_q), _ptr(gamma_k),
                                   _ptr(cos_t), _ptr(sin_t), float(eps),
                                   _stream(stream, ref.device)), "bca_qk_norm_rope")
+
+
+def ulysses_pack(x, send, n_ranks: int, stream=None):
+    """x [rows, H, 128] -> send [n_ranks, rows, H/n_ranks, 128] (block g for rank g)."""
+    rows, H, d = x.shape
+    _check(lib().bca_ulysses_pack(_ptr(x), _ptr(send), rows, H, d, int(n_ranks),
+                                  _stream(stream, x.device)), "bca_ulysses_pack")
+
+
+def ulysses_unpack(recv, x, n_ranks: int, stream=None):
+    """recv [n_ranks, rows, H/n_ranks, 128] (block g from rank g) -> x [rows, H, 128]."""
+    rows, H, d = x.shape
+    _check(lib().bca_ulysses_unpack(_ptr(recv), _ptr(x), rows, H, d, int(n_ranks),
+                                    _stream(stream, x.device)), "bca_ulysses_unpack")
 
 
 class StepGraph:

@@ -5,7 +5,9 @@
 //   bca_kv_store     prefix K/V cache layout, bf16 or OFP8 E4M3 with per-head scales
 //   bca_step_attend  cached-step target attention for a ragged same-phase batch
 // and around them: bca_qk_norm_rope (Q/K RMS norm + rotary embedding of the rows
-// entering attention) and bca_step_graph_* (all layers' cached steps as one graph).
+// entering attention), bca_step_graph_* (all layers' cached steps as one graph) and
+// bca_ulysses_pack/unpack (layouts around the all-to-all of head-sharded
+// sequence parallelism).
 // Every step of the path runs in the kernels of attn_kernel.cuh and
 // kv_store_kernel.cuh; this file only checks arguments and enqueues them.
 #include <cuda.h>
@@ -24,6 +26,7 @@
 #include "attn_kernel.cuh"
 #include "kv_store_kernel.cuh"
 #include "qk_norm_rope_kernel.cuh"
+#include "ulysses_kernel.cuh"
 
 namespace {
 
@@ -731,4 +734,41 @@ extern "C" bca_status bca_qk_norm_rope(void* q, void* k, int64_t rows, int32_t h
   const int blocks = static_cast<int>(std::min<int64_t>(want, static_cast<int64_t>(sms) * 8));
   bca::qk_norm_rope_kernel<<<blocks, bca::kNormThreads, 0, static_cast<cudaStream_t>(stream)>>>(p);
   return cudaGetLastError() == cudaSuccess ? BCA_OK : BCA_ERR_CUDA;
+}
+
+// ---------------------------------------------------------------------------
+// Ulysses re-sharding copies
+// ---------------------------------------------------------------------------
+namespace {
+template <bool kPack>
+bca_status ulysses_copy(const void* src, void* dst, int64_t rows, int32_t heads, int32_t hd,
+                        int32_t n_ranks, void* stream) {
+  if (hd != 128) return BCA_ERR_UNSUPPORTED;
+  if (rows < 0 || n_ranks < 1 || heads < 1 || heads > 256 || heads % n_ranks != 0)
+    return BCA_ERR_INVALID_ARG;
+  if (rows == 0) return BCA_OK;
+  if (!src || !dst || !aligned16(src) || !aligned16(dst)) return BCA_ERR_INVALID_ARG;
+  const int sms = sm_count();
+  if (sms <= 0) return BCA_ERR_CUDA;
+  const int64_t n = rows * heads * 16;
+  const int blocks = static_cast<int>(
+      std::min<int64_t>((n + bca::kUlyssesThreads - 1) / bca::kUlyssesThreads,
+                        static_cast<int64_t>(sms) * 8));
+  bca::ulysses_copy_kernel<kPack><<<blocks, bca::kUlyssesThreads, 0,
+                                    static_cast<cudaStream_t>(stream)>>>(
+      static_cast<const uint4*>(src), static_cast<uint4*>(dst), rows, heads, n_ranks);
+  return cudaGetLastError() == cudaSuccess ? BCA_OK : BCA_ERR_CUDA;
+}
+}  // namespace
+
+extern "C" bca_status bca_ulysses_pack(const void* x, void* send, int64_t rows_local,
+                                       int32_t heads, int32_t head_dim, int32_t n_ranks,
+                                       void* stream) {
+  return ulysses_copy<true>(x, send, rows_local, heads, head_dim, n_ranks, stream);
+}
+
+extern "C" bca_status bca_ulysses_unpack(const void* recv, void* x, int64_t rows_local,
+                                         int32_t heads, int32_t head_dim, int32_t n_ranks,
+                                         void* stream) {
+  return ulysses_copy<false>(recv, x, rows_local, heads, head_dim, n_ranks, stream);
 }

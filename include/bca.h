@@ -211,6 +211,28 @@ bca_status bca_qk_norm_rope(void* q, void* k, int64_t rows, int32_t heads, int32
                             const float* gamma_q, const float* gamma_k, const float* cos_t,
                             const float* sin_t, float eps, void* stream);
 
+/* ---- Head-sharded (Ulysses) sequence parallelism -----------------------------
+ * "Qwen/Qwen-Image-2.1" (recipes.vllm.ai), "Overview" and "Limitations": the
+ * engine's sequence parallelism is Ulysses; "SGLang-Diffusion stöder Qwen-Image-2.1
+ * på dag noll", "Hur en driftsättning faktiskt ser ut": Ulysses attention is a
+ * verified multi-GPU mode.  N ranks each hold rows_local rows of all H heads; one
+ * all-to-all (the caller's, e.g. NCCL) gives each rank all rows of H/N heads, the
+ * attention calls run on that head shard (cache slots hold the rank's H/N heads),
+ * and a second all-to-all returns O to the row shards.  These two copies lay the
+ * buffers out around the exchange (Hn = heads / n_ranks, d = head_dim = 128, bf16):
+ *   bca_ulysses_pack   : x[t, g*Hn + j, :] -> send[g, t, j, :]  (block g for rank g)
+ *   bca_ulysses_unpack : recv[g, t, j, :] -> x[t, g*Hn + j, :]  (block g from rank g)
+ * for t < rows_local.  A received Q/K/V buffer [N][rows_local][Hn][d] is already
+ * the [N*rows_local, Hn, d] layout the attention calls take.  x and the buffers
+ * must not overlap.  Errors: BCA_ERR_UNSUPPORTED for head_dim != 128;
+ * BCA_ERR_INVALID_ARG for rows_local < 0, n_ranks < 1, heads not a positive
+ * multiple of n_ranks (at most 256), NULL or non-16-byte-aligned pointers.
+ * rows_local == 0 enqueues nothing. */
+bca_status bca_ulysses_pack(const void* x, void* send, int64_t rows_local, int32_t heads,
+                            int32_t head_dim, int32_t n_ranks, void* stream);
+bca_status bca_ulysses_unpack(const void* recv, void* x, int64_t rows_local, int32_t heads,
+                              int32_t head_dim, int32_t n_ranks, void* stream);
+
 /* ---- Cached-step graphs ----------------------------------------------------
  * "Qwen-Image-2.1 + vLLM-Omni day-0", "vLLM-Omni's day-0 support" and "Serving
  * architecture: the cross-step prefix KV cache": besides the prefix reuse, the

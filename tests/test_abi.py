@@ -187,3 +187,17 @@ def test_qk_norm_rope_argument_errors(L):
     assert call(gq=None) == 1
     assert call(k=None, gk=None, c=None) == 1
     assert call(s=ctypes.c_void_p((1 << 24) + 4)) == 1
+
+
+def test_ulysses_copy_argument_errors(L):
+    for fn in (L.bca_ulysses_pack, L.bca_ulysses_unpack):
+        call = lambda **kw: fn(kw.get("a", FAKE), kw.get("b", FAKE), kw.get("rows", 16),
+                               kw.get("H", 32), kw.get("d", 128), kw.get("n", 4), None)
+        assert call(d=64) == 2
+        assert call(n=0) == 1
+        assert call(n=3) == 1  # 32 heads over 3 ranks
+        assert call(H=0) == 1
+        assert call(rows=-1) == 1
+        assert call(a=None) == 1
+        assert call(b=ctypes.c_void_p((1 << 24) + 8)) == 1
+        assert call(a=None, rows=0) == 0  # nothing to move
