@@ -123,6 +123,32 @@ def test_t2i_1024_sampled_rows(cuda_device):
     assert_parity(o[torch.from_numpy(rows).to(cuda_device)], want, what="t2i sampled")
 
 
+@pytest.mark.parametrize("wl_index", [2, 3])
+def test_full_size_cached_step_sampled_rows(cuda_device, wl_index):
+    """The 4-ref edit (text 512 + four refs, target 4096: 16864 cached keys) and
+    native-2K (text 1024 + ref 4096, target 16384) cached steps at full size, in the
+    benchmark's launch configuration (workspace, split last round), sampled target
+    rows x all heads plus KV-tile boundaries of the target +-1 (16 of them)."""
+    wl = W.workload(wl_index)
+    req = wl.requests[0]
+    P = req.prefix
+    q0, k0, v0 = W.qkv(wl, 2, 0, 0, cuda_device)
+    slot = bca.KVSlot(P, wl.heads)
+    bca.kv_store(k0, v0, P, slot, epoch=1)
+    q, k, v = W.qkv(wl, 2, 7, 0, cuda_device)
+    o = torch.empty_like(q)
+    ws = bca.step_workspace(cuda_device)
+    bca.step_attend(q, k, v, o, [0, q.shape[0]], [slot], wl.scale, workspace=ws)
+    torch.cuda.synchronize()
+    T = q.shape[0]
+    tiles = list(range(128, T, 128))
+    rows = sample_rows(T, 24, seed=10 + wl_index, boundaries=tiles[:: max(1, len(tiles) // 16)])
+    kc = k0[:P].permute(1, 0, 2).contiguous()
+    vc = v0[:P].permute(1, 0, 2).contiguous()
+    want = oracle.cached_step(q, k, v, kc, vc, P, wl.scale, rows=rows)
+    assert_parity(o[torch.from_numpy(rows).to(cuda_device)], want, what=f"{wl.name} cached step")
+
+
 def test_repeated_calls_are_deterministic(cuda_device):
     req = make_request(300, 200, 2, 55, cuda_device)
     a, _ = run_batch([req], 2, cuda_device)
