@@ -943,20 +943,36 @@ __global__ void __launch_bounds__(256)
   if (!BCA_CHECK(p.dev_status, grow < p.o_rows && c.h < p.heads, 5)) return;
   constexpr size_t kStride = kChunkBytes / 4;
   const float* ws0 = p.workspace + static_cast<size_t>(su) * k * kStride;
+  // Every load of every chunk is issued before any of them is used.
+  float m[kMaxSplit], l[kMaxSplit];
+  float4 a[kMaxSplit];
+#pragma unroll
+  for (int ci = 0; ci < kMaxSplit; ++ci) {
+    if (ci < k) {
+      const float* chunk = ws0 + ci * kStride;
+      m[ci] = chunk[kChunkRows * kHeadDim + r2];
+      l[ci] = chunk[kChunkRows * kHeadDim + kChunkRows + r2];
+      a[ci] = reinterpret_cast<const float4*>(chunk + static_cast<size_t>(r2) * kHeadDim)[lane];
+    } else {
+      m[ci] = -INFINITY;
+      l[ci] = 0.f;
+      a[ci] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+  }
   float M = -INFINITY;
-  for (int ci = 0; ci < k; ++ci) M = fmaxf(M, ws0[ci * kStride + kChunkRows * kHeadDim + r2]);
+#pragma unroll
+  for (int ci = 0; ci < kMaxSplit; ++ci) M = fmaxf(M, m[ci]);
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
   float L = 0.f;
-  for (int ci = 0; ci < k; ++ci) {
-    const float* chunk = ws0 + ci * kStride;
-    const float wgt = ex2_approx(chunk[kChunkRows * kHeadDim + r2] - M);
-    L += wgt * chunk[kChunkRows * kHeadDim + kChunkRows + r2];
-    const float4 a =
-        reinterpret_cast<const float4*>(chunk + static_cast<size_t>(r2) * kHeadDim)[lane];
-    acc.x += wgt * a.x;
-    acc.y += wgt * a.y;
-    acc.z += wgt * a.z;
-    acc.w += wgt * a.w;
+#pragma unroll
+  for (int ci = 0; ci < kMaxSplit; ++ci) {
+    if (ci >= k) break;
+    const float wgt = ex2_approx(m[ci] - M);
+    L += wgt * l[ci];
+    acc.x += wgt * a[ci].x;
+    acc.y += wgt * a[ci].y;
+    acc.z += wgt * a[ci].z;
+    acc.w += wgt * a[ci].w;
   }
   const float inv = 1.0f / L;
   uint2* dst = reinterpret_cast<uint2*>(p.o + (static_cast<size_t>(grow) * p.heads + c.h) * kHeadDim);
