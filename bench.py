@@ -66,9 +66,9 @@ def step_flops(req, H, d=128) -> float:
 # dram__bytes_write.sum) from the ncu capture summarised in
 # profiles/attn_fwd_cached_step_t2i1024.md, valid only for the kernel sources it was
 # taken from (their sha256 below); any later change reports null instead.
-ATTN_TRAFFIC = {"bytes_per_launch": 109.33e6 + 13.79e6, "workload": 1,
+ATTN_TRAFFIC = {"bytes_per_launch": 109.22e6 + 14.75e6, "workload": 1,
                 "sources": {"block_causal_attention_dit_b200/csrc/attn_kernel.cuh":
-                            "a0dfc044881073dc60933061f04c88d7f946a50a3168e0483962686bca8a4e1d",
+                            "3fd425854e076ff78aee8b5c15ad78ee5243f3eea3ad26b12658609b7a413ab5",
                             "block_causal_attention_dit_b200/csrc/ptx.cuh":
                             "0a502641c086d1c990ea14655d28721c277848084e0fb2dd1e0195c7b78ce88f"}}
 
