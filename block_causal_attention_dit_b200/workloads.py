@@ -15,7 +15,8 @@ Shapes (cited by page title and section):
   * --step-execution --max-num-seqs 8 batches requests at the same KV-cache
     phase -- recipe, "Online serving".
   * DiT: 32 layers -- "Qwen-Image-2.1: SGLang vs vLLM-Omni Measured on a Single
-    L20", introduction.  H = 32 heads of head_dim 128 is this build's reading.
+    L20", introduction.  H = 32 heads of head_dim 128 is a reading (the pages give no
+    head count).
 
 Inputs: bf16 <- fp32 N(0, 1) from torch.randn with a seeded torch.Generator on
 the target device, rounded to bf16 (RNE).  Seed of tensor t (q=0, k=1, v=2) of
