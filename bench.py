@@ -15,6 +15,8 @@ e2e    = the same through the Python/C-ABI calls with pinned HOST buffers: every
          the timed region.
 roofline: the dominant kernel (cached-step attention) against the measured
          dense bf16 tensor peak; cpu_baseline: the fp64 oracle on the host cores.
+kv_store = bca_kv_store of every request's prefix, GB/s on the algorithmic bytes
+         (and on the bytes moved) against the measured HBM copy bandwidth.
 qk_norm_rope = the Q/K RMS norm + rotary embedding call on the cached step's
          target rows, GB/s against the measured HBM copy bandwidth.
 graph  = the same pass with each step's cached-step calls of all layers replayed
@@ -432,6 +434,44 @@ def norm_rope_leg(device, peaks, rows: int, heads: int, calls: int = 20):
             "frac": gbs / peak, "l2": "4 input sets cycled (536 MB for the T2I shape)"}
 
 
+def store_leg(runner, peaks, reps: int = 5):
+    """bca_kv_store of every request's prefix (layer 0's inputs) into fresh slots of
+    the workload's cache dtype: GB/s on the algorithmic bytes (K and V prefix rows
+    read once, the cache written once, the scales) and on the bytes moved (an e4m3
+    tensor's prefix is read twice: absmax pass, then encode pass)."""
+    import torch
+    bca, wl, H = runner.bca, runner.wl, runner.H
+    dt = {"bf16": (2, 2), "fp8_v": (2, 1), "fp8": (1, 1)}[wl.kv_dtype]  # bytes of K, V codes
+    slots = [bca.KVSlot(max(r.prefix, 1), H, wl.kv_dtype, device=runner.device)
+             for r in wl.requests]
+    alg = moved = 0
+    for r in wl.requests:
+        n = r.prefix * H * 128
+        alg += 2 * n * 2 + n * (dt[0] + dt[1]) + (8 * H if wl.kv_dtype != "bf16" else 0)
+        moved += 2 * n * 2 + n * (dt[0] + dt[1]) + n * 2 * (int(dt[0] == 1) + int(dt[1] == 1))
+
+    def run(epoch):
+        for i, r in enumerate(wl.requests):
+            q, k, v = runner.pre[0][i]
+            bca.kv_store(k, v, r.prefix, slots[i], epoch)
+
+    run(1)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for i in range(reps):
+        run(2 + i)
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / reps
+    peak = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    gbs = alg / (ms / 1e3) / 1e9
+    return {"bound": "hbm", "kv_cache": wl.kv_dtype, "prefix_rows": [r.prefix for r in wl.requests],
+            "ms_per_store": ms, "algorithmic_bytes": alg, "achieved": gbs, "peak": peak,
+            "unit": "GB/s", "frac": gbs / peak, "moved_bytes": moved,
+            "moved_gbs": moved / (ms / 1e3) / 1e9}
+
+
 def timed(fn, steps: int, warmup: int, dist_on: bool):
     import torch
     import torch.distributed as dist
@@ -600,6 +640,8 @@ def main():
                  "ms_per_graph_launch": g_launch_ms, "layers_per_graph": layers,
                  "graphs": len(nodes), "kernel_nodes_per_graph": max(nodes)}
 
+    store = store_leg(runner, peaks)
+
     norm = None
     if not args.no_norm:
         norm = norm_rope_leg(device, peaks, sum(r.target for r in wl.requests), wl.heads)
@@ -627,7 +669,7 @@ def main():
                                  "burst": 100 * achieved / peak_burst, "source": peak_src},
             "prefill_and_store_ms_per_step": ms_per_step - sum(step_ms) / args.steps,
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "graph": graph,
-            "qk_norm_rope": norm,
+            "qk_norm_rope": norm, "kv_store": store,
             "gpu_launches": runner.launches_per_step * args.steps, "clocks": clocks}
     if rank == 0:
         print(json.dumps(line), flush=True)

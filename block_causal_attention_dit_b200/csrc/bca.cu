@@ -260,7 +260,8 @@ bca_status enqueue_kv_store(const void* k, const void* v, int32_t n_prefix, int6
   }
   const int64_t chunks = static_cast<int64_t>(n_prefix) * p.heads * 16;
   const int64_t want = (chunks + bca::kStoreThreads - 1) / bca::kStoreThreads;
-  const int grid = static_cast<int>(std::min<int64_t>(want, 148 * 8));
+  const int sms = std::max(sm_count(), 1);
+  const int grid = static_cast<int>(std::min<int64_t>(want, static_cast<int64_t>(sms) * 8));
   bca::kv_write_kernel<<<dim3(grid, 2), bca::kStoreThreads, 0, stream>>>(p);
   if (any_quant) bca::kv_scale_finalize_kernel<<<dim3(1, 2), 256, 0, stream>>>(p);
   return cudaGetLastError() == cudaSuccess ? BCA_OK : BCA_ERR_CUDA;
