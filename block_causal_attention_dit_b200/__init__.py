@@ -32,7 +32,8 @@ __all__ = [
     "lib", "prefill", "kv_store", "step_attend", "step_workspace", "step_workspace_bytes",
     "StepGraph", "qk_norm_rope", "ulysses_pack", "ulysses_unpack",
     "slot_bytes", "set_wait_timeout_ns",
-    "selftest_wait_timeout", "selftest_exp2", "status_string", "version", "LIB_PATH",
+    "selftest_wait_timeout", "selftest_exp2", "selftest_e4m3_division", "status_string",
+    "version", "LIB_PATH",
 ]
 
 # BCA_LIBRARY may name another build of the same library (e.g. the self-checking
@@ -116,6 +117,8 @@ def lib():
     L.bca_set_wait_timeout_ns.argtypes = [u64]
     L.bca_selftest_wait_timeout.restype = ctypes.c_int
     L.bca_selftest_wait_timeout.argtypes = [P, u64, P]
+    L.bca_selftest_e4m3_division.restype = ctypes.c_int
+    L.bca_selftest_e4m3_division.argtypes = [P, P]
     L.bca_selftest_exp2.restype = ctypes.c_int
     L.bca_selftest_exp2.argtypes = [P, P, P, i32, P]
     L.bca_debug_set_trace.restype = ctypes.c_int
@@ -373,6 +376,16 @@ def selftest_wait_timeout(dev_status, timeout_ns: int, stream=None):
     _check(lib().bca_selftest_wait_timeout(_ptr(dev_status), int(timeout_ns),
                                            _stream(stream, dev_status.device)),
            "bca_selftest_wait_timeout")
+
+
+def selftest_e4m3_division(device="cuda", stream=None):
+    """Pairs (bf16 x, bf16 amax) whose e4m3 code from the encoder's division differs
+    from the code of the correctly rounded x / (amax / 448) (0 expected)."""
+    import torch
+    n = torch.zeros(1, dtype=torch.int64, device=device)
+    _check(lib().bca_selftest_e4m3_division(_ptr(n), _stream(stream, n.device)),
+           "bca_selftest_e4m3_division")
+    return int(n.item())
 
 
 def selftest_exp2(x, stream=None):

@@ -559,6 +559,13 @@ __global__ void selftest_exp2_kernel(const float* x, float* y_poly, float* y_muf
 }
 }  // namespace
 
+extern "C" bca_status bca_selftest_e4m3_division(unsigned long long* mismatches, void* stream) {
+  if (!mismatches) return BCA_ERR_INVALID_ARG;
+  bca::e4m3_division_selftest_kernel<<<0x7F7F, 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      mismatches);
+  return cudaGetLastError() == cudaSuccess ? BCA_OK : BCA_ERR_CUDA;
+}
+
 extern "C" bca_status bca_selftest_exp2(const float* x, float* y_poly, float* y_mufu, int32_t n,
                                         void* stream) {
   if (n < 0 || (n > 0 && (!x || !y_poly || !y_mufu))) return BCA_ERR_INVALID_ARG;

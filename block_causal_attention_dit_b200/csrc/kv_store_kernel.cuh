@@ -82,6 +82,21 @@ __device__ __forceinline__ float scale_from_amax_bits(unsigned bits) {
   return amax == 0.0f ? 1.0f : __fdiv_rn(amax, 448.0f);
 }
 
+// x / s for the encoder, from y = RN(1/s): q = RN(x y), then one correction with the
+// exact residual x - q s (an FMA):  RN(q + (x - q s) y) -- the division scheme of
+// P. Markstein, "IA-64 and Elementary Functions: Speed and Precision" (2000), ch. 8.
+// For heads whose amax is below 2^-95 (bf16 bits < kFastDivMinBits) the reciprocal
+// and the residual leave the normal range, so those take the correctly rounded
+// division.  bca_selftest_e4m3_division checks that the resulting codes equal those
+// of the correctly rounded quotient for every bf16 amax and every bf16 |x| <= amax.
+constexpr unsigned kFastDivMinBits = 0x1000u;
+__device__ __forceinline__ float div_by_scale(float x, float s, float y, bool fast) {
+  if (!fast) return __fdiv_rn(x, s);
+  const float q = x * y;
+  const float r = fmaf(-q, s, x);
+  return copysignf(fmaf(r, y, q), x);  // s > 0: the quotient has x's sign (also for -0)
+}
+
 // Two fp32 -> packed e4m3x2, round to nearest even, saturate to +-448;
 // `lo` lands in bits [0, 8).
 __device__ __forceinline__ uint16_t e4m3x2_rn_satfinite(float lo, float hi) {
@@ -105,23 +120,34 @@ __global__ void __launch_bounds__(kStoreThreads) kv_write_kernel(KvStoreParams p
   for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total;
        i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
     const int c = static_cast<int>(i & 15);
-    const int64_t th = i >> 4;
-    const int h = static_cast<int>(th % p.heads);
-    const int64_t t = th / p.heads;
+    int h;
+    int64_t t;
+    if (total < (int64_t{1} << 31)) {  // 32-bit index arithmetic when it fits
+      const uint32_t th = static_cast<uint32_t>(i) >> 4;
+      t = th / static_cast<uint32_t>(p.heads);
+      h = static_cast<int>(th - static_cast<uint32_t>(t) * static_cast<uint32_t>(p.heads));
+    } else {
+      const int64_t th = i >> 4;
+      h = static_cast<int>(th % p.heads);
+      t = th / p.heads;
+    }
     const uint4 v = __ldg(reinterpret_cast<const uint4*>(src + t * p.row_stride + h * 128 + c * 8));
     const int64_t drow = static_cast<int64_t>(h) * p.cap + t;
     if (!quant) {
       reinterpret_cast<uint4*>(static_cast<uint16_t*>(dst) + drow * 128)[c] = v;
     } else {
-      const float s = scale_from_amax_bits(amax_bits[h]);
+      const unsigned ab = amax_bits[h];
+      const float s = scale_from_amax_bits(ab);
+      const float y = __frcp_rn(s);
+      const bool fast = ab >= kFastDivMinBits;
       const uint32_t w[4] = {v.x, v.y, v.z, v.w};
       uint32_t out[2];
 #pragma unroll
       for (int k = 0; k < 2; ++k) {
-        const uint16_t a = e4m3x2_rn_satfinite(__fdiv_rn(bf16_lo(w[2 * k]), s),
-                                               __fdiv_rn(bf16_hi(w[2 * k]), s));
-        const uint16_t b = e4m3x2_rn_satfinite(__fdiv_rn(bf16_lo(w[2 * k + 1]), s),
-                                               __fdiv_rn(bf16_hi(w[2 * k + 1]), s));
+        const uint16_t a = e4m3x2_rn_satfinite(div_by_scale(bf16_lo(w[2 * k]), s, y, fast),
+                                               div_by_scale(bf16_hi(w[2 * k]), s, y, fast));
+        const uint16_t b = e4m3x2_rn_satfinite(div_by_scale(bf16_lo(w[2 * k + 1]), s, y, fast),
+                                               div_by_scale(bf16_hi(w[2 * k + 1]), s, y, fast));
         out[k] = static_cast<uint32_t>(a) | (static_cast<uint32_t>(b) << 16);
       }
       reinterpret_cast<uint2*>(static_cast<uint8_t*>(dst) + drow * 128)[c] =
@@ -137,6 +163,28 @@ __global__ void kv_scale_finalize_kernel(KvStoreParams p) {
   float* sc = t ? p.scale[1] : p.scale[0];
   for (int h = threadIdx.x; h < p.heads; h += blockDim.x)
     sc[h] = scale_from_amax_bits(__float_as_uint(sc[h]));
+}
+
+// Self-check of div_by_scale as the encoder uses it: for every positive finite bf16
+// amax (blockIdx.x + 1 as magnitude bits) and every bf16 x with |x| <= amax, the e4m3
+// code of div_by_scale(x, s, RN(1/s), amax >= 2^-95) must equal the code of the
+// correctly rounded x / s.
+__global__ void __launch_bounds__(256) e4m3_division_selftest_kernel(unsigned long long* mismatch) {
+  const unsigned amax_bits = blockIdx.x + 1;  // 0x0001 .. 0x7F7F
+  const float s = scale_from_amax_bits(amax_bits);
+  const float y = __frcp_rn(s);
+  const float amax = __uint_as_float(amax_bits << 16);
+  unsigned long long bad = 0;
+  for (unsigned m = threadIdx.x; m <= amax_bits; m += blockDim.x) {
+    const float xp = __uint_as_float(m << 16);
+    if (!(xp <= amax)) continue;
+    const uint16_t want = e4m3x2_rn_satfinite(__fdiv_rn(xp, s), __fdiv_rn(-xp, s));
+    const bool fast = amax_bits >= kFastDivMinBits;
+    const uint16_t got =
+        e4m3x2_rn_satfinite(div_by_scale(xp, s, y, fast), div_by_scale(-xp, s, y, fast));
+    bad += want != got;
+  }
+  if (bad) atomicAdd(mismatch, bad);
 }
 
 }  // namespace bca

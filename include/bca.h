@@ -306,6 +306,13 @@ bca_status bca_selftest_wait_timeout(int32_t* dev_status, uint64_t timeout_ns, v
 bca_status bca_selftest_exp2(const float* x, float* y_poly, float* y_mufu, int32_t n,
                              void* stream);
 
+/* Self-check of the e4m3 encoder's division: for every positive finite bf16 amax
+ * and every bf16 x with |x| <= amax, counts (atomically adds to *mismatches, a
+ * device uint64 the caller zeroes) the pairs whose e4m3 code from the encoder's
+ * reciprocal-and-correction quotient differs from the code of the correctly rounded
+ * x / s (s = amax / 448).  Diagnostic only; 0 is expected. */
+bca_status bca_selftest_e4m3_division(unsigned long long* mismatches, void* stream);
+
 /* Pipeline tracing (diagnostic; builds compiled with BCA_TRACE only, otherwise
  * BCA_ERR_UNSUPPORTED): attention launches enqueued afterwards record clock64()
  * stamps of CTA `cta`'s producer/MMA/softmax events into dev_buffer

@@ -92,3 +92,32 @@ def test_empty_prefix_only_stamps(cuda_device):
     x = torch.zeros((1, 2, 128), dtype=torch.bfloat16, device=cuda_device)
     bca.kv_store(x, x, 0, slot, epoch=5)
     assert slot.n_tokens == 0 and slot.epoch == 5
+
+
+def test_fp8_heads_with_tiny_and_huge_amax_bit_exact(cuda_device):
+    """Heads whose absmax is below 2^-95 take the encoder's correctly rounded
+    division (the reciprocal would leave the normal range); a head near the top of
+    the bf16 range takes the fast one.  Bytes and scales equal the oracle's."""
+    P, H = 200, 4
+    base = randn_bf16((P, H, 128), 41, cuda_device).float()
+    base[::7, :, ::5] = -0.0  # negative zeros keep their sign in the codes (0x80)
+    factors = torch.tensor([2.0 ** -120, 2.0 ** -100, 1.0, 2.0 ** 100], device=cuda_device)
+    k = (base * factors[None, :, None]).to(torch.bfloat16)
+    v = (base.flip(0) * factors.flip(0)[None, :, None]).to(torch.bfloat16)
+    slot = bca.KVSlot(P, H, "fp8")
+    bca.kv_store(k, v, P, slot, epoch=1)
+    torch.cuda.synchronize()
+    for x, codes, scales in ((k, slot.k_view(), slot.k_scale_view()),
+                             (v, slot.v_view(), slot.v_scale_view())):
+        want_c, want_s = oracle.quantize_prefix(x.cpu(), P, P)
+        assert np.array_equal(codes.cpu().numpy(), want_c)
+        assert np.array_equal(scales.cpu().numpy(), want_s)
+
+
+def test_encoder_division_matches_correct_rounding_exhaustively(cuda_device):
+    """The e4m3 encoder divides by the head's scale with a reciprocal and one
+    FMA-residual correction (Markstein's scheme), or, for heads with amax below
+    2^-95, with the correctly rounded division.  For every positive finite bf16 amax
+    and every bf16 x with |x| <= amax (about 10^9 pairs), the resulting e4m3 code
+    equals the code of the correctly rounded fp32 quotient."""
+    assert bca.selftest_e4m3_division(cuda_device) == 0
