@@ -114,6 +114,7 @@ struct AttnParams {
   CUtensorMap tm_q;  // [rows, H, 128] bf16, dims (128, H, rows), box (64, 1, 128)
   CUtensorMap tm_k;  // own keys, same geometry
   CUtensorMap tm_v;
+  CUtensorMap tm_o;  // output, same geometry (bf16 mode: whole Q tiles stored by TMA)
   CUtensorMap tm_kc[MAXR];  // cache K of request r: dims (128, n_tokens, H), box (64, 128, 1)
                             // (e4m3: box (128, 128, 1) into the staging buffers)
   CUtensorMap tm_vc[MAXR];
@@ -170,7 +171,9 @@ struct Smem {
   static constexpr int bStgEmpty = 13 + 2 * kStages;   // 2
   static constexpr int bConv = 15 + 2 * kStages;       // 1 (64 converter arrivals per tile)
   static constexpr int bQEmpty = 16 + 2 * kStages;     // 2 (Q tile w of an item consumed)
-  static constexpr int kNumBars = 18 + 2 * kStages;
+  static constexpr int bEpiFull = 18 + 2 * kStages;    // 2 (O box of tile w in smem: 128)
+  static constexpr int bEpiFree = 20 + 2 * kStages;    // 2 (its TMA store has read it)
+  static constexpr int kNumBars = 22 + 2 * kStages;
   static constexpr int kTmemSlot = kBars + 8 * kNumBars;
   static constexpr int kAbort = kTmemSlot + 4;
   static constexpr int kBytes = kAbort + 4;
@@ -554,9 +557,23 @@ __device__ void mma_role(const AttnParams<MAXR>& p, uint32_t sbase, uint32_t bar
       const int itK = 2 * t, itV = 2 * t - 1;
       const int stK = itK % kStages;
       BCA_TRACE_AT(p, t, 21);
+      if (has_prev) wait(Smem::bKvFull + prev_stV, static_cast<uint32_t>(itV / kStages) & 1u);
+      // At an item boundary the previous item's last P V does not need this item's Q
+      // or K: issue it first, so that its O (and the epilogue) is not held up by the
+      // new item's loads.
+      bool pv_issued[2] = {false, false};
+      if (j == c.j0 && has_prev && ok) {
+        tc_fence_after();
+#pragma unroll
+        for (int w = 0; w < 2; ++w) {
+          if (prev_pv[w] && ok) {
+            issue_pv(w, prev_stV, prev_first[w], prev_last[w]);
+            pv_issued[w] = true;
+          }
+        }
+      }
       wait(Smem::bKvFull + stK, static_cast<uint32_t>(itK / kStages) & 1u);
       BCA_TRACE_AT(p, t, 22);
-      if (has_prev) wait(Smem::bKvFull + prev_stV, static_cast<uint32_t>(itV / kStages) & 1u);
       if (j == c.j0) {
         wait(Smem::bQFull + 0, static_cast<uint32_t>(nq) & 1u);
         wait(Smem::bQFull + 1, static_cast<uint32_t>(nq) & 1u);
@@ -568,7 +585,7 @@ __device__ void mma_role(const AttnParams<MAXR>& p, uint32_t sbase, uint32_t bar
       const uint64_t dk = sdesc_sw128(sbase + Smem::kRing + stK * kTileBytes, 16, 1024);
 #pragma unroll
       for (int w = 0; w < 2; ++w) {
-        if (has_prev && prev_pv[w]) {
+        if (has_prev && prev_pv[w] && !pv_issued[w]) {
           issue_pv(w, prev_stV, prev_first[w], prev_last[w]);
           if (!ok) break;
           BCA_TRACE_AT(p, t, 1 + 2 * w);
@@ -634,8 +651,8 @@ __device__ void mma_role(const AttnParams<MAXR>& p, uint32_t sbase, uint32_t bar
 // Softmax + epilogue: 128 threads (one warpgroup) per Q tile, one row each.
 // ---------------------------------------------------------------------------
 template <int MAXR>
-__device__ void softmax_role(const AttnParams<MAXR>& p, int w, uint32_t bars, uint32_t tmem,
-                             volatile int* abort) {
+__device__ void softmax_role(const AttnParams<MAXR>& p, int w, uint32_t sbase, uint32_t bars,
+                             uint32_t tmem, volatile int* abort) {
   auto bar = [&](int i) { return bars + 8u * static_cast<uint32_t>(i); };
   const int warp = (threadIdx.x / 32) % 4;
   const int lane = threadIdx.x % 32;
@@ -648,6 +665,7 @@ __device__ void softmax_role(const AttnParams<MAXR>& p, int w, uint32_t bars, ui
   const uint32_t b_s = bar(Smem::bSFull + w);
   const uint32_t b_o = bar(Smem::bOFull + w);
   int ns = 0, no = 0;  // S tiles and O results consumed (barrier phases)
+  int nep = 0;         // O boxes stored through shared memory (epilogue barrier phases)
   for (int item = blockIdx.x; item < p.n_items; item += gridDim.x) {
     const Item c = decode_item(p, item);
     if (!tile_active(c, w)) continue;
@@ -794,7 +812,56 @@ __device__ void softmax_role(const AttnParams<MAXR>& p, int w, uint32_t bars, ui
       }
     }
     tc_fence_after();
-    if (c.partial < 0) {
+    const bool tma_epilogue = c.partial < 0 && rows_w == kBM && !p.k_fp8 && !p.v_fp8;
+    if (tma_epilogue) {
+      // Whole bf16 Q tile: normalise into a 64-column box in shared memory (the e4m3
+      // staging buffer of tile w, unused with a bf16 cache) and store it with one TMA
+      // copy per box -- full 128-byte rows instead of 16-byte pieces 8 KiB apart.
+      const float inv = 1.0f / l_run;
+      const uint32_t stg = sbase + Smem::kStage8 + w * kTile8Bytes;
+#pragma unroll
+      for (int half = 0; half < 2; ++half, ++nep) {
+        if (!__all_sync(0xffffffffu,
+                        mbar_wait_bounded(bar(Smem::bEpiFree + w),
+                                          (static_cast<uint32_t>(nep) & 1u) ^ 1u, abort,
+                                          p.timeout_ns))) {
+          raise_abort(abort, p.dev_status, 66);
+          return;
+        }
+#pragma unroll
+        for (int part = 0; part < 2; ++part) {  // 32 columns = chunks 4 part .. 4 part + 3
+          uint32_t o[32];
+          tmem_ld_32x32b_x32(tO + 64 * half + 32 * part, o);
+          tmem_wait_ld();
+#pragma unroll
+          for (int qq = 0; qq < 4; ++qq) {  // 16-byte chunk q of the row, 128-byte swizzle
+            const int q = 4 * part + qq;
+            uint32_t pk[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+              pk[e] = pack_bf16x2(__uint_as_float(o[8 * qq + 2 * e]) * inv,
+                                  __uint_as_float(o[8 * qq + 2 * e + 1]) * inv);
+            asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(
+                             stg + row * 128 + ((q ^ (row & 7)) << 4)),
+                         "r"(pk[0]), "r"(pk[1]), "r"(pk[2]), "r"(pk[3])
+                         : "memory");
+          }
+        }
+        fence_proxy_async_smem();
+        mbar_arrive(bar(Smem::bEpiFull + w));
+        if (row == 0) {
+          if (!mbar_wait_bounded(bar(Smem::bEpiFull + w), static_cast<uint32_t>(nep) & 1u, abort,
+                                 p.timeout_ns)) {
+            raise_abort(abort, p.dev_status, 67);
+          } else {
+            tma_store_3d(&p.tm_o, stg, 64 * half, c.h, c.q_row0 + w * kBM);
+            bulk_commit();
+            bulk_wait_read();
+          }
+          mbar_arrive(bar(Smem::bEpiFree + w));
+        }
+      }
+    } else if (c.partial < 0) {
       const float inv = 1.0f / l_run;
       const bool store = row < rows_w &&
                          BCA_CHECK(p.dev_status, grow < p.o_rows && c.h < p.heads, 3);
@@ -836,6 +903,7 @@ __device__ void softmax_role(const AttnParams<MAXR>& p, int w, uint32_t bars, ui
     // O of this item has been read: the next item's first P V (accumulate = 0) only
     // runs after our next P arrival, which follows these TMEM loads in program order.
   }
+  if (row == 0) bulk_wait_all();  // this thread's TMA stores of O are in global memory
 }
 
 // ---------------------------------------------------------------------------
@@ -866,6 +934,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       mbar_init(bar(Smem::bPFull + 2 * i), 128);
       mbar_init(bar(Smem::bPFull + 2 * i + 1), 128);
       mbar_init(bar(Smem::bOFull + i), 1);
+      mbar_init(bar(Smem::bEpiFull + i), 128);
+      mbar_init(bar(Smem::bEpiFree + i), 1);
       mbar_init(bar(Smem::bStgFull + i), 1);
       mbar_init(bar(Smem::bStgEmpty + i), 1);
     }
@@ -894,7 +964,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 
   if (warp < 8) {
     regs_increase<kSoftmaxRegs>();
-    softmax_role(p, warp / 4, bars, tmem, abort);
+    softmax_role(p, warp / 4, sbase, bars, tmem, abort);
   } else {
     regs_decrease<kOtherRegs>();
     if (warp == kWarpProducer) {

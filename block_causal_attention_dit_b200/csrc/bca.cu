@@ -378,6 +378,7 @@ bca_status bca_prefill(const void* q, const void* k, const void* v, void* o, int
   AttnParams<1> p;
   std::memset(&p, 0, sizeof(p));
   if (!map_thd(&p.tm_q, q, seq_len, heads) || !map_thd(&p.tm_k, k, seq_len, heads) ||
+      !map_thd(&p.tm_o, o, seq_len, heads) ||
       !map_thd(&p.tm_v, v, seq_len, heads))
     return BCA_ERR_CUDA;
   p.tm_kc[0] = p.tm_k;  // unused in prefill mode
@@ -455,6 +456,7 @@ bca_status bca_step_attend(const void* q_t, const void* k_t, const void* v_t, vo
   auto fill = [&](auto& p) -> bca_status {
     std::memset(&p, 0, sizeof(p));
     if (!map_thd(&p.tm_q, q_t, total, heads) || !map_thd(&p.tm_k, k_t, total, heads) ||
+        !map_thd(&p.tm_o, o_t, total, heads) ||
         !map_thd(&p.tm_v, v_t, total, heads))
       return BCA_ERR_CUDA;
     p.o = static_cast<__nv_bfloat16*>(o_t);
