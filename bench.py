@@ -68,11 +68,11 @@ def step_flops(req, H, d=128) -> float:
 # dram__bytes_write.sum) from the ncu capture summarised in
 # profiles/attn_fwd_cached_step_t2i1024.md, valid only for the kernel sources it was
 # taken from (their sha256 below); any later change reports null instead.
-ATTN_TRAFFIC = {"bytes_per_launch": 109.22e6 + 14.75e6, "workload": 1,
+ATTN_TRAFFIC = {"bytes_per_launch": 109.25e6 + 19.77e6, "workload": 1,
                 "sources": {"block_causal_attention_dit_b200/csrc/attn_kernel.cuh":
-                            "3fd425854e076ff78aee8b5c15ad78ee5243f3eea3ad26b12658609b7a413ab5",
+                            "6604b0ce62ee85e9934d53b1bb58d814fb0ddeef83153b52391abf4a035b0e84",
                             "block_causal_attention_dit_b200/csrc/ptx.cuh":
-                            "0a502641c086d1c990ea14655d28721c277848084e0fb2dd1e0195c7b78ce88f"}}
+                            "064a676f712ab6459821cddd509ca1ead0931009ed67e85a5b07ae0a6815a3d7"}}
 
 
 def measured_traffic(workload: int):
