@@ -147,6 +147,46 @@ def _check(status: int, where: str):
         raise BcaError(status, where)
 
 
+# Checks of what the C ABI cannot see (it receives bare pointers): every tensor is a
+# CUDA tensor of the expected dtype, dense where the library assumes density, and
+# large enough for the rows the call will read or write.  A failed check raises
+# BcaError(BCA_ERR_INVALID_ARG) before anything is enqueued.
+def _need(cond, call: str, what: str):
+    if not cond:
+        raise BcaError(1, f"{call} ({what})")
+
+
+def _cuda(t, call, name, dtype=None, device=None):
+    import torch
+    _need(isinstance(t, torch.Tensor) and t.is_cuda, call, f"{name} must be a CUDA tensor")
+    if dtype is not None:
+        _need(t.dtype == dtype, call, f"{name} must be {dtype}")
+    if device is not None:
+        _need(t.device == device, call, f"{name} must be on {device}")
+
+
+def _rows_tensor(t, call, name, like=None):
+    """[rows, H, d] bf16, contiguous (the library's THD layout); `like`: same shape
+    and device as that tensor."""
+    import torch
+    _cuda(t, call, name, torch.bfloat16, None if like is None else like.device)
+    _need(t.dim() == 3 and t.is_contiguous(), call, f"{name} must be a contiguous [rows, H, d]")
+    if like is not None:
+        _need(t.shape == like.shape, call, f"{name} must have shape {tuple(like.shape)}")
+
+
+def _aux(t, call, name, device, dtype=None, min_numel=1):
+    if t is None:
+        return
+    _cuda(t, call, name, dtype, device)
+    _need(t.is_contiguous() and t.numel() >= min_numel, call,
+          f"{name} must be contiguous with at least {min_numel} elements")
+
+
+def _slot_device(slot, call, device):
+    _need(slot.buffer.device == device, call, f"slot buffers must be on {device}")
+
+
 def _ptr(t):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
 
@@ -246,8 +286,25 @@ class KVSlot:
 
 def kv_store(k, v, n_prefix: int, slot: KVSlot, epoch: int, row_stride: int | None = None,
              dev_status=None, stream=None):
+    """Prefix rows [0, n_prefix) of k and v into the slot.  k and v are bf16 CUDA
+    tensors [rows, H, d] or [rows, H*d] whose rows are dense and `row_stride`
+    elements apart (default: their stride(0)); both use the same row stride."""
+    import torch
+    call = "bca_kv_store"
+    for name, t in (("k", k), ("v", v)):
+        _cuda(t, call, name, torch.bfloat16, k.device)
+        _need(t.dim() in (2, 3) and t.stride(-1) == 1 and
+              (t.dim() == 2 or t.stride(1) == t.shape[2]), call, f"{name} rows must be dense")
+        width = t.shape[1] * (t.shape[2] if t.dim() == 3 else 1)
+        _need(width == slot.struct.num_heads * slot.struct.head_dim, call,
+              f"{name} rows must hold the slot's heads x head_dim values")
+        _need(t.shape[0] >= int(n_prefix), call, f"{name} has fewer than n_prefix rows")
     if row_stride is None:
-        row_stride = k.shape[1] * k.shape[2] if k.dim() == 3 else k.stride(0)
+        row_stride = k.stride(0) if k.shape[0] > 1 else width
+    _need(k.shape[0] <= 1 or (k.stride(0) == row_stride and v.stride(0) == row_stride), call,
+          "k and v rows must be row_stride elements apart")
+    _slot_device(slot, call, k.device)
+    _aux(dev_status, call, "dev_status", k.device, torch.int32)
     _check(lib().bca_kv_store(_ptr(k), _ptr(v), int(n_prefix), int(row_stride),
                               ctypes.byref(slot.struct), int(epoch), _ptr(dev_status),
                               _stream(stream, k.device)), "bca_kv_store")
@@ -255,6 +312,14 @@ def kv_store(k, v, n_prefix: int, slot: KVSlot, epoch: int, row_stride: int | No
 
 def prefill(q, k, v, o, block_offsets, scale: float, slot: KVSlot | None = None,
             epoch: int = 0, dev_status=None, stream=None):
+    import torch
+    call = "bca_prefill"
+    _rows_tensor(q, call, "q")
+    for name, t in (("k", k), ("v", v), ("o", o)):
+        _rows_tensor(t, call, name, like=q)
+    if slot is not None:
+        _slot_device(slot, call, q.device)
+    _aux(dev_status, call, "dev_status", q.device, torch.int32)
     S, H, d = q.shape
     off = _i32_array(block_offsets)
     _check(lib().bca_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(o), S, off, len(off) - 1, H, d,
@@ -273,10 +338,27 @@ def step_workspace(device="cuda"):
     return torch.empty(max(step_workspace_bytes(), 256), dtype=torch.uint8, device=device)
 
 
+def _check_step_args(call, q_t, k_t, v_t, o_t, cu_target, slots):
+    _rows_tensor(q_t, call, "q_t")
+    for name, t in (("k_t", k_t), ("v_t", v_t), ("o_t", o_t)):
+        _rows_tensor(t, call, name, like=q_t)
+    cu = [int(x) for x in cu_target]
+    _need(len(cu) == len(slots) + 1, call, "cu_target needs one entry per slot plus one")
+    _need(cu[-1] <= q_t.shape[0], call, "cu_target[-1] exceeds the rows of q_t")
+    for sl in slots:
+        _slot_device(sl, call, q_t.device)
+    return cu
+
+
 def step_attend(q_t, k_t, v_t, o_t, cu_target, slots, scale: float, workspace=None,
                 dev_status=None, stream=None):
+    import torch
+    call = "bca_step_attend"
+    cu = _check_step_args(call, q_t, k_t, v_t, o_t, cu_target, slots)
+    _aux(workspace, call, "workspace", q_t.device)
+    _aux(dev_status, call, "dev_status", q_t.device, torch.int32)
     _, H, d = q_t.shape
-    cu = _i32_array(cu_target)
+    cu = _i32_array(cu)
     arr = (SlotStruct * len(slots))(*[s.struct for s in slots])
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check(lib().bca_step_attend(_ptr(q_t), _ptr(k_t), _ptr(v_t), _ptr(o_t), cu, arr,
@@ -290,10 +372,23 @@ def qk_norm_rope(q, k, gamma_q, gamma_k, cos_t, sin_t, eps: float = 1e-6, stream
     RMS norm over the head dim with weights gamma_* ([128] fp32), then the rotary
     embedding of channel pairs (2i, 2i+1) by the angles whose cos/sin are
     cos_t[t, i], sin_t[t, i] ([rows, 64] fp32)."""
+    import torch
+    call = "bca_qk_norm_rope"
     ref = q if q is not None else k
     if ref is None:
-        raise BcaError(1, "bca_qk_norm_rope")
+        raise BcaError(1, call)
+    _rows_tensor(ref, call, "q" if q is not None else "k")
+    if q is not None and k is not None:
+        _rows_tensor(k, call, "k", like=q)
     rows, H, d = ref.shape
+    if rows > 0:
+        for name, t, x in (("gamma_q", gamma_q, q), ("gamma_k", gamma_k, k)):
+            if x is not None:
+                _need(t is not None, call, f"{name} is required with its tensor")
+                _aux(t, call, name, ref.device, torch.float32, d)
+        for name, t in (("cos_t", cos_t), ("sin_t", sin_t)):
+            _need(t is not None, call, f"{name} is required")
+            _aux(t, call, name, ref.device, torch.float32, rows * (d // 2))
     _check(lib().bca_qk_norm_rope(_ptr(q), _ptr(k), rows, H, d, _ptr(gamma_q), _ptr(gamma_k),
                                   _ptr(cos_t), _ptr(sin_t), float(eps),
                                   _stream(stream, ref.device)), "bca_qk_norm_rope")
@@ -301,6 +396,9 @@ def qk_norm_rope(q, k, gamma_q, gamma_k, cos_t, sin_t, eps: float = 1e-6, stream
 
 def ulysses_pack(x, send, n_ranks: int, stream=None):
     """x [rows, H, 128] -> send [n_ranks, rows, H/n_ranks, 128] (block g for rank g)."""
+    import torch
+    _rows_tensor(x, "bca_ulysses_pack", "x")
+    _aux(send, "bca_ulysses_pack", "send", x.device, torch.bfloat16, x.numel())
     rows, H, d = x.shape
     _check(lib().bca_ulysses_pack(_ptr(x), _ptr(send), rows, H, d, int(n_ranks),
                                   _stream(stream, x.device)), "bca_ulysses_pack")
@@ -308,6 +406,9 @@ def ulysses_pack(x, send, n_ranks: int, stream=None):
 
 def ulysses_unpack(recv, x, n_ranks: int, stream=None):
     """recv [n_ranks, rows, H/n_ranks, 128] (block g from rank g) -> x [rows, H, 128]."""
+    import torch
+    _rows_tensor(x, "bca_ulysses_unpack", "x")
+    _aux(recv, "bca_ulysses_unpack", "recv", x.device, torch.bfloat16, x.numel())
     rows, H, d = x.shape
     _check(lib().bca_ulysses_unpack(_ptr(recv), _ptr(x), rows, H, d, int(n_ranks),
                                     _stream(stream, x.device)), "bca_ulysses_unpack")
@@ -328,6 +429,14 @@ class StepGraph:
         assert n == len(k_layers) == len(v_layers) == len(o_layers) == len(slots_per_layer)
         n_req = len(slots_per_layer[0])
         assert all(len(sl) == n_req for sl in slots_per_layer)
+        import torch
+        call = "bca_step_graph_create"
+        for l in range(n):
+            _check_step_args(call, q_layers[l], k_layers[l], v_layers[l], o_layers[l], cu_target,
+                             slots_per_layer[l])
+            _need(q_layers[l].shape == q_layers[0].shape, call, "layers must share one layout")
+        _aux(workspace, call, "workspace", q_layers[0].device)
+        _aux(dev_status, call, "dev_status", q_layers[0].device, torch.int32)
         _, H, d = q_layers[0].shape
         self._keep = (list(q_layers), list(k_layers), list(v_layers), list(o_layers),
                       [list(sl) for sl in slots_per_layer], workspace, dev_status)

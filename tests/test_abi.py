@@ -201,3 +201,22 @@ def test_ulysses_copy_argument_errors(L):
         assert call(a=None) == 1
         assert call(b=ctypes.c_void_p((1 << 24) + 8)) == 1
         assert call(a=None, rows=0) == 0  # nothing to move
+
+
+def test_binding_rejects_host_tensors_before_the_library_is_called():
+    """The Python binding passes bare pointers to the C ABI, so it checks what the
+    ABI cannot: host (CPU) tensors are refused with BCA_ERR_INVALID_ARG before
+    anything is enqueued."""
+    import torch
+    x = torch.zeros((4, 2, 128), dtype=torch.bfloat16)
+    calls = [
+        lambda: bca.step_attend(x, x, x, x, [0, 4], [], 0.1),
+        lambda: bca.prefill(x, x, x, x, [0, 4], 0.1),
+        lambda: bca.qk_norm_rope(x, None, None, None, None, None),
+        lambda: bca.ulysses_pack(x, torch.empty_like(x), 2),
+        lambda: bca.ulysses_unpack(torch.empty_like(x), x, 2),
+    ]
+    for call in calls:
+        with pytest.raises(bca.BcaError) as e:
+            call()
+        assert e.value.status == 1 and "CUDA tensor" in str(e.value)

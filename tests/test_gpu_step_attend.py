@@ -311,3 +311,51 @@ def test_many_items_per_cta_with_half_empty_q_pairs(cuda_device, mode):
             rows = sample_rows(128, 24, seed=i)
             got = o[cu[i]:cu[i + 1]][torch.from_numpy(rows).to(cuda_device)]
             assert_parity(got, oracle_for(r, rows=rows), rel_l2=tol, what=f"req {i}")
+
+
+@pytest.mark.parametrize("n_req,mode", [(9, "bf16"), (64, "bf16"), (64, "fp8")])
+def test_batches_beyond_eight_requests(cuda_device, n_req, mode):
+    """Batches of 9..64 requests take the largest parameter block (64 requests per
+    launch, the call's maximum); ragged T and P, empty requests included, with and
+    without the split round."""
+    H = 2
+    rng = np.random.default_rng(n_req)
+    # every seventh request of the 64 is empty (9 requests: none, so that all of
+    # them reach the kernel)
+    shapes = [(0 if (n_req > 9 and i % 7 == 3) else int(rng.integers(1, 300)),
+               int(rng.integers(0, 400))) for i in range(n_req)]
+    reqs = [make_request(T, P, H, seed=1200 + i, device=cuda_device, cap=P + 2, mode=mode)
+            for i, (T, P) in enumerate(shapes)]
+    tol = REL_L2_FP8 if mode != "bf16" else 5e-3
+    for ws in (None, bca.step_workspace(cuda_device)):
+        o, cu = run_batch(reqs, H, cuda_device, workspace=ws)
+        for i, r in enumerate(reqs):
+            if r["T"] == 0:
+                continue
+            assert_parity(o[cu[i]:cu[i + 1]], oracle_for(r), rel_l2=tol, what=f"req {i}")
+
+
+def test_binding_rejects_tensors_the_kernels_cannot_read(cuda_device):
+    """Wrong dtype, a non-contiguous view, mismatched shapes, target rows beyond the
+    tensors, a slot on the wrong side of cu_target: BCA_ERR_INVALID_ARG from the
+    binding, nothing enqueued, and the library still works afterwards."""
+    req = make_request(256, 128, 2, seed=1300, device=cuda_device)
+    q, k, v, slot = req["q"], req["k"], req["v"], req["slot"]
+    o = torch.empty_like(q)
+    bad = [
+        (q.float(), k, v, o, [0, 256]),
+        (q.transpose(0, 1).contiguous().transpose(0, 1), k, v, o, [0, 256]),
+        (q, k[:255], v, o, [0, 256]),
+        (q, k, v, o, [0, 300]),
+        (q, k, v, o, [0, 100, 256]),
+    ]
+    for args in bad:
+        with pytest.raises(bca.BcaError) as e:
+            bca.step_attend(*args, [slot], SCALE)
+        assert e.value.status == 1
+    with pytest.raises(bca.BcaError):
+        bca.kv_store(k.float(), v, 128, slot, epoch=3)
+    with pytest.raises(bca.BcaError):
+        bca.kv_store(k[:100], v[:100], 128, slot, epoch=3)  # fewer rows than the prefix
+    o2, _ = run_batch([req], 2, cuda_device)
+    assert_parity(o2, oracle_for(req), what="after rejected calls")
