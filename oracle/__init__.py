@@ -75,7 +75,7 @@ def _load():
         lib.bca_oracle_cached_step.restype = ctypes.c_int
         lib.bca_oracle_cached_step.argtypes = [P, P, P, i64, i64, i64, P, ctypes.c_int, P,
                                                P, ctypes.c_int, P, i64, i64, ctypes.c_double,
-                                               P, i64, P, ctypes.c_int]
+                                               P, i64, P, ctypes.c_int, P, P]
         lib.bca_oracle_rms_norm.restype = None
         lib.bca_oracle_rms_norm.argtypes = [P, i64, i64, P, ctypes.c_double, P]
         lib.bca_oracle_rope.restype = None
@@ -179,9 +179,12 @@ def prefill(q, k, v, block_offsets, scale: float, rows=None, nthreads: int = 0) 
 
 def cached_step(q_t, k_t, v_t, k_cache, v_cache, P: int, scale: float, k_kind=KIND_BF16,
                 v_kind=KIND_BF16, k_scale=None, v_scale=None, rows=None,
-                nthreads: int = 0) -> np.ndarray:
+                nthreads: int = 0, q8=None) -> np.ndarray:
     """Target rows [T, H, d] over [cache rows 0..P-1 ; own rows 0..T-1].
-    Caches are [H, cap, d]: bf16 bits (kind 0) or e4m3 codes (kind 1) with [H] scales."""
+    Caches are [H, cap, d]: bf16 bits (kind 0) or e4m3 codes (kind 1) with [H] scales.
+    q8 = (codes [H, T, d] uint8, scales [H] fp32): the e4m3-Q reading -- the scores
+    against the cached keys use the dequantised Q codes (quantize_prefix(q_t, T)
+    gives them), those against the own keys the bf16 Q."""
     qb, kb, vb = _bits16(q_t), _bits16(k_t), _bits16(v_t)
     T, H, d = qb.shape
     kc = _bits16(k_cache) if k_kind == KIND_BF16 else _bytes8(k_cache)
@@ -193,11 +196,17 @@ def cached_step(q_t, k_t, v_t, k_cache, v_cache, P: int, scale: float, k_kind=KI
     rws = None if rows is None else np.ascontiguousarray(rows, dtype=np.int64)
     n = T if rws is None else len(rws)
     out = np.empty((n, H, d), dtype=np.float64)
+    qc = qs = None
+    if q8 is not None:
+        qc = np.ascontiguousarray(q8[0], dtype=np.uint8)
+        qs = np.ascontiguousarray(q8[1], dtype=np.float32)
+        assert qc.shape == (H, T, d) and qs.shape == (H,)
     rc = _load().bca_oracle_cached_step(
         _ptr(qb), _ptr(kb), _ptr(vb), T, H, d, _ptr(kc), int(k_kind),
         None if ks is None else _ptr(ks), _ptr(vc), int(v_kind),
         None if vs is None else _ptr(vs), int(P), int(cap), float(scale),
-        None if rws is None else _ptr(rws), n, _ptr(out), int(nthreads))
+        None if rws is None else _ptr(rws), n, _ptr(out), int(nthreads),
+        None if qc is None else _ptr(qc), None if qs is None else _ptr(qs))
     if rc != 0:
         raise ValueError("oracle cached_step: bad arguments")
     return out

@@ -155,16 +155,18 @@ static double src_elem(const kv_src* s, int64_t j, int64_t c) {
 
 /* One output row: softmax(q . k_j * scale) over the keys of the sources, in
  * order (source 0 rows 0..n0-1, then source 1 rows 0..n1-1, ...), applied to the
- * matching values.  Keys not listed are simply absent from the sum (that is the
- * mask).  scores[] is caller scratch of length >= total keys. */
-static void attend_row(const double* q, int64_t d, const kv_src* ks, const kv_src* vs,
+ * matching values.  q[s] is the query row that meets source s's keys (the same
+ * row for every source, except where the query is quantised for one of them).
+ * Keys not listed are simply absent from the sum (that is the mask).  scores[] is
+ * caller scratch of length >= total keys. */
+static void attend_row(const double* const* q, int64_t d, const kv_src* ks, const kv_src* vs,
                        int nsrc, double scale, double* scores, double* out) {
   int64_t nk = 0;
   double m = -INFINITY;
   for (int s = 0; s < nsrc; ++s)
     for (int64_t j = 0; j < ks[s].n; ++j) {
       double dot = 0.0;
-      for (int64_t c = 0; c < d; ++c) dot += q[c] * src_elem(&ks[s], j, c);
+      for (int64_t c = 0; c < d; ++c) dot += q[s][c] * src_elem(&ks[s], j, c);
       double sc = scale * dot;
       scores[nk++] = sc;
       if (sc > m) m = sc;
@@ -242,7 +244,8 @@ int bca_oracle_prefill(const uint16_t* q, const uint16_t* k, const uint16_t* v, 
       kv_src ks = {k + h * d, SRC_BF16, H * d, lim, 1.0f};
       kv_src vs = {v + h * d, SRC_BF16, H * d, lim, 1.0f};
       for (int64_t c = 0; c < d; ++c) qrow[c] = bca_oracle_bf16_to_f64(q[(i * H + h) * d + c]);
-      attend_row(qrow, d, &ks, &vs, 1, scale, scores, out + (r * H + h) * d);
+      const double* qs[1] = {qrow};
+      attend_row(qs, d, &ks, &vs, 1, scale, scores, out + (r * H + h) * d);
     }
     free(scores);
     free(qrow);
@@ -258,15 +261,22 @@ int bca_oracle_prefill(const uint16_t* q, const uint16_t* k, const uint16_t* v, 
  * kind 1 = e4m3 codes dequantised with k_scale[h] / v_scale[h].
  * Every target row attends to all P cached keys and all T target keys (the
  * target is the last block), in that order.  rows: target rows to compute
- * (NULL = all).  out: [n_rows, H, d] fp64. */
+ * (NULL = all).  out: [n_rows, H, d] fp64.
+ * q_codes, q_scale (both NULL, or both given): the e4m3-Q reading of the cached
+ * step -- the request's Q quantised per head like a cache tensor (codes [H, T, d],
+ * scales [H], the same encoder and scale rule), and the scores against the cached
+ * keys taken with the dequantised Q, fp32(decode(code) * scale); the scores
+ * against the target's own keys keep the bf16 Q. */
 int bca_oracle_cached_step(const uint16_t* q_t, const uint16_t* k_t, const uint16_t* v_t,
                            int64_t T, int64_t H, int64_t d, const void* k_cache, int k_kind,
                            const float* k_scale, const void* v_cache, int v_kind,
                            const float* v_scale, int64_t P, int64_t cap, double scale,
-                           const int64_t* rows, int64_t n_rows, double* out, int nthreads) {
+                           const int64_t* rows, int64_t n_rows, double* out, int nthreads,
+                           const uint8_t* q_codes, const float* q_scale) {
   if (T < 1 || H < 1 || d < 1 || P < 0 || cap < P) return -1;
   if (P > 0 && (!k_cache || !v_cache)) return -1;
   if ((k_kind == SRC_E4M3 && !k_scale) || (v_kind == SRC_E4M3 && !v_scale)) return -1;
+  if ((q_codes == NULL) != (q_scale == NULL)) return -1;
   if (!rows) n_rows = T;
   for (int64_t r = 0; r < n_rows; ++r)
     if (rows && (rows[r] < 0 || rows[r] >= T)) return -1;
@@ -275,6 +285,7 @@ int bca_oracle_cached_step(const uint16_t* q_t, const uint16_t* k_t, const uint1
   {
     double* scores = (double*)malloc(sizeof(double) * (size_t)(P + T));
     double* qrow = (double*)malloc(sizeof(double) * (size_t)d);
+    double* q8row = (double*)malloc(sizeof(double) * (size_t)d);
 #pragma omp for schedule(dynamic, 1)
     for (int64_t rh = 0; rh < n_rows * H; ++rh) {
       int64_t r = rh / H, h = rh % H;
@@ -289,10 +300,17 @@ int bca_oracle_cached_step(const uint16_t* q_t, const uint16_t* k_t, const uint1
            v_kind == SRC_E4M3 ? v_scale[h] : 1.0f},
           {v_t + h * d, SRC_BF16, H * d, T, 1.0f}};
       for (int64_t c = 0; c < d; ++c) qrow[c] = bca_oracle_bf16_to_f64(q_t[(i * H + h) * d + c]);
-      attend_row(qrow, d, ks, vs, 2, scale, scores, out + (r * H + h) * d);
+      if (q_codes) {
+        kv_src qs = {q_codes + (size_t)(h * T * d), SRC_E4M3, d, T, q_scale[h]};
+        for (int64_t c = 0; c < d; ++c) q8row[c] = src_elem(&qs, i, c);
+      }
+      /* source 0 = the cached keys, source 1 = the target's own keys */
+      const double* qsrc[2] = {q_codes ? q8row : qrow, qrow};
+      attend_row(qsrc, d, ks, vs, 2, scale, scores, out + (r * H + h) * d);
     }
     free(scores);
     free(qrow);
+    free(q8row);
   }
   return 0;
 }
