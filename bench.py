@@ -68,11 +68,11 @@ def step_flops(req, H, d=128) -> float:
 # dram__bytes_write.sum) from the ncu capture summarised in
 # profiles/attn_fwd_cached_step_t2i1024.md, valid only for the kernel sources it was
 # taken from (their sha256 below); any later change reports null instead.
-ATTN_TRAFFIC = {"bytes_per_launch": 109.25e6 + 19.77e6, "workload": 1,
+ATTN_TRAFFIC = {"bytes_per_launch": 109.24e6 + 15.60e6, "workload": 1,
                 "sources": {"block_causal_attention_dit_b200/csrc/attn_kernel.cuh":
-                            "6604b0ce62ee85e9934d53b1bb58d814fb0ddeef83153b52391abf4a035b0e84",
+                            "62fa4d412f679f5ec6ff71e4bdc882816523bcb78718570f549bc38ce9976a9f",
                             "block_causal_attention_dit_b200/csrc/ptx.cuh":
-                            "064a676f712ab6459821cddd509ca1ead0931009ed67e85a5b07ae0a6815a3d7"}}
+                            "5e3e72b92fd39e9479a83a124160be0c84fbd8c7f66acf214212d88f2723b8c3"}}
 
 
 def measured_traffic(workload: int):
@@ -472,6 +472,73 @@ def store_leg(runner, peaks, reps: int = 5):
             "moved_gbs": moved / (ms / 1e3) / 1e9}
 
 
+def q8_leg(device, peaks, calls: int = 10):
+    """bca_step_attend_q8 against bca_step_attend on the step-batched serving
+    workload (8 requests, ragged prefixes, target 4096, H=32, e4m3 K and V cache),
+    one layer's cached step, inputs larger than L2.  The e4m3-Q call includes its Q
+    quantisation pre-pass.  Its peak blends the FP8 peak (the measured bf16 peak x
+    the nominal fp8/bf16 ratio of 2) for the cached keys' Q K^T FLOPs with the bf16
+    peak for the rest."""
+    import numpy as np
+    import torch
+    import block_causal_attention_dit_b200 as bca
+    from block_causal_attention_dit_b200 import workloads as W
+    wl = W.workload(4)
+    H = wl.heads
+    slots = []
+    for i, r in enumerate(wl.requests):
+        _, k0, v0 = W.qkv(wl, 0, 0, i, device)
+        s = bca.KVSlot(r.prefix, H, "fp8", device=device)
+        bca.kv_store(k0, v0, r.prefix, s, epoch=1)
+        slots.append(s)
+        del k0, v0
+    qkv = [W.qkv(wl, 0, 1, i, device) for i in range(len(wl.requests))]
+    q, k, v = (torch.cat([t[j] for t in qkv]) for j in range(3))
+    del qkv
+    o_a, o_b = torch.empty_like(q), torch.empty_like(q)
+    cu = [0]
+    for r in wl.requests:
+        cu.append(cu[-1] + r.target)
+    ws = bca.step_workspace(device)
+    scratch = bca.step_q8_scratch(cu[-1], len(slots), H, device)
+    status = torch.zeros(1, dtype=torch.int32, device=device)
+    calls_ = {"dequant": lambda: bca.step_attend(q, k, v, o_a, cu, slots, wl.scale, workspace=ws,
+                                                 dev_status=status),
+              "q8": lambda: bca.step_attend_q8(q, k, v, o_b, cu, slots, wl.scale,
+                                               q8_scratch=scratch, workspace=ws,
+                                               dev_status=status)}
+    for f in calls_.values():
+        for _ in range(2):
+            f()
+    torch.cuda.synchronize()
+    times = {n: [] for n in calls_}
+    for _ in range(calls):
+        for n, f in calls_.items():
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            f()
+            e1.record()
+            times[n].append((e0, e1))
+    torch.cuda.synchronize()
+    if int(status.item()) != 0:
+        raise RuntimeError(f"device status {int(status.item())} (q8 leg)")
+    ms = {n: sum(a.elapsed_time(b) for a, b in t) / len(t) for n, t in times.items()}
+    flops = sum(step_flops(r, H) for r in wl.requests)
+    flops_f8 = sum(2.0 * 128 * H * r.target * r.prefix for r in wl.requests)
+    bf16_peak = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
+    mixed_peak = flops / (flops_f8 / (2 * bf16_peak) + (flops - flops_f8) / bf16_peak)
+    a, b = o_a.float(), o_b.float()
+    rel = float(torch.linalg.vector_norm(a - b) / torch.linalg.vector_norm(a))
+    t8 = flops / (ms["q8"] / 1e3) / 1e12
+    return {"workload": wl.name, "dequant_ms": ms["dequant"], "q8_ms": ms["q8"],
+            "dequant_tflops": flops / (ms["dequant"] / 1e3) / 1e12, "q8_tflops": t8,
+            "speedup": ms["dequant"] / ms["q8"], "fp8_flop_share": flops_f8 / flops,
+            "peak": mixed_peak, "frac": t8 / mixed_peak,
+            "peak_kind": "fp8 (2x measured bf16 sustained) for the cached keys' Q K^T, "
+                         "bf16 sustained for the rest",
+            "rel_l2_q8_vs_dequant": rel}
+
+
 def timed(fn, steps: int, warmup: int, dist_on: bool):
     import torch
     import torch.distributed as dist
@@ -541,6 +608,8 @@ def main():
                     help="skip the Q/K norm + rotary embedding leg")
     ap.add_argument("--no-graph", action="store_true",
                     help="skip the leg that replays the cached steps from CUDA graphs")
+    ap.add_argument("--no-q8", action="store_true",
+                    help="skip the e4m3-Q cached-step leg (serving workload, one layer)")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     args = ap.parse_args()
 
@@ -646,6 +715,10 @@ def main():
     if not args.no_norm:
         norm = norm_rope_leg(device, peaks, sum(r.target for r in wl.requests), wl.heads)
 
+    q8 = None
+    if not args.no_q8 and n_gpus == 1:
+        q8 = q8_leg(device, peaks)
+
     e2e = None
     if not args.no_e2e:
         e = E2ERunner(runner)
@@ -669,7 +742,7 @@ def main():
                                  "burst": 100 * achieved / peak_burst, "source": peak_src},
             "prefill_and_store_ms_per_step": ms_per_step - sum(step_ms) / args.steps,
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "graph": graph,
-            "qk_norm_rope": norm, "kv_store": store,
+            "qk_norm_rope": norm, "kv_store": store, "fp8_q8_step": q8,
             "gpu_launches": runner.launches_per_step * args.steps, "clocks": clocks}
     if rank == 0:
         print(json.dumps(line), flush=True)

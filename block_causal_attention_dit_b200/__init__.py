@@ -11,6 +11,8 @@ three calls of the method mirror include/bca.h one to one:
   step_attend(q_t, k_t, v_t, o_t, cu_target, slots, scale)
       cached-step attention of packed target rows over [cache ; own K/V] for a
       ragged batch of requests at the same phase.
+  step_attend_q8(q_t, k_t, v_t, o_t, cu_target, slots, scale, q8_scratch)
+      the same over e4m3 ("fp8") slots with e4m3 Q against the e4m3 cached keys.
   qk_norm_rope(q, k, gamma_q, gamma_k, cos_t, sin_t, eps)
       Q/K RMS norm + rotary embedding of the rows entering attention (in place).
   StepGraph(q_layers, k_layers, v_layers, o_layers, cu_target, slots_per_layer, scale)
@@ -30,6 +32,7 @@ import os
 __all__ = [
     "BcaError", "KVSlot", "KV_BF16", "KV_FP8_V", "KV_FP8_KV", "MAX_BLOCKS", "MAX_BATCH",
     "lib", "prefill", "kv_store", "step_attend", "step_workspace", "step_workspace_bytes",
+    "step_attend_q8", "step_q8_scratch", "step_q8_scratch_bytes", "q8_views",
     "StepGraph", "qk_norm_rope", "ulysses_pack", "ulysses_unpack",
     "slot_bytes", "set_wait_timeout_ns",
     "selftest_wait_timeout", "selftest_exp2", "selftest_e4m3_division", "status_string",
@@ -111,6 +114,11 @@ def lib():
                                   P, P]
     L.bca_step_workspace_bytes.restype = ctypes.c_size_t
     L.bca_step_workspace_bytes.argtypes = []
+    L.bca_step_attend_q8.restype = ctypes.c_int
+    L.bca_step_attend_q8.argtypes = [P, P, P, P, P, SP, i32, i32, i32, f32, P, ctypes.c_size_t,
+                                     P, ctypes.c_size_t, P, P]
+    L.bca_step_q8_scratch_bytes.restype = ctypes.c_size_t
+    L.bca_step_q8_scratch_bytes.argtypes = [ctypes.c_int64, i32, i32]
     L.bca_status_string.restype = ctypes.c_char_p
     L.bca_status_string.argtypes = [ctypes.c_int]
     L.bca_set_wait_timeout_ns.restype = None
@@ -365,6 +373,51 @@ def step_attend(q_t, k_t, v_t, o_t, cu_target, slots, scale: float, workspace=No
                                  len(slots), H, d, float(scale), _ptr(workspace), ws_bytes,
                                  _ptr(dev_status), _stream(stream, q_t.device)),
            "bca_step_attend")
+
+
+def step_q8_scratch_bytes(rows: int, n_req: int, heads: int) -> int:
+    return int(lib().bca_step_q8_scratch_bytes(int(rows), int(n_req), int(heads)))
+
+
+def step_q8_scratch(rows: int, n_req: int, heads: int, device="cuda"):
+    """Scratch for step_attend_q8 (uint8 CUDA tensor of step_q8_scratch_bytes())."""
+    import torch
+    n = step_q8_scratch_bytes(rows, n_req, heads)
+    if n == 0:
+        raise BcaError(1, "bca_step_q8_scratch_bytes")
+    return torch.empty(n, dtype=torch.uint8, device=device)
+
+
+def q8_views(q8_scratch, rows: int, n_req: int, heads: int):
+    """(codes [H, rows, 128] uint8, scales [n_req, H] fp32) inside a q8 scratch."""
+    import torch
+    nc = (heads * rows * 128 + 255) // 256 * 256
+    codes = q8_scratch[:heads * rows * 128].view(heads, rows, 128)
+    scales = q8_scratch[nc:nc + 4 * n_req * heads].view(torch.float32).view(n_req, heads)
+    return codes, scales
+
+
+def step_attend_q8(q_t, k_t, v_t, o_t, cu_target, slots, scale: float, q8_scratch=None,
+                   workspace=None, dev_status=None, stream=None):
+    """step_attend over "fp8" slots with e4m3 Q for the scores of cached keys (Q of
+    each request quantised per head like a cache tensor, into q8_scratch)."""
+    import torch
+    call = "bca_step_attend_q8"
+    cu = _check_step_args(call, q_t, k_t, v_t, o_t, cu_target, slots)
+    _, H, d = q_t.shape
+    if q8_scratch is None:
+        q8_scratch = step_q8_scratch(cu[-1], len(slots), H, q_t.device)
+    _aux(q8_scratch, call, "q8_scratch", q_t.device)
+    _aux(workspace, call, "workspace", q_t.device)
+    _aux(dev_status, call, "dev_status", q_t.device, torch.int32)
+    arr = (SlotStruct * len(slots))(*[s.struct for s in slots])
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib().bca_step_attend_q8(_ptr(q_t), _ptr(k_t), _ptr(v_t), _ptr(o_t), _i32_array(cu),
+                                    arr, len(slots), H, d, float(scale), _ptr(workspace),
+                                    ws_bytes, _ptr(q8_scratch),
+                                    q8_scratch.numel() * q8_scratch.element_size(),
+                                    _ptr(dev_status), _stream(stream, q_t.device)), call)
+    return q8_scratch
 
 
 def qk_norm_rope(q, k, gamma_q, gamma_k, cos_t, sin_t, eps: float = 1e-6, stream=None):

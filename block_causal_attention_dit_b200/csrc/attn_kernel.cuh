@@ -22,6 +22,10 @@
 //                  S_w = Q_w K_j^T (both operands in smem) and O_w += P_w V_j (P from
 //                  TMEM, V in smem, MN-major), fp32 accumulators in TMEM.
 //  * warps 10-11 : e4m3 cache tiles -> bf16 in shared memory (FP8 cache only).
+//  * e4m3-Q mode (kQ8, bca_step_attend_q8): Q quantised per (request, head) like a
+//    cache tensor; S of cached keys = Q8 K8^T by tcgen05.mma kind::f8f6f4 with both
+//    operands as stored (Q8 tiles in the staging buffers, K8 tiles straight into
+//    the ring); only V tiles are expanded, in place in their ring slot.
 //  * warps 0..3  : softmax of Q tile 0, warps 4..7: Q tile 1.  One thread per row:
 //                  load S from TMEM, mask ragged / block-causal keys, online softmax
 //                  in the exp2 domain, write P (bf16) back over S in TMEM.  O is
@@ -115,6 +119,7 @@ struct AttnParams {
   CUtensorMap tm_k;  // own keys, same geometry
   CUtensorMap tm_v;
   CUtensorMap tm_o;  // output, same geometry (bf16 mode: whole Q tiles stored by TMA)
+  CUtensorMap tm_q8;  // e4m3-Q mode: codes [H, rows, 128], dims (128, rows, H), box (128, 128, 1)
   CUtensorMap tm_kc[MAXR];  // cache K of request r: dims (128, n_tokens, H), box (64, 128, 1)
                             // (e4m3: box (128, 128, 1) into the staging buffers)
   CUtensorMap tm_vc[MAXR];
@@ -150,6 +155,7 @@ struct AttnParams {
   int32_t v_fp8;
   const float* k_scale[MAXR];
   const float* v_scale[MAXR];
+  const float* q_scale[MAXR];  // e4m3-Q mode: [H] scales of request i's Q codes
 };
 
 // Shared memory map (offsets from a 1024-byte aligned base).
@@ -318,10 +324,18 @@ __device__ __forceinline__ bool tile_is_fp8(const AttnParams<MAXR>& p, const Ite
   return p.mode == kModeStep && j < it.n_cache_tiles && (kv ? p.v_fp8 : p.k_fp8) != 0;
 }
 
+// e4m3 cache tiles the converter warps expand to bf16: all of them, except in
+// e4m3-Q mode, where K tiles go to the MMA as stored and only V tiles are expanded.
+template <int MAXR, bool kQ8>
+__device__ __forceinline__ bool tile_is_converted(const AttnParams<MAXR>& p, const Item& it,
+                                                  int j, int kv) {
+  return tile_is_fp8(p, it, j, kv) && (!kQ8 || kv == 1);
+}
+
 // ---------------------------------------------------------------------------
 // Producer: one thread.
 // ---------------------------------------------------------------------------
-template <int MAXR>
+template <int MAXR, bool kQ8>
 __device__ void producer_role(const AttnParams<MAXR>& p, uint32_t sbase, uint32_t bars,
                               volatile int* abort) {
   auto bar = [&](int i) { return bars + 8u * static_cast<uint32_t>(i); };
@@ -343,9 +357,13 @@ __device__ void producer_role(const AttnParams<MAXR>& p, uint32_t sbase, uint32_
       }
       const uint32_t dst = sbase + (w == 0 ? Smem::kQ0 : Smem::kQ1);
       const int z = c.q_row0 + w * kBM;
-      mbar_arrive_expect_tx(bar(Smem::bQFull + w), kTileBytes);
+      mbar_arrive_expect_tx(bar(Smem::bQFull + w), kTileBytes + (kQ8 ? kTile8Bytes : 0));
       tma_load_3d(dst, &p.tm_q, bar(Smem::bQFull + w), 0, c.h, z);
       tma_load_3d(dst + kHalfBytes, &p.tm_q, bar(Smem::bQFull + w), 64, c.h, z);
+      // e4m3-Q mode: the tile's Q codes go to staging buffer w (unused otherwise).
+      if (kQ8)
+        tma_load_3d(sbase + Smem::kStage8 + w * kTile8Bytes, &p.tm_q8, bar(Smem::bQFull + w), 0,
+                    z, c.h);
     }
     if (!ok) break;
     if (item + static_cast<int>(gridDim.x) < p.n_items) {
@@ -359,8 +377,10 @@ __device__ void producer_role(const AttnParams<MAXR>& p, uint32_t sbase, uint32_
     }
     for (int j = c.j0; j < c.j1 && ok; ++j) {
       for (int kv = 0; kv < 2; ++kv, ++it) {
-        if (tile_is_fp8(p, c, j, kv)) {
+        if (tile_is_converted<MAXR, kQ8>(p, c, j, kv)) {
           // e4m3 cache tile -> staging buffer; the converter warps fill the ring slot.
+          // e4m3-Q mode: the staging buffers hold Q codes, so the (V) tile lands in
+          // the upper half of its own ring slot and is expanded in place.
           const int ss = fi & 1;
           const uint32_t ph = static_cast<uint32_t>(fi >> 1) & 1u;
           if (!mbar_wait_bounded(bar(Smem::bStgEmpty + ss), ph ^ 1u, abort, p.timeout_ns)) {
@@ -368,11 +388,22 @@ __device__ void producer_role(const AttnParams<MAXR>& p, uint32_t sbase, uint32_
             ok = false;
             break;
           }
+          uint32_t dst8 = sbase + Smem::kStage8 + ss * kTile8Bytes;
+          if (kQ8) {
+            const int st = it % kStages;
+            if (!mbar_wait_bounded(bar(Smem::bKvEmpty + st),
+                                   (static_cast<uint32_t>(it / kStages) & 1u) ^ 1u, abort,
+                                   p.timeout_ns)) {
+              raise_abort(abort, p.dev_status, 13);
+              ok = false;
+              break;
+            }
+            dst8 = sbase + Smem::kRing + st * kTileBytes + kTile8Bytes;
+          }
           const uint32_t fb = bar(Smem::bStgFull + ss);
           mbar_arrive_expect_tx(fb, kTile8Bytes);
           if (BCA_CHECK(p.dev_status, c.req < p.n_req && j * kBN < c.n_cache && c.h < p.heads, 1))
-            tma_load_3d(sbase + Smem::kStage8 + ss * kTile8Bytes,
-                        kv ? &p.tm_vc[c.req] : &p.tm_kc[c.req], fb, 0, j * kBN, c.h);
+            tma_load_3d(dst8, kv ? &p.tm_vc[c.req] : &p.tm_kc[c.req], fb, 0, j * kBN, c.h);
           ++fi;
           continue;
         }
@@ -386,6 +417,13 @@ __device__ void producer_role(const AttnParams<MAXR>& p, uint32_t sbase, uint32_
         const uint32_t dst = sbase + Smem::kRing + st * kTileBytes;
         const uint32_t fb = bar(Smem::bKvFull + st);
         BCA_TRACE_AT(p, it / 2, 23 + kv);
+        if (kQ8 && tile_is_fp8(p, c, j, kv)) {
+          // e4m3-Q mode, K cache tile: read by the MMA as stored (16 KiB).
+          mbar_arrive_expect_tx(fb, kTile8Bytes);
+          if (BCA_CHECK(p.dev_status, c.req < p.n_req && j * kBN < c.n_cache && c.h < p.heads, 6))
+            tma_load_3d(dst, &p.tm_kc[c.req], fb, 0, j * kBN, c.h);
+          continue;
+        }
         mbar_arrive_expect_tx(fb, kTileBytes);
         if (p.mode == kModeStep && j < c.n_cache_tiles) {
           const CUtensorMap* m = kv ? &p.tm_vc[c.req] : &p.tm_kc[c.req];
@@ -430,7 +468,7 @@ __device__ __forceinline__ uint32_t e4m3x2_to_bf16x2(uint32_t two) {
   return pack_bf16x2(lo, hi);
 }
 
-template <int MAXR>
+template <int MAXR, bool kQ8>
 __device__ void converter_role(const AttnParams<MAXR>& p, uint32_t sbase, uint32_t bars,
                                volatile int* abort) {
   auto bar = [&](int i) { return bars + 8u * static_cast<uint32_t>(i); };
@@ -440,31 +478,39 @@ __device__ void converter_role(const AttnParams<MAXR>& p, uint32_t sbase, uint32
     const Item ci = decode_item(p, item);
     for (int j = ci.j0; j < ci.j1; ++j) {
       for (int kv = 0; kv < 2; ++kv, ++it) {
-        if (!tile_is_fp8(p, ci, j, kv)) continue;
+        if (!tile_is_converted<MAXR, kQ8>(p, ci, j, kv)) continue;
         const int ss = fi & 1;
         const int st = it % kStages;
+        // (e4m3-Q mode: the producer waited for the ring slot before loading into it.)
         const bool got =
             mbar_wait_bounded(bar(Smem::bStgFull + ss), static_cast<uint32_t>(fi >> 1) & 1u,
                               abort, p.timeout_ns) &&
-            mbar_wait_bounded(bar(Smem::bKvEmpty + st),
-                              (static_cast<uint32_t>(it / kStages) & 1u) ^ 1u, abort, p.timeout_ns);
+            (kQ8 || mbar_wait_bounded(bar(Smem::bKvEmpty + st),
+                                      (static_cast<uint32_t>(it / kStages) & 1u) ^ 1u, abort,
+                                      p.timeout_ns));
         if (!got) {
           raise_abort(abort, p.dev_status, 21);
           return;
         }
-        const uint32_t src = sbase + Smem::kStage8 + ss * kTile8Bytes;
         const uint32_t dst = sbase + Smem::kRing + st * kTileBytes;
+        const uint32_t src = kQ8 ? dst + kTile8Bytes : sbase + Smem::kStage8 + ss * kTile8Bytes;
 #pragma unroll 4
         for (int k = 0; k < 16; ++k) {
           const int gid = k * kConvThreads + c;
           const int row = gid >> 3, ch = gid & 7;
-          if (!BCA_CHECK(p.dev_status, row < kBN && src + row * 128 + 128 <= sbase + Smem::kBars &&
-                                           dst + kTileBytes <= sbase + Smem::kStage8, 2))
-            continue;
-          uint32_t w0, w1, w2, w3;
-          asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
-                       : "=r"(w0), "=r"(w1), "=r"(w2), "=r"(w3)
-                       : "r"(src + row * 128 + ((ch ^ (row & 7)) << 4)));
+          const bool in_bounds =
+              BCA_CHECK(p.dev_status, row < kBN && src + row * 128 + 128 <= sbase + Smem::kBars &&
+                                          dst + kTileBytes <= sbase + Smem::kStage8, 2);
+          uint32_t w0 = 0, w1 = 0, w2 = 0, w3 = 0;
+          if (in_bounds)
+            asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                         : "=r"(w0), "=r"(w1), "=r"(w2), "=r"(w3)
+                         : "r"(src + row * 128 + ((ch ^ (row & 7)) << 4)));
+          // In place (e4m3-Q mode), the upper half of row `row`'s output overwrites
+          // the row's own source bytes, which the row's 8 threads (8 lanes of one
+          // warp) read above: every lane's load comes before any lane's store.
+          if (kQ8) __syncwarp();
+          if (!in_bounds) continue;
           const uint32_t o0 = e4m3x2_to_bf16x2(w0), o1 = e4m3x2_to_bf16x2(w0 >> 16);
           const uint32_t o2 = e4m3x2_to_bf16x2(w1), o3 = e4m3x2_to_bf16x2(w1 >> 16);
           const uint32_t o4 = e4m3x2_to_bf16x2(w2), o5 = e4m3x2_to_bf16x2(w2 >> 16);
@@ -502,7 +548,7 @@ __device__ void converter_role(const AttnParams<MAXR>& p, uint32_t sbase, uint32
 // ---------------------------------------------------------------------------
 // MMA issuer: the whole warp (values stay warp-uniform); one elected lane issues.
 // ---------------------------------------------------------------------------
-template <int MAXR>
+template <int MAXR, bool kQ8>
 __device__ void mma_role(const AttnParams<MAXR>& p, uint32_t sbase, uint32_t bars, uint32_t tmem,
                          volatile int* abort) {
   // The items of this CTA are one stream of KV tiles.  Iteration t issues, per Q tile
@@ -512,6 +558,7 @@ __device__ void mma_role(const AttnParams<MAXR>& p, uint32_t sbase, uint32_t bar
   auto bar = [&](int i) { return bars + 8u * static_cast<uint32_t>(i); };
   constexpr uint32_t kIdescS = idesc_bf16_f32(kBM, kBN, false);      // Q K^T: K-major B
   constexpr uint32_t kIdescO = idesc_bf16_f32(kBM, kHeadDim, true);  // P V: MN-major B
+  constexpr uint32_t kIdescS8 = idesc_e4m3_f32(kBM, kBN);            // Q8 K8^T (e4m3-Q mode)
   bool ok = true;
   auto wait = [&](int b, uint32_t parity) {
     if (ok) {
@@ -593,10 +640,23 @@ __device__ void mma_role(const AttnParams<MAXR>& p, uint32_t sbase, uint32_t bar
         const int jend = w ? c.jend[1] : c.jend[0];
         if (act[w] && j < jend) {
           if (elect_one()) {
+            if (kQ8 && j < c.n_cache_tiles) {
+              // Q codes of tile w in staging buffer w, K codes in the ring slot: one
+              // 128-byte swizzle atom per row; the 4 MMAs of K = 32 step 32 bytes.
+              // (Not unrolled: the unrolled descriptors spill the 104-register
+              // warpgroup.)
+              const uint64_t dq8 =
+                  sdesc_sw128(sbase + Smem::kStage8 + w * kTile8Bytes, 16, 1024);
+#pragma unroll 1
+              for (int s = 0; s < kHeadDim / 32; ++s)
+                mma_e4m3_ss(tmem + col_s(w), dq8 + ((s * 32) >> 4), dk + ((s * 32) >> 4),
+                            kIdescS8, s > 0 ? 1u : 0u);
+            } else {
 #pragma unroll
-            for (int s = 0; s < kHeadDim / 16; ++s) {
-              const uint32_t koff = ((s / 4) * kHalfBytes + (s % 4) * 32) >> 4;
-              mma_bf16_ss(tmem + col_s(w), dq[w] + koff, dk + koff, kIdescS, s > 0 ? 1u : 0u);
+              for (int s = 0; s < kHeadDim / 16; ++s) {
+                const uint32_t koff = ((s / 4) * kHalfBytes + (s % 4) * 32) >> 4;
+                mma_bf16_ss(tmem + col_s(w), dq[w] + koff, dk + koff, kIdescS, s > 0 ? 1u : 0u);
+              }
             }
             mma_commit(bar(Smem::bSFull + w));
             // Last S_w of the item: Q tile w may be reloaded once this MMA is done.
@@ -650,7 +710,7 @@ __device__ void mma_role(const AttnParams<MAXR>& p, uint32_t sbase, uint32_t bar
 // ---------------------------------------------------------------------------
 // Softmax + epilogue: 128 threads (one warpgroup) per Q tile, one row each.
 // ---------------------------------------------------------------------------
-template <int MAXR>
+template <int MAXR, bool kQ8>
 __device__ void softmax_role(const AttnParams<MAXR>& p, int w, uint32_t sbase, uint32_t bars,
                              uint32_t tmem, volatile int* abort) {
   auto bar = [&](int i) { return bars + 8u * static_cast<uint32_t>(i); };
@@ -682,6 +742,9 @@ __device__ void softmax_role(const AttnParams<MAXR>& p, int w, uint32_t sbase, u
                                        (!p.v_fp8 || p.v_scale[c.req]), 4))
         return;
       if (p.k_fp8) sl2_cache *= __ldg(p.k_scale[c.req] + c.h);
+      // e4m3-Q mode: cached keys' scores are Q8 K8^T, so Q's scale joins K's.
+      if (kQ8 && BCA_CHECK(p.dev_status, p.q_scale[c.req] != nullptr, 7))
+        sl2_cache *= __ldg(p.q_scale[c.req] + c.h);
       if (p.v_fp8) {
         const float vs = __ldg(p.v_scale[c.req] + c.h);
         lg_vs = __log2f(vs);
@@ -909,7 +972,7 @@ __device__ void softmax_role(const AttnParams<MAXR>& p, int w, uint32_t sbase, u
 // ---------------------------------------------------------------------------
 // The kernel (persistent: one CTA per SM, static round-robin over work items)
 // ---------------------------------------------------------------------------
-template <int MAXR>
+template <int MAXR, bool kQ8>
 __global__ void __launch_bounds__(kAttnThreads, 1)
     attn_fwd_kernel(const __grid_constant__ AttnParams<MAXR> p) {
   extern __shared__ uint8_t smem_raw[];
@@ -952,6 +1015,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     tma_prefetch_desc(&p.tm_q);
     tma_prefetch_desc(&p.tm_k);
     tma_prefetch_desc(&p.tm_v);
+    if (kQ8) tma_prefetch_desc(&p.tm_q8);
   }
   if (warp == kWarpMma) {
     tmem_alloc(smem_u32(tmem_slot), 512);
@@ -964,16 +1028,16 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 
   if (warp < 8) {
     regs_increase<kSoftmaxRegs>();
-    softmax_role(p, warp / 4, sbase, bars, tmem, abort);
+    softmax_role<MAXR, kQ8>(p, warp / 4, sbase, bars, tmem, abort);
   } else {
     regs_decrease<kOtherRegs>();
     if (warp == kWarpProducer) {
-      if (lane == 0) producer_role(p, sbase, bars, abort);
+      if (lane == 0) producer_role<MAXR, kQ8>(p, sbase, bars, abort);
     } else if (warp == kWarpMma) {
-      mma_role(p, sbase, bars, tmem, abort);
+      mma_role<MAXR, kQ8>(p, sbase, bars, tmem, abort);
       __syncwarp();
     } else if (p.mode == kModeStep && (p.k_fp8 || p.v_fp8)) {
-      converter_role(p, sbase, bars, abort);
+      converter_role<MAXR, kQ8>(p, sbase, bars, abort);
     }
   }
   tc_fence_before();

@@ -4,12 +4,14 @@
 //   bca_prefill      step-1 block-causal attention (+ prefix K/V into a slot)
 //   bca_kv_store     prefix K/V cache layout, bf16 or OFP8 E4M3 with per-head scales
 //   bca_step_attend  cached-step target attention for a ragged same-phase batch
-// and around them: bca_qk_norm_rope (Q/K RMS norm + rotary embedding of the rows
+// and around them: bca_step_attend_q8 (the cached step with e4m3 Q against e4m3
+// cached keys), bca_qk_norm_rope (Q/K RMS norm + rotary embedding of the rows
 // entering attention), bca_step_graph_* (all layers' cached steps as one graph) and
 // bca_ulysses_pack/unpack (layouts around the all-to-all of head-sharded
 // sequence parallelism).
-// Every step of the path runs in the kernels of attn_kernel.cuh and
-// kv_store_kernel.cuh; this file only checks arguments and enqueues them.
+// Every step of the path runs in the kernels of attn_kernel.cuh, kv_store_kernel.cuh,
+// q8_kernel.cuh, qk_norm_rope_kernel.cuh and ulysses_kernel.cuh; this file only
+// checks arguments and enqueues them.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -20,11 +22,13 @@
 #include <cstring>
 #include <mutex>
 #include <numeric>
+#include <type_traits>
 #include <vector>
 
 #include "../../include/bca.h"
 #include "attn_kernel.cuh"
 #include "kv_store_kernel.cuh"
+#include "q8_kernel.cuh"
 #include "qk_norm_rope_kernel.cuh"
 #include "ulysses_kernel.cuh"
 
@@ -121,6 +125,22 @@ bool v_is_fp8(int32_t dt) { return dt == BCA_KV_FP8_V || dt == BCA_KV_FP8_KV; }
 
 size_t round256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
+template <typename T>
+struct MaxRequests;
+template <int MAXR>
+struct MaxRequests<AttnParams<MAXR>> {
+  static constexpr int value = MAXR;
+};
+
+// e4m3-Q scratch: codes [H, rows, 128], then scales [n_req][H] fp32, then the
+// absmax pass's [n_req][H] words.
+size_t q8_codes_bytes(int64_t rows, int heads) {
+  return round256(static_cast<size_t>(rows) * static_cast<size_t>(heads) * 128);
+}
+size_t q8_table_bytes(int n_req, int heads) {
+  return round256(static_cast<size_t>(n_req) * static_cast<size_t>(heads) * 4);
+}
+
 struct SlotLayout {
   size_t k_off, v_off, ks_off, vs_off, total;
 };
@@ -150,13 +170,10 @@ bca_status check_slot_shape(const bca_kv_slot* s, int heads, int hd) {
   return BCA_OK;
 }
 
-std::vector<char> g_attr_attn1, g_attr_attn8, g_attr_attn64;
-
-template <int MAXR>
+template <int MAXR, bool kQ8>
 std::vector<char>& attr_flags() {
-  if (MAXR == 1) return g_attr_attn1;
-  if (MAXR == 8) return g_attr_attn8;
-  return g_attr_attn64;
+  static std::vector<char> done;  // per device: attributes set
+  return done;
 }
 
 int sm_count() {
@@ -197,9 +214,10 @@ int plan_items(AttnParams<MAXR>& p, int units, int grid, size_t ws_chunks, Tiles
 
 // One-time (per device) kernel attributes; also run before a stream capture so that
 // no attribute call happens inside it.
-template <int MAXR>
+template <int MAXR, bool kQ8 = false>
 bool prepare_attn() {
-  if (!ensure_smem_attr(bca::attn_fwd_kernel<MAXR>, bca::Smem::kDynamicBytes, attr_flags<MAXR>()))
+  if (!ensure_smem_attr(bca::attn_fwd_kernel<MAXR, kQ8>, bca::Smem::kDynamicBytes,
+                        attr_flags<MAXR, kQ8>()))
     return false;
   // The kernel re-splits its launch registers between warpgroups (setmaxnreg); that
   // only works if the compiled register count provides the pool the split assumes.
@@ -207,21 +225,22 @@ bool prepare_attn() {
   static bool regs_ok = false;
   std::call_once(regs_once, [] {
     cudaFuncAttributes a{};
-    regs_ok = cudaFuncGetAttributes(&a, bca::attn_fwd_kernel<MAXR>) == cudaSuccess &&
+    regs_ok = cudaFuncGetAttributes(&a, bca::attn_fwd_kernel<MAXR, kQ8>) == cudaSuccess &&
               static_cast<uint32_t>(a.numRegs) * bca::kAttnThreads >=
                   128u * (2u * bca::kSoftmaxRegs + bca::kOtherRegs);
   });
   return regs_ok;
 }
 
-template <int MAXR>
+template <int MAXR, bool kQ8 = false>
 bca_status launch_attn(const AttnParams<MAXR>& p, int n_split_units, cudaStream_t stream) {
   if (p.n_items <= 0) return BCA_OK;
-  if (!prepare_attn<MAXR>()) return BCA_ERR_CUDA;
+  if (!prepare_attn<MAXR, kQ8>()) return BCA_ERR_CUDA;
   const int sms = sm_count();
   if (sms <= 0) return BCA_ERR_CUDA;
   const int grid = std::min(sms, p.n_items);
-  bca::attn_fwd_kernel<MAXR><<<grid, bca::kAttnThreads, bca::Smem::kDynamicBytes, stream>>>(p);
+  bca::attn_fwd_kernel<MAXR, kQ8>
+      <<<grid, bca::kAttnThreads, bca::Smem::kDynamicBytes, stream>>>(p);
   if (cudaGetLastError() != cudaSuccess) return BCA_ERR_CUDA;
   if (n_split_units > 0) {
     const int rows = n_split_units * bca::kChunkRows;
@@ -414,10 +433,17 @@ size_t bca_step_workspace_bytes(void) {
   return sms > 0 ? static_cast<size_t>(sms) * bca::kChunkBytes : 0;
 }
 
-bca_status bca_step_attend(const void* q_t, const void* k_t, const void* v_t, void* o_t,
-                           const int32_t* cu, const bca_kv_slot* slots, int32_t n_req,
-                           int32_t heads, int32_t head_dim, float scale, void* workspace,
-                           size_t workspace_bytes, int32_t* dev_status, void* stream) {
+size_t bca_step_q8_scratch_bytes(int64_t rows, int32_t n_req, int32_t heads) {
+  if (rows < 0 || n_req < 1 || n_req > BCA_MAX_BATCH || heads < 1 || heads > 256) return 0;
+  return q8_codes_bytes(rows, heads) + 2 * q8_table_bytes(n_req, heads);
+}
+
+// The cached step; with q8_scratch, in e4m3-Q mode (bca_step_attend_q8).
+static bca_status step_attend_impl(const void* q_t, const void* k_t, const void* v_t, void* o_t,
+                                   const int32_t* cu, const bca_kv_slot* slots, int32_t n_req,
+                                   int32_t heads, int32_t head_dim, float scale, void* workspace,
+                                   size_t workspace_bytes, bool q8, void* q8_scratch,
+                                   size_t q8_bytes, int32_t* dev_status, void* stream) {
   if (workspace && (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return BCA_ERR_INVALID_ARG;
   const size_t ws_chunks = workspace ? workspace_bytes / bca::kChunkBytes : 0;
   if (!cu || !slots) return BCA_ERR_INVALID_ARG;
@@ -441,9 +467,46 @@ bca_status bca_step_attend(const void* q_t, const void* k_t, const void* v_t, vo
       return BCA_ERR_INVALID_ARG;
     if (slots[r].dtype != slots[0].dtype) return BCA_ERR_UNSUPPORTED;
   }
+  if (q8) {
+    if (slots[0].dtype != BCA_KV_FP8_KV) return BCA_ERR_UNSUPPORTED;
+    if (!q8_scratch || (reinterpret_cast<uintptr_t>(q8_scratch) & 255u) != 0)
+      return BCA_ERR_INVALID_ARG;
+    if (q8_bytes < bca_step_q8_scratch_bytes(total, n_req, heads)) return BCA_ERR_CAPACITY;
+  }
   if (total == 0) return BCA_OK;
   const int32_t dt = slots[0].dtype;
   if (!get_encode()) return BCA_ERR_CUDA;
+  uint8_t* q8_codes = static_cast<uint8_t*>(q8_scratch);
+  float* q8_scale = q8 ? reinterpret_cast<float*>(q8_codes + q8_codes_bytes(total, heads)) : nullptr;
+  if (q8) {
+    // Q codes and scales of every request, before the attention reads them.
+    bca::Q8Params qp{};
+    qp.q = static_cast<const uint16_t*>(q_t);
+    qp.codes = q8_codes;
+    qp.scale = q8_scale;
+    qp.amax = reinterpret_cast<unsigned*>(reinterpret_cast<uint8_t*>(q8_scale) +
+                                          q8_table_bytes(n_req, heads));
+    qp.rows = total;
+    qp.heads = heads;
+    qp.n_req = n_req;
+    int max_len = 0;
+    for (int r = 0; r < n_req; ++r) {
+      qp.q_start[r] = cu[r];
+      qp.q_len[r] = cu[r + 1] - cu[r];
+      max_len = std::max(max_len, qp.q_len[r]);
+    }
+    const int sms = std::max(sm_count(), 1);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    bca::q8_amax_init_kernel<<<1, 256, 0, s>>>(qp);
+    const int ax = (max_len + bca::kQ8RowsPerBlock - 1) / bca::kQ8RowsPerBlock;
+    bca::q8_amax_kernel<<<dim3(ax, n_req), bca::kQ8Threads, 0, s>>>(qp);
+    const int64_t want = (static_cast<int64_t>(max_len) * heads * 16 + bca::kQ8Threads - 1) /
+                         bca::kQ8Threads;
+    const int ex = static_cast<int>(
+        std::max<int64_t>(1, std::min<int64_t>(want, std::max(1, 4 * sms / n_req))));
+    bca::q8_encode_kernel<<<dim3(ex, n_req), bca::kQ8Threads, 0, s>>>(qp);
+    if (cudaGetLastError() != cudaSuccess) return BCA_ERR_CUDA;
+  }
 
   // Longest key sequence first (largest per-unit work scheduled first).
   std::vector<int> order;
@@ -484,6 +547,7 @@ bca_status bca_step_attend(const void* q_t, const void* k_t, const void* v_t, vo
       if (!kok || !vok) return BCA_ERR_CUDA;
       p.k_scale[i] = sl.k_scale;
       p.v_scale[i] = sl.v_scale;
+      p.q_scale[i] = q8 ? q8_scale + static_cast<size_t>(r) * heads : nullptr;
       p.q_start[i] = cu[r];
       p.q_len[i] = cu[r + 1] - cu[r];
       p.n_cache[i] = sl.n_tokens;
@@ -491,6 +555,11 @@ bca_status bca_step_attend(const void* q_t, const void* k_t, const void* v_t, vo
       units += heads * ((p.q_len[i] + 2 * bca::kBM - 1) / (2 * bca::kBM));
     }
     p.unit_start[nr] = units;
+    // e4m3-Q codes [H, total, 128]: one 128-byte box row per (head, row).
+    if (q8 && !make_map_3d(&p.tm_q8, q8_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 128,
+                           static_cast<uint64_t>(total), static_cast<uint64_t>(heads), 128,
+                           static_cast<uint64_t>(total) * 128, 128, 128, 1))
+      return BCA_ERR_CUDA;
     p.workspace = static_cast<float*>(workspace);
     const int sms = sm_count();
     if (sms <= 0) return BCA_ERR_CUDA;
@@ -499,7 +568,9 @@ bca_status bca_step_attend(const void* q_t, const void* k_t, const void* v_t, vo
       while (i + 1 < nr && unit >= p.unit_start[i + 1]) ++i;
       return (p.n_cache[i] + bca::kBN - 1) / bca::kBN + (p.q_len[i] + bca::kBN - 1) / bca::kBN;
     });
-    return launch_attn(p, n_split, static_cast<cudaStream_t>(stream));
+    constexpr int kMaxR = MaxRequests<std::remove_reference_t<decltype(p)>>::value;
+    return q8 ? launch_attn<kMaxR, true>(p, n_split, static_cast<cudaStream_t>(stream))
+              : launch_attn<kMaxR, false>(p, n_split, static_cast<cudaStream_t>(stream));
   };
   if (nr <= 1) {
     AttnParams<1> p;
@@ -510,6 +581,23 @@ bca_status bca_step_attend(const void* q_t, const void* k_t, const void* v_t, vo
   }
   AttnParams<64> p;
   return fill(p);
+}
+
+bca_status bca_step_attend(const void* q_t, const void* k_t, const void* v_t, void* o_t,
+                           const int32_t* cu, const bca_kv_slot* slots, int32_t n_req,
+                           int32_t heads, int32_t head_dim, float scale, void* workspace,
+                           size_t workspace_bytes, int32_t* dev_status, void* stream) {
+  return step_attend_impl(q_t, k_t, v_t, o_t, cu, slots, n_req, heads, head_dim, scale, workspace,
+                          workspace_bytes, false, nullptr, 0, dev_status, stream);
+}
+
+bca_status bca_step_attend_q8(const void* q_t, const void* k_t, const void* v_t, void* o_t,
+                              const int32_t* cu, const bca_kv_slot* slots, int32_t n_req,
+                              int32_t heads, int32_t head_dim, float scale, void* workspace,
+                              size_t workspace_bytes, void* q8_scratch, size_t q8_scratch_bytes,
+                              int32_t* dev_status, void* stream) {
+  return step_attend_impl(q_t, k_t, v_t, o_t, cu, slots, n_req, heads, head_dim, scale, workspace,
+                          workspace_bytes, true, q8_scratch, q8_scratch_bytes, dev_status, stream);
 }
 
 }  // extern "C"

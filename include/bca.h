@@ -161,6 +161,34 @@ bca_status bca_step_attend(const void* q_t, const void* k_t, const void* v_t, vo
                            int32_t heads, int32_t head_dim, float scale, void* workspace,
                            size_t workspace_bytes, int32_t* dev_status, void* stream);
 
+/* The cached step of bca_step_attend with e4m3 Q against e4m3 cached keys (all
+ * slots BCA_KV_FP8_KV).  Each request's target Q rows are first quantised per head
+ * with the cache's own rule (scale = absmax / 448, codes = e4m3_rn_satfinite(q /
+ * scale); "Qwen/Qwen-Image-2.1" vLLM recipe, "Prefix KV cache", applied to Q), and
+ * the scores against cached keys are those of the e4m3 Q with the e4m3 K, read by
+ * the tensor cores as stored (tcgen05.mma kind::f8f6f4); the scale of Q joins K's
+ * in the softmax scale.  Scores against the request's own keys use the bf16 Q, and
+ * P and V are as in bca_step_attend (V codes expanded exactly to bf16, P bf16).
+ *   q8_scratch,
+ *   q8_scratch_bytes : device scratch, 256-byte aligned, caller-owned, at least
+ *                      bca_step_q8_scratch_bytes(cu_target[n_req], n_req, heads).
+ *                      After the call it holds the Q codes [heads, rows, 128] at
+ *                      offset 0 and the fp32 scales [n_req][heads] (by request
+ *                      index) at offset round_up(heads * rows * 128, 256); calls
+ *                      sharing it must not overlap.
+ * Other arguments, results and errors: as bca_step_attend, plus
+ * BCA_ERR_UNSUPPORTED if the slots are not BCA_KV_FP8_KV, BCA_ERR_INVALID_ARG for a
+ * NULL or misaligned scratch and BCA_ERR_CAPACITY for a small one. */
+bca_status bca_step_attend_q8(const void* q_t, const void* k_t, const void* v_t, void* o_t,
+                              const int32_t* cu_target, const bca_kv_slot* slots, int32_t n_req,
+                              int32_t heads, int32_t head_dim, float scale, void* workspace,
+                              size_t workspace_bytes, void* q8_scratch, size_t q8_scratch_bytes,
+                              int32_t* dev_status, void* stream);
+
+/* Bytes of bca_step_attend_q8's scratch for `rows` packed target rows of n_req
+ * requests (0 for arguments out of range). */
+size_t bca_step_q8_scratch_bytes(int64_t rows, int32_t n_req, int32_t heads);
+
 /* Bytes of the optional bca_step_attend workspace that lets the kernel split the
  * last partial round of work along the keys (so that every SM finishes at the same
  * time) for the current device: one chunk of 256 rows x (128 + 2) fp32 per SM.
