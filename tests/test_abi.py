@@ -138,6 +138,31 @@ def test_step_attend_argument_errors(L):
     assert call(ws=ctypes.c_void_p((1 << 24) + 16), ws_bytes=1 << 20) == 1  # misaligned workspace
 
 
+def test_step_attend_q8_argument_errors(L):
+    """bca_step_attend_q8 checks, before anything is enqueued: e4m3 K and V slots
+    (an e4m3 Q meets e4m3 K codes), a non-NULL 256-byte aligned scratch, and its
+    size; bca_step_q8_scratch_bytes gives that size."""
+    H, rows = 2, 228
+    need = L.bca_step_q8_scratch_bytes(rows, 2, H)
+    codes = (H * rows * 128 + 255) // 256 * 256
+    assert need == codes + 2 * 256
+    assert L.bca_step_q8_scratch_bytes(-1, 2, H) == 0
+    assert L.bca_step_q8_scratch_bytes(rows, 0, H) == 0
+    assert L.bca_step_q8_scratch_bytes(rows, 65, H) == 0
+    assert L.bca_step_q8_scratch_bytes(rows, 2, 0) == 0
+    cu = (ctypes.c_int32 * 3)(0, 100, rows)
+    fp8 = (bca.SlotStruct * 2)(_slot(L, dt=2), _slot(L, dt=2, n=20))
+    scratch = ctypes.c_void_p(1 << 28)
+    call = lambda **kw: L.bca_step_attend_q8(
+        FAKE, FAKE, FAKE, FAKE, cu, kw.get("arr", fp8), 2, H, 128, 0.1, None, 0,
+        kw.get("scratch", scratch), kw.get("bytes", need), None, None)
+    assert call(arr=(bca.SlotStruct * 2)(_slot(L), _slot(L, n=20))) == 2  # bf16 slots
+    assert call(arr=(bca.SlotStruct * 2)(_slot(L, dt=1), _slot(L, dt=1, n=20))) == 2  # fp8_v
+    assert call(scratch=None) == 1
+    assert call(scratch=ctypes.c_void_p((1 << 28) + 16)) == 1  # not 256-byte aligned
+    assert call(bytes=need - 1) == 3
+
+
 def test_selftest_wait_rejects_bad_bounds(L):
     assert L.bca_selftest_wait_timeout(None, 10_000_000, None) == 1
     assert L.bca_selftest_wait_timeout(FAKE, 10, None) == 1
