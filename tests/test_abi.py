@@ -236,6 +236,7 @@ def test_binding_rejects_host_tensors_before_the_library_is_called():
     x = torch.zeros((4, 2, 128), dtype=torch.bfloat16)
     calls = [
         lambda: bca.step_attend(x, x, x, x, [0, 4], [], 0.1),
+        lambda: bca.step_attend_q8(x, x, x, x, [0, 4], [], 0.1),
         lambda: bca.prefill(x, x, x, x, [0, 4], 0.1),
         lambda: bca.qk_norm_rope(x, None, None, None, None, None),
         lambda: bca.ulysses_pack(x, torch.empty_like(x), 2),
