@@ -71,6 +71,7 @@ class StepGraphDesc(ctypes.Structure):
         ("n_req", ctypes.c_int32), ("heads", ctypes.c_int32), ("head_dim", ctypes.c_int32),
         ("scale", ctypes.c_float), ("workspace", ctypes.c_void_p),
         ("workspace_bytes", ctypes.c_size_t), ("dev_status", ctypes.c_void_p),
+        ("q8_scratch", ctypes.c_void_p), ("q8_scratch_bytes", ctypes.c_size_t),
     ]
 
 
@@ -468,7 +469,8 @@ def ulysses_unpack(recv, x, n_ranks: int, stream=None):
 
 
 class StepGraph:
-    """The cached-step attention of every layer of one layout as one CUDA graph.
+    """The cached-step attention of every layer of one layout as one CUDA graph
+    (with q8_scratch: the e4m3-Q cached step, step_attend_q8, of e4m3 slots).
 
     q_layers..o_layers: per-layer packed target tensors [sum T_r, H, 128] (bf16,
     CUDA); slots_per_layer: per-layer lists of KVSlot (one per request, in
@@ -477,7 +479,7 @@ class StepGraph:
     graph exists; close() or garbage collection releases it."""
 
     def __init__(self, q_layers, k_layers, v_layers, o_layers, cu_target, slots_per_layer,
-                 scale: float, workspace=None, dev_status=None):
+                 scale: float, workspace=None, dev_status=None, q8_scratch=None):
         n = len(q_layers)
         assert n == len(k_layers) == len(v_layers) == len(o_layers) == len(slots_per_layer)
         n_req = len(slots_per_layer[0])
@@ -490,9 +492,10 @@ class StepGraph:
             _need(q_layers[l].shape == q_layers[0].shape, call, "layers must share one layout")
         _aux(workspace, call, "workspace", q_layers[0].device)
         _aux(dev_status, call, "dev_status", q_layers[0].device, torch.int32)
+        _aux(q8_scratch, call, "q8_scratch", q_layers[0].device)
         _, H, d = q_layers[0].shape
         self._keep = (list(q_layers), list(k_layers), list(v_layers), list(o_layers),
-                      [list(sl) for sl in slots_per_layer], workspace, dev_status)
+                      [list(sl) for sl in slots_per_layer], workspace, dev_status, q8_scratch)
         ptrs = lambda ts: (ctypes.c_void_p * n)(*[t.data_ptr() for t in ts])
         self._q, self._k, self._v, self._o = (ptrs(q_layers), ptrs(k_layers), ptrs(v_layers),
                                               ptrs(o_layers))
@@ -506,7 +509,9 @@ class StepGraph:
             ctypes.cast(self._slots, ctypes.c_void_p), self._cu, n_req, H, d, float(scale),
             None if workspace is None else workspace.data_ptr(),
             0 if workspace is None else workspace.numel() * workspace.element_size(),
-            None if dev_status is None else dev_status.data_ptr())
+            None if dev_status is None else dev_status.data_ptr(),
+            None if q8_scratch is None else q8_scratch.data_ptr(),
+            0 if q8_scratch is None else q8_scratch.numel() * q8_scratch.element_size())
         self.device = q_layers[0].device
         self._g = ctypes.c_void_p()
         import torch

@@ -736,6 +736,9 @@ extern "C" bca_status bca_step_graph_create(const bca_step_graph_desc* d, bca_st
   if (!prepare_attn<1>() || !prepare_attn<8>() || !prepare_attn<64>() || sm_count() <= 0 ||
       !get_encode())
     return BCA_ERR_CUDA;
+  const bool q8 = d->q8_scratch != nullptr;
+  if (q8 && (!prepare_attn<1, true>() || !prepare_attn<8, true>() || !prepare_attn<64, true>()))
+    return BCA_ERR_CUDA;
   cudaStream_t cs = nullptr;
   if (cudaStreamCreateWithFlags(&cs, cudaStreamNonBlocking) != cudaSuccess) return BCA_ERR_CUDA;
   // Each layer's call checks its arguments before it records anything; the first
@@ -746,10 +749,10 @@ extern "C" bca_status bca_step_graph_create(const bca_step_graph_desc* d, bca_st
     st = BCA_ERR_CUDA;
   } else {
     for (int l = 0; l < d->n_layers && st == BCA_OK; ++l)
-      st = bca_step_attend(d->q_t[l], d->k_t[l], d->v_t[l], d->o_t[l], d->cu_target,
-                           d->slots + static_cast<size_t>(l) * d->n_req, d->n_req, d->heads,
-                           d->head_dim, d->scale, d->workspace, d->workspace_bytes,
-                           d->dev_status, cs);
+      st = step_attend_impl(d->q_t[l], d->k_t[l], d->v_t[l], d->o_t[l], d->cu_target,
+                            d->slots + static_cast<size_t>(l) * d->n_req, d->n_req, d->heads,
+                            d->head_dim, d->scale, d->workspace, d->workspace_bytes, q8,
+                            d->q8_scratch, d->q8_scratch_bytes, d->dev_status, cs);
     if (cudaStreamEndCapture(cs, &graph) != cudaSuccess && st == BCA_OK) st = BCA_ERR_CUDA;
   }
   cudaStreamDestroy(cs);

@@ -281,7 +281,8 @@ bca_status bca_ulysses_unpack(const void* recv, void* x, int64_t rows_local, int
  * the outputs are bit-identical to the eager bca_step_attend calls on the same
  * contents.  Pointers, row counts, slot shapes and n_tokens are fixed when the
  * graph is created; another layout needs another graph.  bf16 and e4m3 caches are
- * captured alike.  The graph object lives in host memory (the CUDA driver keeps
+ * captured alike, and with q8_scratch the e4m3-Q step (its Q quantisation
+ * included) is recorded.  The graph object lives in host memory (the CUDA driver keeps
  * its own copy of the recorded launches); the library allocates no device memory. */
 typedef struct bca_step_graph bca_step_graph; /* opaque */
 
@@ -298,6 +299,9 @@ typedef struct {
   void* workspace;          /* as bca_step_attend (nullable), shared by the layers */
   size_t workspace_bytes;
   int32_t* dev_status;      /* nullable */
+  void* q8_scratch;         /* nullable; non-NULL: the layers' bca_step_attend_q8 calls
+                               are recorded instead (e4m3 slots), sharing this scratch */
+  size_t q8_scratch_bytes;
 } bca_step_graph_desc;
 
 /* Builds the graph on the current device.  Errors: BCA_ERR_INVALID_ARG for a NULL
@@ -308,7 +312,8 @@ bca_status bca_step_graph_create(const bca_step_graph_desc* desc, bca_step_graph
 /* Enqueues one replay (all layers) on `stream` (of the graph's device). */
 bca_status bca_step_graph_launch(const bca_step_graph* graph, void* stream);
 
-/* Kernel launches one replay performs (attention + chunk-merge kernels). */
+/* Kernel launches one replay performs (attention + chunk-merge kernels, and the Q
+ * quantisation kernels of an e4m3-Q graph). */
 int32_t bca_step_graph_kernel_nodes(const bca_step_graph* graph);
 
 /* Releases the graph (NULL is ignored).  No replay may be pending on the GPU. */
@@ -327,9 +332,10 @@ void bca_set_wait_timeout_ns(uint64_t timeout_ns);
  * device timeout without hanging or faulting the GPU. */
 bca_status bca_selftest_wait_timeout(int32_t* dev_status, uint64_t timeout_ns, void* stream);
 
-/* Self-check of the software 2^x the attention kernels evaluate on the FMA pipe
- * for part of each softmax row (range reduction to [-1/2, 1/2] plus a degree-3
- * minimax polynomial; inputs <= -127 give exactly 0).  Writes it to y_poly and the
+/* Self-check of the software 2^x that the attention kernel can evaluate on the FMA
+ * pipe for part of each softmax row (builds with BCA_POLY_PAIRS > 0; the default
+ * build uses MUFU ex2 only): range reduction to [-1/2, 1/2] plus a degree-3
+ * minimax polynomial; inputs <= -127 give exactly 0.  Writes it to y_poly and the
  * hardware ex2.approx to y_mufu for the n device floats x[].  Diagnostic only. */
 bca_status bca_selftest_exp2(const float* x, float* y_poly, float* y_mufu, int32_t n,
                              void* stream);

@@ -134,3 +134,33 @@ def test_graph_without_target_rows_is_a_no_op(cuda_device):
     assert g.kernel_nodes == 0
     g.launch()
     torch.cuda.synchronize()
+
+
+def test_e4m3_q_graph_replay_equals_eager(cuda_device):
+    """With a q8 scratch the graph records each layer's bca_step_attend_q8 (its Q
+    quantisation kernels included): replays, also after new contents are written
+    into the same buffers, are bit-identical to the eager e4m3-Q calls."""
+    H = 4
+    cu, L = _layout(cuda_device, H, [256, 131, 300], [128, 0, 77], layers=2, mode="fp8",
+                    seed=70)
+    ws = bca.step_workspace(cuda_device)
+    scratch = bca.step_q8_scratch(cu[-1], len(cu) - 1, H, cuda_device)
+    status = torch.zeros(1, dtype=torch.int32, device=cuda_device)
+    g = bca.StepGraph([x["q"] for x in L], [x["k"] for x in L], [x["v"] for x in L],
+                      [x["o"] for x in L], cu, [[s for s, *_ in x["slots"]] for x in L], SCALE,
+                      workspace=ws, dev_status=status, q8_scratch=scratch)
+    assert g.kernel_nodes >= 2 * 4  # per layer: 3 Q-quantisation kernels + attention
+    for rnd in range(2):
+        if rnd:
+            for l, x in enumerate(L):
+                x["q"].copy_(randn_bf16(tuple(x["q"].shape), 9500 + l, cuda_device))
+        g.launch()
+        torch.cuda.synchronize()
+        assert int(status.item()) == 0
+        for x in L:
+            o = torch.empty_like(x["q"])
+            bca.step_attend_q8(x["q"], x["k"], x["v"], o, cu, [s for s, *_ in x["slots"]],
+                               SCALE, workspace=ws)
+            torch.cuda.synchronize()
+            assert torch.equal(x["o"], o)
+    g.close()
