@@ -15,8 +15,12 @@ e2e    = the same through the Python/C-ABI calls with pinned HOST buffers: every
          the timed region.
 roofline: the dominant kernel (cached-step attention) against the measured
          dense bf16 tensor peak; cpu_baseline: the fp64 oracle on the host cores.
-kv_store = bca_kv_store of every request's prefix, GB/s on the algorithmic bytes
-         (and on the bytes moved) against the measured HBM copy bandwidth.
+kv_store = bca_kv_store_batch of every request's prefix (one launch), GB/s on the
+         algorithmic bytes against the measured HBM copy bandwidth.
+per_workload_one_layer = one layer of each of the T2I, 4-ref edit, native-2K and
+         serving workloads: prefill, store and cached step timed on their own.
+oracle_extra = the oracle on the tiny workload in full, and its rate on samples of
+         the larger workloads extrapolated to 40 steps x 32 layers.
 qk_norm_rope = the Q/K RMS norm + rotary embedding call on the cached step's
          target rows, GB/s against the measured HBM copy bandwidth.
 graph  = the same pass with each step's cached-step calls of all layers replayed
@@ -64,10 +68,37 @@ def step_flops(req, H, d=128) -> float:
     return 4.0 * d * H * req.target * (req.prefix + req.target)
 
 
+# Launch counts, mirroring the library's schedules (a chunk-merge kernel follows the
+# attention kernel when the schedule splits units along the keys).
+def step_split_launches(reqs, H, sms) -> int:
+    """Cached step: units = sum_r H * ceil(T_r / 256); the last partial round is
+    split when at most half the SMs would be busy in it."""
+    units = sum(H * -(-r.target // 256) for r in reqs if r.target > 0)
+    return int(units > sms and units % sms != 0 and sms // (units % sms) >= 2)
+
+
+def prefill_split_launches(req, H, sms) -> int:
+    """Prefill with a workspace: Q-tile pairs heaviest first; the heavy ones' (at
+    least half the heaviest) last partial round is split."""
+    off, S = req.offsets, req.seq_len
+    nqp = -(-S // 256)
+    tiles = []
+    for qp in range(nqp - 1, -1, -1):
+        last = min(S, (qp + 1) * 256) - 1
+        lim = next(o for o in off[1:] if last < o)
+        tiles += [-(-lim // 128)] * H
+    heavy = sum(1 for t in tiles if 2 * t >= tiles[0])
+    rem = heavy % sms
+    if rem == 0:
+        return 0
+    k = min(sms // rem, 8, sms // rem, min(tiles[heavy - rem:heavy]))
+    return int(k >= 2)
+
+
 # DRAM traffic of one cached-step attention launch (dram__bytes_read.sum +
-# dram__bytes_write.sum) from the ncu capture summarised in
-# profiles/attn_fwd_cached_step_t2i1024.md, valid only for the kernel sources it was
-# taken from (their sha256 below); any later change reports null instead.
+# dram__bytes_write.sum) from one ncu capture of the T2I cached step, valid only for
+# the kernel sources it was taken from (their sha256 below); any later change
+# reports null instead.
 ATTN_TRAFFIC = {"bytes_per_launch": 109.24e6 + 15.60e6, "workload": 1,
                 "sources": {"block_causal_attention_dit_b200/csrc/attn_kernel.cuh":
                             "62fa4d412f679f5ec6ff71e4bdc882816523bcb78718570f549bc38ce9976a9f",
@@ -203,18 +234,11 @@ class Runner:
         self.flops_step_call = sum(step_flops(r, H) for r in reqs)
         self.flops_steps = self.flops_step_call * layers * (wl.steps - 1)
         self.flops = self.flops_prefill + self.flops_steps
-        kv_store_launches = 1 if wl.kv_dtype == "bf16" else 4
-        self.launches_per_step = (layers * len(reqs) * (1 + kv_store_launches)
-                                  + layers * (wl.steps - 1) * (1 + self.split_launches()))
-
-    def split_launches(self) -> int:
-        """1 if cached steps also launch the chunk-merge kernel (the last partial
-        round of units is split along the keys), else 0 -- mirrors the library's
-        schedule: units = sum_r H * ceil(T_r / 256) over the SMs."""
-        import torch
-        sms = torch.cuda.get_device_properties(self.device).multi_processor_count
-        units = sum(self.H * -(-r.target // 256) for r in self.wl.requests)
-        return int(units > sms and units % sms != 0 and sms // (units % sms) >= 2)
+        sms = torch.cuda.get_device_properties(device).multi_processor_count
+        # per prefill: attention (+ chunk merge when split) + one store launch
+        self.launches_per_step = (
+            layers * sum(2 + prefill_split_launches(r, H, sms) for r in reqs)
+            + layers * (wl.steps - 1) * (1 + step_split_launches(reqs, H, sms)))
 
     def step(self, events=None):
         """One pass of the hot path.  events: optional list collecting
@@ -229,7 +253,7 @@ class Runner:
                         q, k, v = self.pre[l][i]
                         bca.prefill(q, k, v, self.o_pre[i], r.offsets, wl.scale,
                                     slot=self.slots[l][i], epoch=self.epoch,
-                                    dev_status=self.status)
+                                    dev_status=self.status, workspace=self.workspace)
                 else:
                     q, k, v = self.pool[(l * (wl.steps - 1) + s - 1) % len(self.pool)]
                     if events is not None:
@@ -267,7 +291,7 @@ class Runner:
             for i, r in enumerate(wl.requests):
                 q, k, v = self.pre[l][i]
                 bca.prefill(q, k, v, self.o_pre[i], r.offsets, wl.scale, slot=self.slots[l][i],
-                            epoch=self.epoch, dev_status=self.status)
+                            epoch=self.epoch, dev_status=self.status, workspace=self.workspace)
         for s in range(1, wl.steps):
             g = self.graph_for_step(s)
             if events is not None:
@@ -357,7 +381,8 @@ class E2ERunner:
                         self._call(b, self.h_pre[l % len(self.h_pre)][i], (q, k, v),
                                    lambda q=q, k=k, v=v, o=o, req=req, slot=slot: bca.prefill(
                                        q, k, v, o, req.offsets, wl.scale, slot=slot,
-                                       epoch=r.epoch, dev_status=r.status),
+                                       epoch=r.epoch, dev_status=r.status,
+                                       workspace=r.workspace),
                                    (o,), (self.h_out_pre[b][i],))
                         b ^= 1
                 else:
@@ -435,41 +460,168 @@ def norm_rope_leg(device, peaks, rows: int, heads: int, calls: int = 20):
 
 
 def store_leg(runner, peaks, reps: int = 5):
-    """bca_kv_store of every request's prefix (layer 0's inputs) into fresh slots of
-    the workload's cache dtype: GB/s on the algorithmic bytes (K and V prefix rows
-    read once, the cache written once, the scales) and on the bytes moved (an e4m3
-    tensor's prefix is read twice: absmax pass, then encode pass)."""
+    """bca_kv_store_batch of every request's prefix (layer 0's inputs) into fresh
+    slots of the workload's cache dtype, one kernel launch per store, timed with
+    events around each enqueue: GB/s on the algorithmic bytes (K and V prefix rows
+    read once, the cache written once, the scales)."""
     import torch
     bca, wl, H = runner.bca, runner.wl, runner.H
     dt = {"bf16": (2, 2), "fp8_v": (2, 1), "fp8": (1, 1)}[wl.kv_dtype]  # bytes of K, V codes
     slots = [bca.KVSlot(max(r.prefix, 1), H, wl.kv_dtype, device=runner.device)
              for r in wl.requests]
-    alg = moved = 0
+    alg = 0
     for r in wl.requests:
         n = r.prefix * H * 128
         alg += 2 * n * 2 + n * (dt[0] + dt[1]) + (8 * H if wl.kv_dtype != "bf16" else 0)
-        moved += 2 * n * 2 + n * (dt[0] + dt[1]) + n * 2 * (int(dt[0] == 1) + int(dt[1] == 1))
 
-    def run(epoch):
-        for i, r in enumerate(wl.requests):
-            q, k, v = runner.pre[0][i]
-            bca.kv_store(k, v, r.prefix, slots[i], epoch)
-
-    run(1)
+    items = [(runner.pre[0][i][1], runner.pre[0][i][2], r.prefix, slots[i])
+             for i, r in enumerate(wl.requests)]
+    bca.kv_store_batch(items, 1)
     torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for i in range(reps):
-        run(2 + i)
-    e1.record()
+    ev = []
+    for i in range(reps):  # one enqueue (one kernel launch) per store, events around it
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        bca.kv_store_batch(items, 2 + i)
+        e1.record()
+        ev.append((e0, e1))
     torch.cuda.synchronize()
-    ms = e0.elapsed_time(e1) / reps
+    ms = sum(a.elapsed_time(b) for a, b in ev) / reps
     peak = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
     gbs = alg / (ms / 1e3) / 1e9
     return {"bound": "hbm", "kv_cache": wl.kv_dtype, "prefix_rows": [r.prefix for r in wl.requests],
             "ms_per_store": ms, "algorithmic_bytes": alg, "achieved": gbs, "peak": peak,
-            "unit": "GB/s", "frac": gbs / peak, "moved_bytes": moved,
-            "moved_gbs": moved / (ms / 1e3) / 1e9}
+            "unit": "GB/s", "frac": gbs / peak, "launches_per_store": 1,
+            "timing": "CUDA events around each bca_kv_store_batch enqueue"}
+
+
+def config_leg(index: int, device, peaks, reps: int = 3):
+    """One layer of workload `index` on its own: the prefill of every request
+    (bca_prefill with the workspace, attention only), the prefix store of all
+    requests (one bca_kv_store_batch launch) and one cached step of all requests
+    (bca_step_attend), each timed with CUDA events around its enqueues.  Two cached-
+    step input sets alternate (larger than L2 together).  The 40-step projection is
+    32 layers x (prefill + store) + 32 x 39 cached steps from these timings."""
+    import torch
+    import block_causal_attention_dit_b200 as bca
+    from block_causal_attention_dit_b200 import workloads as W
+    wl = W.workload(index)
+    H, reqs = wl.heads, wl.requests
+    ws = bca.step_workspace(device)
+    status = torch.zeros(1, dtype=torch.int32, device=device)
+    pre = [W.qkv(wl, 0, 0, i, device) for i in range(len(reqs))]
+    o_pre = [torch.empty_like(x[0]) for x in pre]
+    slots = [bca.KVSlot(max(r.prefix, 1), H, wl.kv_dtype, device=device) for r in reqs]
+    items = [(pre[i][1], pre[i][2], r.prefix, slots[i]) for i, r in enumerate(reqs)]
+    sets = []
+    for l in range(2):
+        per = [W.qkv(wl, l, 1, i, device) for i in range(len(reqs))]
+        sets.append(tuple(torch.cat([x[j] for x in per]) for j in range(3)))
+        del per
+    o_step = torch.empty_like(sets[0][0])
+    cu = [0]
+    for r in reqs:
+        cu.append(cu[-1] + r.target)
+    epoch = [0]
+
+    def prefill():
+        for i, r in enumerate(reqs):
+            bca.prefill(pre[i][0], pre[i][1], pre[i][2], o_pre[i], r.offsets, wl.scale,
+                        dev_status=status, workspace=ws)
+
+    def store():
+        epoch[0] += 1
+        bca.kv_store_batch(items, epoch[0], dev_status=status)
+
+    def step(n):
+        q, k, v = sets[n % 2]
+        bca.step_attend(q, k, v, o_step, cu, slots, wl.scale, workspace=ws, dev_status=status)
+
+    def time_it(fn, n):
+        fn(0)
+        torch.cuda.synchronize()
+        ev = []
+        for i in range(n):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            fn(i)
+            e1.record()
+            ev.append((e0, e1))
+        torch.cuda.synchronize()
+        return statistics.median(a.elapsed_time(b) for a, b in ev)
+
+    store()
+    torch.cuda.synchronize()
+    p_ms = time_it(lambda i: prefill(), reps)
+    s_ms = time_it(lambda i: store(), reps)
+    c_ms = time_it(step, 2 * reps)
+    if int(status.item()) != 0:
+        raise RuntimeError(f"device status {int(status.item())} (workload {index})")
+    pk_sus = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
+    pk_burst = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    f_pre = sum(prefill_flops(r, H) for r in reqs)
+    f_step = sum(step_flops(r, H) for r in reqs)
+    cb = {"bf16": 4, "fp8_v": 3, "fp8": 2}[wl.kv_dtype]  # code bytes per element, K + V
+    st_bytes = sum(r.prefix * H * 128 * (4 + cb) + (8 * H if wl.kv_dtype != "bf16" else 0)
+                   for r in reqs)
+    t_pre, t_step = f_pre / (p_ms / 1e3) / 1e12, f_step / (c_ms / 1e3) / 1e12
+    layers = wl.layers
+    total_ms = layers * (p_ms + s_ms) + layers * (wl.steps - 1) * c_ms
+    total_flops = layers * (f_pre + (wl.steps - 1) * f_step)
+    return {"workload": wl.name, "kv_cache": wl.kv_dtype,
+            "prefill_ms_per_layer": p_ms, "prefill_tflops": t_pre,
+            "prefill_frac_sustained": t_pre / pk_sus,
+            "store_ms_per_layer": s_ms, "store_gbs": st_bytes / (s_ms / 1e3) / 1e9,
+            "store_frac_hbm": st_bytes / (s_ms / 1e3) / 1e9 / hbm,
+            "cached_step_ms_per_layer": c_ms, "cached_step_tflops": t_step,
+            "cached_step_frac_sustained": t_step / pk_sus,
+            "cached_step_frac_burst": t_step / pk_burst,
+            "projected_ms_per_40step_attn": total_ms,
+            "projected_tflops_per_generation": total_flops / (total_ms / 1e3) / 1e12,
+            "projection": f"{layers} layers x (prefill + store) + {layers} x {wl.steps - 1} "
+                          f"cached steps, from one layer's median times"}
+
+
+def oracle_leg(seconds: float):
+    """The oracle on the host cores: the tiny workload in full (prefill of the whole
+    sequence, then the cached step), and, for the T2I, 4-ref edit and native-2K
+    workloads, a bounded sample of one cached step whose rate is extrapolated to the
+    whole 40-step x 32-layer attention (labelled as such)."""
+    import oracle
+    from block_causal_attention_dit_b200 import workloads as W
+    wl = W.workload(0)
+    r = wl.requests[0]
+    q0, k0, v0 = W.qkv(wl, 0, 0, 0, "cpu")
+    q1, k1, v1 = W.qkv(wl, 0, 1, 0, "cpu")
+    t0 = time.perf_counter()
+    oracle.prefill(q0, k0, v0, r.offsets, wl.scale)
+    t1 = time.perf_counter()
+    P = r.prefix
+    oracle.cached_step(q1, k1, v1, k0[:P].permute(1, 0, 2).contiguous(),
+                       v0[:P].permute(1, 0, 2).contiguous(), P, wl.scale)
+    t2 = time.perf_counter()
+    out = {"cores": oracle.max_threads(),
+           "tiny_full": {"prefill_s": t1 - t0, "cached_step_s": t2 - t1,
+                         "tflops": (prefill_flops(r, wl.heads) + step_flops(r, wl.heads))
+                         / (t2 - t0) / 1e12}}
+    for idx in (1, 2, 3):
+        w = W.workload(idx)
+        smp = oracle_sample(w, seconds)
+        rr = w.requests[0]
+        total = w.layers * (prefill_flops(rr, w.heads) + (w.steps - 1) * step_flops(rr, w.heads))
+        out[w.name] = {"sample_tflops": smp["value"], "sample": smp["sample"],
+                       "extrapolated_s_per_40step_attn": total / (smp["value"] * 1e12),
+                       "label": "extrapolated"}
+    return out
+
+
+# NVIDIA's datasheet figure for the B200's dense BF16 tensor throughput: the HGX B200
+# datasheet gives 36 PFLOPS FP16/BF16 for 8 GPUs with 2:4 sparsity, i.e. 2.25 PFLOPS
+# dense per GPU.
+DATASHEET_BF16_DENSE_TFLOPS = 2250.0
+DATASHEET_SOURCE = ("NVIDIA HGX B200 datasheet: FP16/BF16 tensor 36 PFLOPS per 8 GPUs with "
+                    "2:4 sparsity = 2.25 PFLOPS dense per GPU")
 
 
 def q8_leg(device, peaks, calls: int = 10):
@@ -611,6 +763,11 @@ def main():
     ap.add_argument("--no-q8", action="store_true",
                     help="skip the e4m3-Q cached-step leg (serving workload, one layer)")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--no-configs", action="store_true",
+                    help="skip the per-workload one-layer leg (T2I, 4-ref edit, native 2K, "
+                         "serving)")
+    ap.add_argument("--no-oracle-extra", action="store_true",
+                    help="skip the oracle's tiny-workload timing and extrapolations")
     args = ap.parse_args()
 
     from block_causal_attention_dit_b200 import workloads as W
@@ -719,6 +876,13 @@ def main():
     if not args.no_q8 and n_gpus == 1:
         q8 = q8_leg(device, peaks)
 
+    configs = None
+    if not args.no_configs and n_gpus == 1:
+        configs = {}
+        for idx in (1, 2, 3, 4):
+            configs[str(idx)] = config_leg(idx, device, peaks)
+            torch.cuda.empty_cache()
+
     e2e = None
     if not args.no_e2e:
         e = E2ERunner(runner)
@@ -731,6 +895,9 @@ def main():
     cpu = None
     if rank == 0 and n_gpus == 1 and not args.no_cpu_baseline:
         cpu = oracle_sample(wl, args.cpu_seconds)
+    oracle_extra = None
+    if rank == 0 and n_gpus == 1 and not args.no_oracle_extra:
+        oracle_extra = oracle_leg(min(args.cpu_seconds, 4.0))
 
     line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": n_gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
@@ -741,8 +908,11 @@ def main():
             "pct_of_bf16_peak": {"sustained": 100 * achieved / peak_sus,
                                  "burst": 100 * achieved / peak_burst, "source": peak_src},
             "prefill_and_store_ms_per_step": ms_per_step - sum(step_ms) / args.steps,
+            "datasheet_bf16": {"tflops": DATASHEET_BF16_DENSE_TFLOPS, "source": DATASHEET_SOURCE,
+                               "cached_step_frac": achieved / DATASHEET_BF16_DENSE_TFLOPS},
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "graph": graph,
             "qk_norm_rope": norm, "kv_store": store, "fp8_q8_step": q8,
+            "per_workload_one_layer": configs, "oracle_extra": oracle_extra,
             "gpu_launches": runner.launches_per_step * args.steps, "clocks": clocks}
     if rank == 0:
         print(json.dumps(line), flush=True)

@@ -8,6 +8,8 @@ three calls of the method mirror include/bca.h one to one:
       (every block but the last) into a KVSlot.
   kv_store(k, v, n_prefix, slot, epoch)
       prefix K/V into a KVSlot, bf16 or OFP8 E4M3 with per-head scales.
+  kv_store_batch([(k, v, n_prefix, slot), ...], epoch)
+      the same for the requests of a batch, in one launch.
   step_attend(q_t, k_t, v_t, o_t, cu_target, slots, scale)
       cached-step attention of packed target rows over [cache ; own K/V] for a
       ragged batch of requests at the same phase.
@@ -31,7 +33,7 @@ import os
 
 __all__ = [
     "BcaError", "KVSlot", "KV_BF16", "KV_FP8_V", "KV_FP8_KV", "MAX_BLOCKS", "MAX_BATCH",
-    "lib", "prefill", "kv_store", "step_attend", "step_workspace", "step_workspace_bytes",
+    "lib", "prefill", "kv_store", "kv_store_batch", "step_attend", "step_workspace", "step_workspace_bytes",
     "step_attend_q8", "step_q8_scratch", "step_q8_scratch_bytes", "q8_views",
     "StepGraph", "qk_norm_rope", "ulysses_pack", "ulysses_unpack",
     "slot_bytes", "set_wait_timeout_ns",
@@ -51,7 +53,7 @@ MAX_BATCH = 64
 
 STATUS_NAMES = {
     0: "BCA_OK", 1: "BCA_ERR_INVALID_ARG", 2: "BCA_ERR_UNSUPPORTED", 3: "BCA_ERR_CAPACITY",
-    4: "BCA_ERR_STATE", 5: "BCA_ERR_CUDA", 6: "BCA_ERR_DEVICE_TIMEOUT",
+    4: "BCA_ERR_STATE", 5: "BCA_ERR_CUDA", 6: "BCA_ERR_DEVICE_TIMEOUT", 7: "BCA_ERR_NONFINITE",
 }
 
 
@@ -86,6 +88,14 @@ class SlotStruct(ctypes.Structure):
     ]
 
 
+class StoreItemStruct(ctypes.Structure):
+    """Mirror of bca_kv_store_item."""
+    _fields_ = [
+        ("k", ctypes.c_void_p), ("v", ctypes.c_void_p), ("n_prefix", ctypes.c_int32),
+        ("row_stride_elems", ctypes.c_int32), ("slot", ctypes.POINTER(SlotStruct)),
+    ]
+
+
 _lib = None
 
 
@@ -108,8 +118,13 @@ def lib():
     L.bca_kv_slot_init.argtypes = [SP, P, i32, i32, i32, ctypes.c_int]
     L.bca_kv_store.restype = ctypes.c_int
     L.bca_kv_store.argtypes = [P, P, i32, i32, SP, u32, P, P]
+    L.bca_kv_store_batch.restype = ctypes.c_int
+    L.bca_kv_store_batch.argtypes = [ctypes.POINTER(StoreItemStruct), i32, u32, P, P]
     L.bca_prefill.restype = ctypes.c_int
     L.bca_prefill.argtypes = [P, P, P, P, i32, P, i32, i32, i32, f32, SP, u32, P, P]
+    L.bca_prefill_ws.restype = ctypes.c_int
+    L.bca_prefill_ws.argtypes = [P, P, P, P, i32, P, i32, i32, i32, f32, SP, u32, P,
+                                 ctypes.c_size_t, P, P]
     L.bca_step_attend.restype = ctypes.c_int
     L.bca_step_attend.argtypes = [P, P, P, P, P, SP, i32, i32, i32, f32, P, ctypes.c_size_t,
                                   P, P]
@@ -293,13 +308,9 @@ class KVSlot:
         return int(self.struct.epoch)
 
 
-def kv_store(k, v, n_prefix: int, slot: KVSlot, epoch: int, row_stride: int | None = None,
-             dev_status=None, stream=None):
-    """Prefix rows [0, n_prefix) of k and v into the slot.  k and v are bf16 CUDA
-    tensors [rows, H, d] or [rows, H*d] whose rows are dense and `row_stride`
-    elements apart (default: their stride(0)); both use the same row stride."""
+def _store_args(call, k, v, n_prefix, slot, row_stride):
+    """Checks of one store's tensors; returns the row stride in elements."""
     import torch
-    call = "bca_kv_store"
     for name, t in (("k", k), ("v", v)):
         _cuda(t, call, name, torch.bfloat16, k.device)
         _need(t.dim() in (2, 3) and t.stride(-1) == 1 and
@@ -313,28 +324,70 @@ def kv_store(k, v, n_prefix: int, slot: KVSlot, epoch: int, row_stride: int | No
     _need(k.shape[0] <= 1 or (k.stride(0) == row_stride and v.stride(0) == row_stride), call,
           "k and v rows must be row_stride elements apart")
     _slot_device(slot, call, k.device)
+    return int(row_stride)
+
+
+def kv_store(k, v, n_prefix: int, slot: KVSlot, epoch: int, row_stride: int | None = None,
+             dev_status=None, stream=None):
+    """Prefix rows [0, n_prefix) of k and v into the slot.  k and v are bf16 CUDA
+    tensors [rows, H, d] or [rows, H*d] whose rows are dense and `row_stride`
+    elements apart (default: their stride(0)); both use the same row stride."""
+    import torch
+    call = "bca_kv_store"
+    row_stride = _store_args(call, k, v, n_prefix, slot, row_stride)
     _aux(dev_status, call, "dev_status", k.device, torch.int32)
     _check(lib().bca_kv_store(_ptr(k), _ptr(v), int(n_prefix), int(row_stride),
                               ctypes.byref(slot.struct), int(epoch), _ptr(dev_status),
                               _stream(stream, k.device)), "bca_kv_store")
 
 
-def prefill(q, k, v, o, block_offsets, scale: float, slot: KVSlot | None = None,
-            epoch: int = 0, dev_status=None, stream=None):
+def kv_store_batch(items, epoch: int, dev_status=None, stream=None):
+    """kv_store for several requests in one launch.  items: (k, v, n_prefix, slot) or
+    (k, v, n_prefix, slot, row_stride) tuples, one per request, distinct slots."""
     import torch
-    call = "bca_prefill"
+    call = "bca_kv_store_batch"
+    _need(len(items) >= 1, call, "at least one item")
+    arr = (StoreItemStruct * len(items))()
+    keep = []
+    for i, it in enumerate(items):
+        k, v, n_prefix, slot = it[:4]
+        rs = _store_args(call, k, v, n_prefix, slot, it[4] if len(it) > 4 else None)
+        _need(k.device == items[0][0].device, call, "all items on one device")
+        arr[i] = StoreItemStruct(k.data_ptr(), v.data_ptr(), int(n_prefix), rs,
+                                 ctypes.pointer(slot.struct))
+        keep.append(slot)
+    dev = items[0][0].device
+    _aux(dev_status, call, "dev_status", dev, torch.int32)
+    _check(lib().bca_kv_store_batch(arr, len(items), int(epoch), _ptr(dev_status),
+                                    _stream(stream, dev)), call)
+
+
+def prefill(q, k, v, o, block_offsets, scale: float, slot: KVSlot | None = None,
+            epoch: int = 0, dev_status=None, stream=None, workspace=None):
+    """Block-causal attention of [S, H, 128]; with `workspace` (step_workspace())
+    through bca_prefill_ws, whose schedule splits the heavy Q-tile pairs' last round."""
+    import torch
+    call = "bca_prefill" if workspace is None else "bca_prefill_ws"
     _rows_tensor(q, call, "q")
     for name, t in (("k", k), ("v", v), ("o", o)):
         _rows_tensor(t, call, name, like=q)
     if slot is not None:
         _slot_device(slot, call, q.device)
     _aux(dev_status, call, "dev_status", q.device, torch.int32)
+    _aux(workspace, call, "workspace", q.device)
     S, H, d = q.shape
     off = _i32_array(block_offsets)
-    _check(lib().bca_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(o), S, off, len(off) - 1, H, d,
-                             float(scale), None if slot is None else ctypes.byref(slot.struct),
-                             int(epoch), _ptr(dev_status), _stream(stream, q.device)),
-           "bca_prefill")
+    sl = None if slot is None else ctypes.byref(slot.struct)
+    if workspace is None:
+        rc = lib().bca_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(o), S, off, len(off) - 1, H, d,
+                               float(scale), sl, int(epoch), _ptr(dev_status),
+                               _stream(stream, q.device))
+    else:
+        rc = lib().bca_prefill_ws(_ptr(q), _ptr(k), _ptr(v), _ptr(o), S, off, len(off) - 1, H,
+                                  d, float(scale), sl, int(epoch), _ptr(workspace),
+                                  workspace.numel() * workspace.element_size(),
+                                  _ptr(dev_status), _stream(stream, q.device))
+    _check(rc, call)
 
 
 def step_workspace_bytes() -> int:

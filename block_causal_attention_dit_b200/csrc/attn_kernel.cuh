@@ -66,28 +66,6 @@ constexpr uint32_t kOtherRegs = 104;
 static_assert(128 * (2 * kSoftmaxRegs + kOtherRegs) <= kAttnThreads * kLaunchRegs,
               "register split exceeds the launch allocation");
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
-#ifndef BCA_POLY_PAIRS
-#define BCA_POLY_PAIRS 0
-#endif
-// Of every 8 column pairs, kPolyPairs are exponentiated on the FMA pipe by the
-// software exp2 (the rest by MUFU ex2).  Measured on B200 for the T2I cached step
-// (kernel alone, TFLOP/s, two runs each in one process order): 0 -> 1145.7 / 1145.4,
-// 1 -> 1127.2 / 1126.5, 2 -> 1103.4; so the default is 0.
-constexpr int kPolyPairs = BCA_POLY_PAIRS;
-// P is handed from the softmax to the MMA in kPHalves parts (1: whole tile; 2: two
-// halves of 64 keys, so P V can start on the first half while the second is made).
-#ifndef BCA_P_HALVES
-#define BCA_P_HALVES 1
-#endif
-constexpr int kPHalves = BCA_P_HALVES;
-// Exponentials of the softmax: 0 = MUFU ex2 (fp32) for most pairs plus the FMA-pipe
-// polynomial for kPolyPairs of every 8; 1 = MUFU ex2 in f16x2 (two per instruction)
-// for every pair.
-#ifndef BCA_EXP_F16
-#define BCA_EXP_F16 0
-#endif
-constexpr bool kExpF16 = BCA_EXP_F16 != 0;
-static_assert(kPHalves == 1 || kPHalves == 2, "kPHalves must be 1 or 2");
 constexpr int kNoLimit = 1 << 30;
 // Split-chunk workspace: per chunk, O [256 rows][128] fp32, then m[256], l[256].
 constexpr int kChunkRows = 2 * kBM;
@@ -132,12 +110,14 @@ struct AttnParams {
   int32_t heads;
   int32_t mode;
   float scale_log2;  // softmax scale * log2(e)
-  // work items: [0, full_items) are whole units; the next units are split into
-  // split_k chunks each (chunk c of a unit with n tiles covers tiles
-  // [c*n/k, (c+1)*n/k)), written to `workspace` and merged by attn_combine_kernel.
+  // work items: [0, full_items) are whole units; the next split_units units are
+  // split into split_k chunks each (chunk c of a unit with n tiles covers tiles
+  // [c*n/k, (c+1)*n/k)), written to `workspace` and merged by attn_combine_kernel;
+  // the units after them (prefill: the light ones) are whole again.
   int32_t n_items;
   int32_t full_items;
   int32_t split_k;
+  int32_t split_units;
   float* workspace;
   // prefill
   int32_t seq_len;
@@ -170,16 +150,16 @@ struct Smem {
   static constexpr int bKvFull = 2;                    // kStages
   static constexpr int bKvEmpty = 2 + kStages;         // kStages
   static constexpr int bSFull = 2 + 2 * kStages;       // 2
-  static constexpr int bPFull = 4 + 2 * kStages;       // 4: [w][half] (128 arrivals each)
-  static constexpr int bOFull = 8 + 2 * kStages;       // 2
-  static constexpr int bDone = 10 + 2 * kStages;       // 1
-  static constexpr int bStgFull = 11 + 2 * kStages;    // 2
-  static constexpr int bStgEmpty = 13 + 2 * kStages;   // 2
-  static constexpr int bConv = 15 + 2 * kStages;       // 1 (64 converter arrivals per tile)
-  static constexpr int bQEmpty = 16 + 2 * kStages;     // 2 (Q tile w of an item consumed)
-  static constexpr int bEpiFull = 18 + 2 * kStages;    // 2 (O box of tile w in smem: 128)
-  static constexpr int bEpiFree = 20 + 2 * kStages;    // 2 (its TMA store has read it)
-  static constexpr int kNumBars = 22 + 2 * kStages;
+  static constexpr int bPFull = 4 + 2 * kStages;       // 2 (128 arrivals each)
+  static constexpr int bOFull = 6 + 2 * kStages;       // 2
+  static constexpr int bDone = 8 + 2 * kStages;        // 1
+  static constexpr int bStgFull = 9 + 2 * kStages;     // 2
+  static constexpr int bStgEmpty = 11 + 2 * kStages;   // 2
+  static constexpr int bConv = 13 + 2 * kStages;       // 1 (64 converter arrivals per tile)
+  static constexpr int bQEmpty = 14 + 2 * kStages;     // 2 (Q tile w of an item consumed)
+  static constexpr int bEpiFull = 16 + 2 * kStages;    // 2 (O box of tile w in smem: 128)
+  static constexpr int bEpiFree = 18 + 2 * kStages;    // 2 (its TMA store has read it)
+  static constexpr int kNumBars = 20 + 2 * kStages;
   static constexpr int kTmemSlot = kBars + 8 * kNumBars;
   static constexpr int kAbort = kTmemSlot + 4;
   static constexpr int kBytes = kAbort + 4;
@@ -218,19 +198,25 @@ __device__ __forceinline__ Item decode_item(const AttnParams<MAXR>& p, int item)
   int unit = item, chunk = 0, k = 1;
   it.partial = -1;
   if (item >= p.full_items) {
-    k = p.split_k;
     const int q = item - p.full_items;
-    unit = p.full_items + q / k;
-    chunk = q % k;
-    it.partial = q;
+    if (q < p.split_units * p.split_k) {
+      k = p.split_k;
+      unit = p.full_items + q / k;
+      chunk = q % k;
+      it.partial = q;
+    } else {
+      unit = p.full_items + p.split_units + (q - p.split_units * p.split_k);
+    }
   }
   int ntiles[2];
   if (p.mode == kModePrefill) {
     const int S = p.seq_len;
     const int nqp = (S + 2 * kBM - 1) / (2 * kBM);
     it.req = 0;
-    it.h = unit / nqp;
-    const int qp = nqp - 1 - unit % nqp;  // heaviest (latest) rows first within a head
+    // Heaviest (latest) Q-tile pairs of every head first: a pair's key limit, and
+    // so its work, never decreases with its rows.
+    it.h = unit % p.heads;
+    const int qp = nqp - 1 - unit / p.heads;
     it.q_row0 = qp * 2 * kBM;
     it.n_cache = 0;
     it.n_cache_tiles = 0;
@@ -552,9 +538,8 @@ template <int MAXR, bool kQ8>
 __device__ void mma_role(const AttnParams<MAXR>& p, uint32_t sbase, uint32_t bars, uint32_t tmem,
                          volatile int* abort) {
   // The items of this CTA are one stream of KV tiles.  Iteration t issues, per Q tile
-  // w, O_w += P_w(t-1) V(t-1) (in two K=64 halves, as the softmax hands P over in
-  // halves) and then S_w(t) = Q_w K(t)^T -- also across item boundaries, so the last
-  // tile of an item overlaps the first tile of the next.
+  // w, O_w += P_w(t-1) V(t-1) and then S_w(t) = Q_w K(t)^T -- also across item
+  // boundaries, so the last tile of an item overlaps the first tile of the next.
   auto bar = [&](int i) { return bars + 8u * static_cast<uint32_t>(i); };
   constexpr uint32_t kIdescS = idesc_bf16_f32(kBM, kBN, false);      // Q K^T: K-major B
   constexpr uint32_t kIdescO = idesc_bf16_f32(kBM, kHeadDim, true);  // P V: MN-major B
@@ -581,20 +566,16 @@ __device__ void mma_role(const AttnParams<MAXR>& p, uint32_t sbase, uint32_t bar
   int t = 0;  // tiles of this CTA so far (ring items 2t, 2t+1)
   auto issue_pv = [&](int w, int stV, bool first_of_item, bool last_of_item) {
     const uint64_t dv = sdesc_sw128(sbase + Smem::kRing + stV * kTileBytes, kHalfBytes, 1024);
-    constexpr int kPer = (kBN / 16) / kPHalves;  // MMAs (K = 16 keys) per part of P
+    if (!wait(Smem::bPFull + w, static_cast<uint32_t>(npv[w]) & 1u)) return;
+    tc_fence_after();
+    if (elect_one()) {
 #pragma unroll
-    for (int half = 0; half < kPHalves; ++half) {
-      if (!wait(Smem::bPFull + 2 * w + half, static_cast<uint32_t>(npv[w]) & 1u)) return;
-      tc_fence_after();
-      if (elect_one()) {
-#pragma unroll
-        for (int s = kPer * half; s < kPer * half + kPer; ++s)
-          mma_bf16_ts(tmem + col_o(w), tmem + col_s(w) + s * 8, dv + ((s * 2048) >> 4), kIdescO,
-                      (!first_of_item || s > 0) ? 1u : 0u);
-        if (half == kPHalves - 1 && last_of_item) mma_commit(bar(Smem::bOFull + w));
-      }
-      __syncwarp();
+      for (int s = 0; s < kBN / 16; ++s)  // K = 16 keys per MMA
+        mma_bf16_ts(tmem + col_o(w), tmem + col_s(w) + s * 8, dv + ((s * 2048) >> 4), kIdescO,
+                    (!first_of_item || s > 0) ? 1u : 0u);
+      if (last_of_item) mma_commit(bar(Smem::bOFull + w));
     }
+    __syncwarp();
     ++npv[w];
   };
   for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x, ++nq) {
@@ -701,10 +682,16 @@ __device__ void mma_role(const AttnParams<MAXR>& p, uint32_t sbase, uint32_t bar
       __syncwarp();
     }
   }
-  // Everything issued must be complete before TMEM is released.
+  // Everything issued must be complete before TMEM is released.  If that wait runs
+  // out, the timeout is reported and the CTA waits once more (bounded) before the
+  // kernel frees TMEM.
   if (elect_one()) mma_commit(bar(Smem::bDone));
   __syncwarp();
-  mbar_wait_bounded(bar(Smem::bDone), 0, nullptr, p.timeout_ns);
+  const bool done = mbar_wait_bounded(bar(Smem::bDone), 0, nullptr, p.timeout_ns);
+  if (!__all_sync(0xffffffffu, done)) {
+    if (elect_one()) raise_abort(abort, p.dev_status, 30 + Smem::bDone);
+    mbar_wait_bounded(bar(Smem::bDone), 0, nullptr, p.timeout_ns);
+  }
 }
 
 // ---------------------------------------------------------------------------
@@ -800,7 +787,9 @@ __device__ void softmax_role(const AttnParams<MAXR>& p, int w, uint32_t sbase, u
         l_run *= f;
         m_run = m_new;
       }
-      const float neg_m = (cache_tile ? lg_vs : 0.f) - m_run;
+      // A row with no allowed key so far (only in a split chunk of a prefill unit
+      // whose rows straddle a block end) keeps m = -inf: its p are exactly 0.
+      const float neg_m = (cache_tile ? lg_vs : 0.f) - (m_run == -INFINITY ? 0.f : m_run);
       // O was last written by P(j-1) V(j-1), complete before S(j) was signalled; it
       // is rescaled before the first half of P(j) is handed over (P(j) V(j) waits).
       if (j > c.j0 && __any_sync(0xffffffffu, need)) {
@@ -821,10 +810,9 @@ __device__ void softmax_role(const AttnParams<MAXR>& p, int w, uint32_t sbase, u
           tmem_st_32x32b_x16(tO + 16 * cc, o);
         }
       }
-      // p = 2^(s * sl2 - m) on column pairs: packed fp32x2 FMA for the exponent,
-      // then MUFU ex2 for most pairs and the FMA-pipe polynomial for kPolyPairs of
-      // every 8 (balances the two pipes); P is packed to bf16 in place over S and
-      // handed to the MMA in two halves of 64 keys.
+      // p = 2^(s * sl2 - m) on column pairs: packed fp32x2 FMA for the exponent, MUFU
+      // ex2 for the power; P is packed to bf16 in place over S (64 columns) and
+      // handed to the MMA as a whole tile.
       const uint64_t sl2x2 = f2_pack(sl2, sl2), negm2 = f2_pack(neg_m, neg_m);
       uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
@@ -834,28 +822,19 @@ __device__ void softmax_role(const AttnParams<MAXR>& p, int w, uint32_t sbase, u
           const uint64_t x =
               f2_fma(f2_pack(__uint_as_float(r[2 * cc]), __uint_as_float(r[2 * cc + 1])), sl2x2,
                      negm2);
-          uint64_t pp;
-          if (kExpF16) {
-            pp = exp2_f16x2(x);
-          } else if ((cc & 7) >= 8 - kPolyPairs) {
-            pp = exp2_poly2(x);
-          } else {
-            float x0, x1;
-            f2_unpack(x, x0, x1);
-            pp = f2_pack(ex2_approx(x0), ex2_approx(x1));
-          }
+          float x0, x1;
+          f2_unpack(x, x0, x1);
+          const uint64_t pp = f2_pack(ex2_approx(x0), ex2_approx(x1));
           acc[cc & 3] = f2_add(acc[cc & 3], pp);
           float p0, p1;
           f2_unpack(pp, p0, p1);
           r[cc] = pack_bf16x2(p0, p1);
         }
         tmem_st_32x32b_x32(tS + 32 * half, *reinterpret_cast<uint32_t(*)[32]>(&r[32 * half]));
-        if (kPHalves == 2 || half == 1) {
-          tmem_wait_st();
-          tc_fence_before();
-          mbar_arrive(bar(Smem::bPFull + 2 * w + (kPHalves == 2 ? half : 0)));
-        }
       }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(bar(Smem::bPFull + w));
       float a0, a1, b0, b1;
       f2_unpack(f2_add(acc[0], acc[1]), a0, a1);
       f2_unpack(f2_add(acc[2], acc[3]), b0, b1);
@@ -994,8 +973,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       mbar_init(bar(Smem::bQFull + i), 1);
       mbar_init(bar(Smem::bQEmpty + i), 1);
       mbar_init(bar(Smem::bSFull + i), 1);
-      mbar_init(bar(Smem::bPFull + 2 * i), 128);
-      mbar_init(bar(Smem::bPFull + 2 * i + 1), 128);
+      mbar_init(bar(Smem::bPFull + i), 128);
       mbar_init(bar(Smem::bOFull + i), 1);
       mbar_init(bar(Smem::bEpiFull + i), 128);
       mbar_init(bar(Smem::bEpiFree + i), 1);
@@ -1082,7 +1060,9 @@ __global__ void __launch_bounds__(256)
   float4 a[kMaxSplit];
 #pragma unroll
   for (int ci = 0; ci < kMaxSplit; ++ci) {
-    if (ci < k) {
+    // A chunk whose key range lies wholly past Q tile w's key limit (prefill units
+    // straddling a block end) wrote nothing for these rows.
+    if (ci < k && (ci == 0 || tile_active(decode_item(p, p.full_items + su * k + ci), w))) {
       const float* chunk = ws0 + ci * kStride;
       m[ci] = chunk[kChunkRows * kHeadDim + r2];
       l[ci] = chunk[kChunkRows * kHeadDim + kChunkRows + r2];

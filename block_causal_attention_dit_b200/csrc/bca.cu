@@ -9,9 +9,9 @@
 // entering attention), bca_step_graph_* (all layers' cached steps as one graph) and
 // bca_ulysses_pack/unpack (layouts around the all-to-all of head-sharded
 // sequence parallelism).
-// Every step of the path runs in the kernels of attn_kernel.cuh, kv_store_kernel.cuh,
-// q8_kernel.cuh, qk_norm_rope_kernel.cuh and ulysses_kernel.cuh; this file only
-// checks arguments and enqueues them.
+// Every step of the path runs in the kernels of attn_kernel.cuh, kv_store_kernel.cuh
+// (also the Q quantisation of the e4m3-Q step), qk_norm_rope_kernel.cuh and
+// ulysses_kernel.cuh; this file only checks arguments and enqueues them.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -28,7 +28,6 @@
 #include "../../include/bca.h"
 #include "attn_kernel.cuh"
 #include "kv_store_kernel.cuh"
-#include "q8_kernel.cuh"
 #include "qk_norm_rope_kernel.cuh"
 #include "ulysses_kernel.cuh"
 
@@ -132,8 +131,7 @@ struct MaxRequests<AttnParams<MAXR>> {
   static constexpr int value = MAXR;
 };
 
-// e4m3-Q scratch: codes [H, rows, 128], then scales [n_req][H] fp32, then the
-// absmax pass's [n_req][H] words.
+// e4m3-Q scratch: codes [H, rows, 128], then scales [n_req][H] fp32.
 size_t q8_codes_bytes(int64_t rows, int heads) {
   return round256(static_cast<size_t>(rows) * static_cast<size_t>(heads) * 128);
 }
@@ -199,6 +197,7 @@ int plan_items(AttnParams<MAXR>& p, int units, int grid, size_t ws_chunks, Tiles
   p.full_items = units;
   p.n_items = units;
   p.split_k = 1;
+  p.split_units = 0;
   if (ws_chunks == 0 || units <= grid) return 0;
   const int rounds = units / grid, rem = units - rounds * grid;
   if (rem == 0) return 0;
@@ -208,7 +207,38 @@ int plan_items(AttnParams<MAXR>& p, int units, int grid, size_t ws_chunks, Tiles
   if (k < 2) return 0;
   p.full_items = rounds * grid;
   p.split_k = k;
+  p.split_units = rem;
   p.n_items = rounds * grid + rem * k;
+  return rem;
+}
+
+// Prefill schedule.  Units are in decreasing order of work (KV tiles).  The heavy
+// units (at least half the heaviest) fill whole rounds; those of their last partial
+// round are split along the keys (as in plan_items); the lighter units follow, whole,
+// and fill the gaps the split chunks leave.  E.g. the T2I prefill (512 units of 36
+// tiles, 64 of 4, 148 SMs): 3 whole rounds, 68 units in 2 chunks, then the 64 light
+// units -- 130 tiles on the busiest SM instead of 144.
+template <int MAXR, typename TilesFn>
+int plan_items_weighted(AttnParams<MAXR>& p, int units, int grid, size_t ws_chunks,
+                        TilesFn unit_tiles) {
+  p.full_items = units;
+  p.n_items = units;
+  p.split_k = 1;
+  p.split_units = 0;
+  if (ws_chunks == 0 || units <= 1) return 0;
+  const int wmax = unit_tiles(0);
+  int heavy = 0;
+  while (heavy < units && 2 * unit_tiles(heavy) >= wmax) ++heavy;
+  const int rounds = heavy / grid, rem = heavy - rounds * grid;
+  if (rem == 0) return 0;
+  int k = std::min<int>(grid / rem, bca::kMaxSplit);
+  k = std::min<int>(k, static_cast<int>(ws_chunks / static_cast<size_t>(rem)));
+  for (int u = rounds * grid; u < heavy && k >= 2; ++u) k = std::min(k, unit_tiles(u));
+  if (k < 2) return 0;
+  p.full_items = rounds * grid;
+  p.split_k = k;
+  p.split_units = rem;
+  p.n_items = units - rem + rem * k;
   return rem;
 }
 
@@ -252,38 +282,75 @@ bca_status launch_attn(const AttnParams<MAXR>& p, int n_split_units, cudaStream_
   return BCA_OK;
 }
 
-// Enqueue the store passes for one slot (no host-side slot updates).
-bca_status enqueue_kv_store(const void* k, const void* v, int32_t n_prefix, int64_t row_stride,
-                            const bca_kv_slot* slot, int32_t* dev_status, cudaStream_t stream) {
-  (void)dev_status;  // the store kernels contain no waits
-  if (n_prefix == 0) return BCA_OK;
-  bca::KvStoreParams p{};
-  p.src[0] = static_cast<const uint16_t*>(k);
-  p.src[1] = static_cast<const uint16_t*>(v);
-  p.dst[0] = slot->k;
-  p.dst[1] = slot->v;
-  p.scale[0] = slot->k_scale;
-  p.scale[1] = slot->v_scale;
-  p.quant[0] = k_is_fp8(slot->dtype) ? 1 : 0;
-  p.quant[1] = v_is_fp8(slot->dtype) ? 1 : 0;
-  p.row_stride = row_stride;
-  p.n_prefix = n_prefix;
-  p.heads = slot->num_heads;
-  p.cap = slot->cap_tokens;
-  const bool any_quant = p.quant[0] || p.quant[1];
-  if (any_quant) {
-    bca::kv_amax_init_kernel<<<dim3(1, 2), 256, 0, stream>>>(p);
-    const int tpb = std::max(8, (n_prefix + 295) / 296);  // ~2 blocks per SM per tensor
-    const int nb = (n_prefix + tpb - 1) / tpb;
-    bca::kv_amax_kernel<<<dim3(nb, 2), bca::kStoreThreads, 0, stream>>>(p, tpb);
+// One tensor (K or V of a request, or a request's Q) for the store kernel.
+struct StoreJob {
+  const void* src;
+  void* dst;
+  float* scale;
+  int64_t row_stride;
+  int64_t head_stride;
+  int32_t rows;
+  int32_t heads;
+  bool quant;
+};
+
+// One launch of bca::kv_store_kernel over every job: tensors with the most rows
+// first, clusters of bca::kStoreCluster CTAs, as many clusters as fit one CTA per SM
+// (so that few columns are in flight and the encode pass re-reads them from L2).
+bca_status launch_store(std::vector<StoreJob> jobs, int32_t* dev_status, cudaStream_t stream) {
+  jobs.erase(std::remove_if(jobs.begin(), jobs.end(), [](const StoreJob& j) { return j.rows == 0; }),
+             jobs.end());
+  if (jobs.empty()) return BCA_OK;
+  if (jobs.size() > static_cast<size_t>(bca::kMaxStoreTensors)) return BCA_ERR_INVALID_ARG;
+  std::stable_sort(jobs.begin(), jobs.end(),
+                   [](const StoreJob& a, const StoreJob& b) { return a.rows > b.rows; });
+  bca::StoreParams p;
+  std::memset(&p, 0, sizeof(p));
+  int cols = 0;
+  for (size_t i = 0; i < jobs.size(); ++i) {
+    bca::StoreTensor& t = p.t[i];
+    t.src = static_cast<const uint16_t*>(jobs[i].src);
+    t.dst = jobs[i].dst;
+    t.scale = jobs[i].scale;
+    t.row_stride = jobs[i].row_stride;
+    t.head_stride = jobs[i].head_stride;
+    t.rows = jobs[i].rows;
+    t.heads = jobs[i].heads;
+    t.quant = jobs[i].quant ? 1 : 0;
+    t.col0 = cols;
+    cols += jobs[i].heads;
   }
-  const int64_t chunks = static_cast<int64_t>(n_prefix) * p.heads * 16;
-  const int64_t want = (chunks + bca::kStoreThreads - 1) / bca::kStoreThreads;
+  p.n_tensors = static_cast<int32_t>(jobs.size());
+  p.n_cols = cols;
+  p.dev_status = dev_status;
   const int sms = std::max(sm_count(), 1);
-  const int grid = static_cast<int>(std::min<int64_t>(want, static_cast<int64_t>(sms) * 8));
-  bca::kv_write_kernel<<<dim3(grid, 2), bca::kStoreThreads, 0, stream>>>(p);
-  if (any_quant) bca::kv_scale_finalize_kernel<<<dim3(1, 2), 256, 0, stream>>>(p);
+  const int clusters = std::max(1, std::min(cols, sms / bca::kStoreCluster));
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(clusters * bca::kStoreCluster));
+  cfg.blockDim = dim3(bca::kStoreThreads);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = bca::kStoreCluster;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, bca::kv_store_kernel, p) != cudaSuccess) return BCA_ERR_CUDA;
   return cudaGetLastError() == cudaSuccess ? BCA_OK : BCA_ERR_CUDA;
+}
+
+// The K and V jobs of one slot's store (no host-side slot updates).
+void store_jobs(const void* k, const void* v, int32_t n_prefix, int64_t row_stride,
+                const bca_kv_slot* slot, std::vector<StoreJob>& jobs) {
+  const void* src[2] = {k, v};
+  void* dst[2] = {slot->k, slot->v};
+  float* sc[2] = {slot->k_scale, slot->v_scale};
+  const bool q[2] = {k_is_fp8(slot->dtype), v_is_fp8(slot->dtype)};
+  for (int t = 0; t < 2; ++t)
+    jobs.push_back(StoreJob{src[t], dst[t], sc[t], row_stride, slot->cap_tokens, n_prefix,
+                            slot->num_heads, q[t]});
 }
 
 bca_status validate_store(const void* k, const void* v, int32_t n_prefix, int64_t row_stride,
@@ -316,6 +383,7 @@ const char* bca_status_string(bca_status s) {
     case BCA_ERR_STATE: return "BCA_ERR_STATE";
     case BCA_ERR_CUDA: return "BCA_ERR_CUDA";
     case BCA_ERR_DEVICE_TIMEOUT: return "BCA_ERR_DEVICE_TIMEOUT";
+    case BCA_ERR_NONFINITE: return "BCA_ERR_NONFINITE";
   }
   return "BCA_UNKNOWN_STATUS";
 }
@@ -366,11 +434,35 @@ bca_status bca_kv_store(const void* k, const void* v, int32_t n_prefix, int32_t 
                         bca_kv_slot* slot, uint32_t epoch, int32_t* dev_status, void* stream) {
   bca_status st = validate_store(k, v, n_prefix, row_stride_elems, slot, epoch);
   if (st != BCA_OK) return st;
-  st = enqueue_kv_store(k, v, n_prefix, row_stride_elems, slot, dev_status,
-                        static_cast<cudaStream_t>(stream));
+  std::vector<StoreJob> jobs;
+  store_jobs(k, v, n_prefix, row_stride_elems, slot, jobs);
+  st = launch_store(std::move(jobs), dev_status, static_cast<cudaStream_t>(stream));
   if (st != BCA_OK) return st;
   slot->n_tokens = n_prefix;
   slot->epoch = epoch;
+  return BCA_OK;
+}
+
+bca_status bca_kv_store_batch(const bca_kv_store_item* items, int32_t n_items, uint32_t epoch,
+                              int32_t* dev_status, void* stream) {
+  if (!items || n_items < 1 || n_items > BCA_MAX_BATCH) return BCA_ERR_INVALID_ARG;
+  for (int i = 0; i < n_items; ++i) {
+    bca_status st = validate_store(items[i].k, items[i].v, items[i].n_prefix,
+                                   items[i].row_stride_elems, items[i].slot, epoch);
+    if (st != BCA_OK) return st;
+    for (int j = 0; j < i; ++j)
+      if (items[j].slot == items[i].slot) return BCA_ERR_INVALID_ARG;
+  }
+  std::vector<StoreJob> jobs;
+  for (int i = 0; i < n_items; ++i)
+    store_jobs(items[i].k, items[i].v, items[i].n_prefix, items[i].row_stride_elems,
+               items[i].slot, jobs);
+  bca_status st = launch_store(std::move(jobs), dev_status, static_cast<cudaStream_t>(stream));
+  if (st != BCA_OK) return st;
+  for (int i = 0; i < n_items; ++i) {
+    items[i].slot->n_tokens = items[i].n_prefix;
+    items[i].slot->epoch = epoch;
+  }
   return BCA_OK;
 }
 
@@ -378,6 +470,16 @@ bca_status bca_prefill(const void* q, const void* k, const void* v, void* o, int
                        const int32_t* off, int32_t n_blocks, int32_t heads, int32_t head_dim,
                        float scale, bca_kv_slot* slot, uint32_t epoch, int32_t* dev_status,
                        void* stream) {
+  return bca_prefill_ws(q, k, v, o, seq_len, off, n_blocks, heads, head_dim, scale, slot, epoch,
+                        nullptr, 0, dev_status, stream);
+}
+
+bca_status bca_prefill_ws(const void* q, const void* k, const void* v, void* o, int32_t seq_len,
+                          const int32_t* off, int32_t n_blocks, int32_t heads, int32_t head_dim,
+                          float scale, bca_kv_slot* slot, uint32_t epoch, void* workspace,
+                          size_t workspace_bytes, int32_t* dev_status, void* stream) {
+  if (workspace && (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return BCA_ERR_INVALID_ARG;
+  const size_t ws_chunks = workspace ? workspace_bytes / bca::kChunkBytes : 0;
   if (!q || !k || !v || !o || !off) return BCA_ERR_INVALID_ARG;
   if (head_dim != 128) return BCA_ERR_UNSUPPORTED;
   if (heads < 1 || heads > 256 || seq_len < 1) return BCA_ERR_INVALID_ARG;
@@ -416,11 +518,27 @@ bca_status bca_prefill(const void* q, const void* k, const void* v, void* o, int
   for (int b = 0; b <= n_blocks; ++b) p.block_off[b] = off[b];
   const int nqp = (seq_len + 2 * bca::kBM - 1) / (2 * bca::kBM);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  plan_items(p, nqp * heads, 1, 0, [](int) { return 1; });  // prefill: whole units only
-  bca_status st = launch_attn(p, 0, s);
+  const int sms = sm_count();
+  if (sms <= 0) return BCA_ERR_CUDA;
+  p.workspace = static_cast<float*>(workspace);
+  // Unit u: Q-tile pair nqp - 1 - u / heads (its last row's block end sets its tiles).
+  const int n_split = plan_items_weighted(p, nqp * heads, sms, ws_chunks, [&](int u) {
+    const int qp = nqp - 1 - u / heads;
+    const int last = std::min(seq_len, (qp + 1) * 2 * bca::kBM) - 1;
+    int lim = seq_len;
+    for (int b = 1; b <= n_blocks; ++b)
+      if (last < off[b]) {
+        lim = off[b];
+        break;
+      }
+    return (lim + bca::kBN - 1) / bca::kBN;
+  });
+  bca_status st = launch_attn(p, n_split, s);
   if (st != BCA_OK) return st;
   if (slot) {
-    st = enqueue_kv_store(k, v, n_prefix, static_cast<int64_t>(heads) * 128, slot, dev_status, s);
+    std::vector<StoreJob> jobs;
+    store_jobs(k, v, n_prefix, static_cast<int64_t>(heads) * 128, slot, jobs);
+    st = launch_store(std::move(jobs), dev_status, s);
     if (st != BCA_OK) return st;
     slot->n_tokens = n_prefix;
     slot->epoch = epoch;
@@ -435,7 +553,7 @@ size_t bca_step_workspace_bytes(void) {
 
 size_t bca_step_q8_scratch_bytes(int64_t rows, int32_t n_req, int32_t heads) {
   if (rows < 0 || n_req < 1 || n_req > BCA_MAX_BATCH || heads < 1 || heads > 256) return 0;
-  return q8_codes_bytes(rows, heads) + 2 * q8_table_bytes(n_req, heads);
+  return q8_codes_bytes(rows, heads) + q8_table_bytes(n_req, heads);
 }
 
 // The cached step; with q8_scratch, in e4m3-Q mode (bca_step_attend_q8).
@@ -479,33 +597,17 @@ static bca_status step_attend_impl(const void* q_t, const void* k_t, const void*
   uint8_t* q8_codes = static_cast<uint8_t*>(q8_scratch);
   float* q8_scale = q8 ? reinterpret_cast<float*>(q8_codes + q8_codes_bytes(total, heads)) : nullptr;
   if (q8) {
-    // Q codes and scales of every request, before the attention reads them.
-    bca::Q8Params qp{};
-    qp.q = static_cast<const uint16_t*>(q_t);
-    qp.codes = q8_codes;
-    qp.scale = q8_scale;
-    qp.amax = reinterpret_cast<unsigned*>(reinterpret_cast<uint8_t*>(q8_scale) +
-                                          q8_table_bytes(n_req, heads));
-    qp.rows = total;
-    qp.heads = heads;
-    qp.n_req = n_req;
-    int max_len = 0;
-    for (int r = 0; r < n_req; ++r) {
-      qp.q_start[r] = cu[r];
-      qp.q_len[r] = cu[r + 1] - cu[r];
-      max_len = std::max(max_len, qp.q_len[r]);
-    }
-    const int sms = std::max(sm_count(), 1);
-    cudaStream_t s = static_cast<cudaStream_t>(stream);
-    bca::q8_amax_init_kernel<<<1, 256, 0, s>>>(qp);
-    const int ax = (max_len + bca::kQ8RowsPerBlock - 1) / bca::kQ8RowsPerBlock;
-    bca::q8_amax_kernel<<<dim3(ax, n_req), bca::kQ8Threads, 0, s>>>(qp);
-    const int64_t want = (static_cast<int64_t>(max_len) * heads * 16 + bca::kQ8Threads - 1) /
-                         bca::kQ8Threads;
-    const int ex = static_cast<int>(
-        std::max<int64_t>(1, std::min<int64_t>(want, std::max(1, 4 * sms / n_req))));
-    bca::q8_encode_kernel<<<dim3(ex, n_req), bca::kQ8Threads, 0, s>>>(qp);
-    if (cudaGetLastError() != cudaSuccess) return BCA_ERR_CUDA;
+    // Q codes and scales of every request, before the attention reads them: each
+    // request's Q is stored like an e4m3 cache tensor into [H, total, 128].
+    std::vector<StoreJob> jobs;
+    const int64_t row_elems = static_cast<int64_t>(heads) * 128;
+    for (int r = 0; r < n_req; ++r)
+      jobs.push_back(StoreJob{static_cast<const uint16_t*>(q_t) + cu[r] * row_elems,
+                              q8_codes + static_cast<int64_t>(cu[r]) * 128,
+                              q8_scale + static_cast<size_t>(r) * heads, row_elems, total,
+                              cu[r + 1] - cu[r], heads, true});
+    bca_status st = launch_store(std::move(jobs), dev_status, static_cast<cudaStream_t>(stream));
+    if (st != BCA_OK) return st;
   }
 
   // Longest key sequence first (largest per-unit work scheduled first).

@@ -9,72 +9,19 @@
 //                 s_h    = fp32(amax_h) / 448 (correctly rounded; 1 if amax_h = 0)
 //                 cache[h, t, c] = e4m3_rn_satfinite(x[t, h, c] / s_h)   (fp32 quotient,
 //                                  correctly rounded), scale[h] = s_h
-// HBM-bound: 16-byte vector loads, coalesced along [t, h, c]; the absmax pass is a
-// separate read so that the encode pass sees the final scale.  The running absmax
-// is kept as bf16 magnitude bits (|x| bit patterns of finite bf16 values order like
-// the values) in the slot's own scale array, which the last pass overwrites with
-// s_h -- no scratch memory.
+// HBM-bound; one kernel (kv_store_kernel below) per store call, whatever the
+// number of requests, with no scratch memory.
 #pragma once
 #include <cuda_bf16.h>
 
 #include <cstdint>
 
+#include "../../include/bca.h"
+
 namespace bca {
-
-struct KvStoreParams {
-  const uint16_t* src[2];  // K, V (bf16 bits), token t head h at t*row_stride + h*128
-  void* dst[2];            // [H, cap, 128] bf16 or e4m3
-  float* scale[2];         // [H] (e4m3 tensors only)
-  int32_t quant[2];        // 1: e4m3, 0: bf16 copy
-  int64_t row_stride;      // elements
-  int32_t n_prefix;
-  int32_t heads;
-  int32_t cap;
-};
-
-constexpr int kStoreThreads = 256;
-
-// Zero the running absmax of every e4m3 tensor.
-__global__ void kv_amax_init_kernel(KvStoreParams p) {
-  const int t = blockIdx.y;
-  if (!(t ? p.quant[1] : p.quant[0])) return;
-  unsigned* a = reinterpret_cast<unsigned*>(t ? p.scale[1] : p.scale[0]);
-  for (int h = threadIdx.x; h < p.heads; h += blockDim.x) a[h] = 0u;
-}
 
 __device__ __forceinline__ uint32_t max_abs_bf16x2(uint32_t m, uint32_t w) {
   return max(m, max(w & 0x7FFFu, (w >> 16) & 0x7FFFu));
-}
-
-// Pass 1: per-head absmax.  blockIdx.y = tensor; a block covers a token range and
-// every (head, 16-byte chunk) pair; 16 lanes share a head.
-__global__ void __launch_bounds__(kStoreThreads) kv_amax_kernel(KvStoreParams p, int tokens_per_block) {
-  const int tsel = blockIdx.y;
-  if (!(tsel ? p.quant[1] : p.quant[0])) return;
-  const uint16_t* src = tsel ? p.src[1] : p.src[0];
-  unsigned* amax = reinterpret_cast<unsigned*>(tsel ? p.scale[1] : p.scale[0]);
-  const int t0 = blockIdx.x * tokens_per_block;
-  const int t1 = min(p.n_prefix, t0 + tokens_per_block);
-  const int pairs = p.heads * 16;
-  for (int base = 0; base < pairs; base += blockDim.x) {
-    const int pr = base + threadIdx.x;
-    const int h = pr >> 4, c = pr & 15;
-    uint32_t m = 0;
-    if (pr < pairs) {
-      const uint16_t* s = src + static_cast<int64_t>(h) * 128 + c * 8;
-      for (int t = t0; t < t1; ++t) {
-        const uint4 v = __ldg(reinterpret_cast<const uint4*>(s + static_cast<int64_t>(t) * p.row_stride));
-        m = max_abs_bf16x2(m, v.x);
-        m = max_abs_bf16x2(m, v.y);
-        m = max_abs_bf16x2(m, v.z);
-        m = max_abs_bf16x2(m, v.w);
-      }
-    }
-#pragma unroll
-    for (int o = 8; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
-    if (pr < pairs && c == 0 && t1 > t0)
-      atomicMax(amax + h, m);
-  }
 }
 
 __device__ __forceinline__ float scale_from_amax_bits(unsigned bits) {
@@ -108,61 +55,196 @@ __device__ __forceinline__ uint16_t e4m3x2_rn_satfinite(float lo, float hi) {
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
-// Pass 2: copy (bf16) or encode (e4m3).  One thread per 16-byte source chunk
-// (8 elements); grid-stride over [t, h, chunk].
-__global__ void __launch_bounds__(kStoreThreads) kv_write_kernel(KvStoreParams p) {
-  const int tsel = blockIdx.y;
-  const uint16_t* src = tsel ? p.src[1] : p.src[0];
-  void* dst = tsel ? p.dst[1] : p.dst[0];
-  const int64_t total = static_cast<int64_t>(p.n_prefix) * p.heads * 16;
-  const bool quant = (tsel ? p.quant[1] : p.quant[0]) != 0;
-  const unsigned* amax_bits = reinterpret_cast<const unsigned*>(tsel ? p.scale[1] : p.scale[0]);
-  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total;
-       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int c = static_cast<int>(i & 15);
-    int h;
-    int64_t t;
-    if (total < (int64_t{1} << 31)) {  // 32-bit index arithmetic when it fits
-      const uint32_t th = static_cast<uint32_t>(i) >> 4;
-      t = th / static_cast<uint32_t>(p.heads);
-      h = static_cast<int>(th - static_cast<uint32_t>(t) * static_cast<uint32_t>(p.heads));
-    } else {
-      const int64_t th = i >> 4;
-      h = static_cast<int>(th % p.heads);
-      t = th / p.heads;
-    }
-    const uint4 v = __ldg(reinterpret_cast<const uint4*>(src + t * p.row_stride + h * 128 + c * 8));
-    const int64_t drow = static_cast<int64_t>(h) * p.cap + t;
-    if (!quant) {
-      reinterpret_cast<uint4*>(static_cast<uint16_t*>(dst) + drow * 128)[c] = v;
-    } else {
-      const unsigned ab = amax_bits[h];
-      const float s = scale_from_amax_bits(ab);
-      const float y = __frcp_rn(s);
-      const bool fast = ab >= kFastDivMinBits;
-      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-      uint32_t out[2];
-#pragma unroll
-      for (int k = 0; k < 2; ++k) {
-        const uint16_t a = e4m3x2_rn_satfinite(div_by_scale(bf16_lo(w[2 * k]), s, y, fast),
-                                               div_by_scale(bf16_hi(w[2 * k]), s, y, fast));
-        const uint16_t b = e4m3x2_rn_satfinite(div_by_scale(bf16_lo(w[2 * k + 1]), s, y, fast),
-                                               div_by_scale(bf16_hi(w[2 * k + 1]), s, y, fast));
-        out[k] = static_cast<uint32_t>(a) | (static_cast<uint32_t>(b) << 16);
-      }
-      reinterpret_cast<uint2*>(static_cast<uint8_t*>(dst) + drow * 128)[c] =
-          make_uint2(out[0], out[1]);
-    }
-  }
+// ---------------------------------------------------------------------------
+// The store kernel.  A launch stores a list of tensors; tensor i has heads_i
+// columns (one per head: rows [0, rows_i) of that head), numbered from col0_i.  A
+// cluster of kStoreCluster CTAs takes whole columns (cluster c: columns c, c +
+// #clusters, ...; the host lists tensors with the most rows first), and its CTAs
+// split the column's rows evenly.
+//  * bf16 column: a copy.
+//  * e4m3 column: pass 1 reads the CTA's rows for the absmax; the CTAs' partial
+//    maxima meet in every CTA's shared memory (distributed shared memory stores,
+//    then a cluster barrier), so each CTA knows amax_h; rank 0 writes s_h.  Pass 2
+//    reads the same rows again, last-read first, so that they still come from L2
+//    (a cluster's column is at most ~4.4 MB and only as many columns are in flight
+//    as there are clusters, ~18 on B200), and writes the codes with streaming
+//    stores.  HBM then sees each source byte read once and each code written once.
+// Every thread owns one 16-byte chunk (8 channels) of a row; 16 threads cover a
+// 256-byte head row, kStoreUnroll rows per thread are loaded before any is used.
+// A non-finite value in an e4m3 column makes its amax Inf or NaN: the column's
+// codes and scale are then meaningless and BCA_ERR_NONFINITE is written to
+// *dev_status (the inputs must be finite).
+// ---------------------------------------------------------------------------
+struct StoreTensor {
+  const uint16_t* src;  // bf16 bits; row t, head h at src + t * row_stride + h * 128
+  void* dst;            // row t, head h at element (h * head_stride + t) * 128 (bf16 or e4m3)
+  float* scale;         // [heads] fp32, e4m3 tensors only
+  int64_t row_stride;   // source elements between consecutive rows
+  int64_t head_stride;  // destination rows between consecutive heads
+  int32_t rows;
+  int32_t heads;
+  int32_t quant;        // 1: e4m3 with a per-head absmax scale, 0: bf16 copy
+  int32_t col0;         // first column of this tensor
+};
+
+constexpr int kMaxStoreTensors = 2 * BCA_MAX_BATCH;
+constexpr int kStoreThreads = 512;
+constexpr int kStoreCluster = 8;
+constexpr int kStoreUnroll = 8;
+constexpr int kStoreRowsPerSweep = kStoreThreads / 16;
+
+struct StoreParams {
+  StoreTensor t[kMaxStoreTensors];
+  int32_t n_tensors;
+  int32_t n_cols;
+  int32_t* dev_status;
+};
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ uint32_t cluster_size() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_nctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ uint32_t cluster_index() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%clusterid.x;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ uint32_t cluster_count() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%nclusterid.x;" : "=r"(r));
+  return r;
+}
+// Every thread of every CTA of the cluster; orders shared-memory writes (local and
+// distributed) before the reads that follow it.
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\t"
+               "barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// 32-bit store into CTA `rank`'s copy of the shared variable at local address `a`.
+__device__ __forceinline__ void st_shared_cluster(uint32_t a, uint32_t rank, uint32_t v) {
+  uint32_t ra;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(ra) : "r"(a), "r"(rank));
+  asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(ra), "r"(v) : "memory");
 }
 
-// Pass 3: running absmax bits -> final fp32 scale.
-__global__ void kv_scale_finalize_kernel(KvStoreParams p) {
-  const int t = blockIdx.y;
-  if (!(t ? p.quant[1] : p.quant[0])) return;
-  float* sc = t ? p.scale[1] : p.scale[0];
-  for (int h = threadIdx.x; h < p.heads; h += blockDim.x)
-    sc[h] = scale_from_amax_bits(__float_as_uint(sc[h]));
+__device__ __forceinline__ uint2 encode_chunk(const uint4 v, float s, float y, bool fast) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  uint32_t out[2];
+#pragma unroll
+  for (int k = 0; k < 2; ++k) {
+    const uint16_t a = e4m3x2_rn_satfinite(div_by_scale(bf16_lo(w[2 * k]), s, y, fast),
+                                           div_by_scale(bf16_hi(w[2 * k]), s, y, fast));
+    const uint16_t b = e4m3x2_rn_satfinite(div_by_scale(bf16_lo(w[2 * k + 1]), s, y, fast),
+                                           div_by_scale(bf16_hi(w[2 * k + 1]), s, y, fast));
+    out[k] = static_cast<uint32_t>(a) | (static_cast<uint32_t>(b) << 16);
+  }
+  return make_uint2(out[0], out[1]);
+}
+
+__global__ void __launch_bounds__(kStoreThreads, 1)
+    kv_store_kernel(const __grid_constant__ StoreParams p) {
+  __shared__ unsigned s_part[2][kStoreCluster];  // partial maxima by rank, double-buffered
+  __shared__ unsigned s_warp[kStoreThreads / 32];
+  const uint32_t crank = cluster_rank(), csize = cluster_size();
+  const int tid = threadIdx.x, lane16 = tid & 15, rslot = tid >> 4;
+  constexpr int kStep = kStoreRowsPerSweep * kStoreUnroll;
+  int ti = 0, nq = 0;
+  for (int col = static_cast<int>(cluster_index()); col < p.n_cols;
+       col += static_cast<int>(cluster_count())) {
+    while (ti + 1 < p.n_tensors && col >= p.t[ti + 1].col0) ++ti;
+    const StoreTensor& T = p.t[ti];
+    const int h = col - T.col0;
+    const int r0 = static_cast<int>(static_cast<int64_t>(T.rows) * crank / csize);
+    const int r1 = static_cast<int>(static_cast<int64_t>(T.rows) * (crank + 1) / csize);
+    const uint16_t* src = T.src + static_cast<int64_t>(h) * 128 + lane16 * 8;
+    const int64_t rs = T.row_stride;
+    const int64_t drow0 = static_cast<int64_t>(h) * T.head_stride;
+    if (!T.quant) {
+      uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(T.dst) + drow0 * 128) + lane16;
+      for (int tb = r0 + rslot; tb < r1; tb += kStep) {
+        uint4 v[kStoreUnroll];
+#pragma unroll
+        for (int u = 0; u < kStoreUnroll; ++u) {
+          const int t = tb + u * kStoreRowsPerSweep;
+          if (t < r1) v[u] = __ldcs(reinterpret_cast<const uint4*>(src + t * rs));
+        }
+#pragma unroll
+        for (int u = 0; u < kStoreUnroll; ++u) {
+          const int t = tb + u * kStoreRowsPerSweep;
+          if (t < r1) __stcs(dst + static_cast<int64_t>(t) * 16, v[u]);
+        }
+      }
+      continue;
+    }
+    // Pass 1: absmax of this CTA's rows, as bf16 magnitude bits.
+    uint32_t m = 0;
+    for (int tb = r0 + rslot; tb < r1; tb += kStep) {
+      uint4 v[kStoreUnroll];
+#pragma unroll
+      for (int u = 0; u < kStoreUnroll; ++u) {
+        const int t = tb + u * kStoreRowsPerSweep;
+        v[u] = t < r1 ? __ldg(reinterpret_cast<const uint4*>(src + t * rs))
+                      : make_uint4(0u, 0u, 0u, 0u);
+      }
+#pragma unroll
+      for (int u = 0; u < kStoreUnroll; ++u) {
+        m = max_abs_bf16x2(m, v[u].x);
+        m = max_abs_bf16x2(m, v[u].y);
+        m = max_abs_bf16x2(m, v[u].z);
+        m = max_abs_bf16x2(m, v[u].w);
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
+    if ((tid & 31) == 0) s_warp[tid >> 5] = m;
+    __syncthreads();
+    if (tid < 32) {
+      uint32_t x = tid < kStoreThreads / 32 ? s_warp[tid] : 0u;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) x = max(x, __shfl_xor_sync(0xffffffffu, x, o));
+      if (tid == 0) {
+        const uint32_t a = static_cast<uint32_t>(__cvta_generic_to_shared(&s_part[nq & 1][crank]));
+        for (uint32_t q = 0; q < csize; ++q) st_shared_cluster(a, q, x);
+      }
+    }
+    cluster_sync();
+    uint32_t amax = 0;
+    for (uint32_t q = 0; q < csize; ++q) amax = max(amax, s_part[nq & 1][q]);
+    ++nq;
+    const float s = scale_from_amax_bits(amax);
+    if (crank == 0 && tid == 0) {
+      T.scale[h] = s;
+      if (amax >= 0x7F80u && p.dev_status)
+        atomicExch(p.dev_status, static_cast<int32_t>(BCA_ERR_NONFINITE));
+    }
+    const float y = __frcp_rn(s);
+    const bool fast = amax >= kFastDivMinBits;
+    // Pass 2: the same rows, last-read first; codes with streaming stores.
+    uint2* dst = reinterpret_cast<uint2*>(static_cast<uint8_t*>(T.dst) + drow0 * 128) + lane16;
+    const int n = r1 - r0;
+    const int last = r0 + (n > 0 ? ((n - 1 - rslot) / kStep) * kStep : 0) + rslot;
+    for (int tb = last; tb >= r0 && n > rslot; tb -= kStep) {
+      uint4 v[kStoreUnroll];
+#pragma unroll
+      for (int u = 0; u < kStoreUnroll; ++u) {
+        const int t = tb + u * kStoreRowsPerSweep;
+        if (t < r1) v[u] = __ldcs(reinterpret_cast<const uint4*>(src + t * rs));
+      }
+#pragma unroll
+      for (int u = 0; u < kStoreUnroll; ++u) {
+        const int t = tb + u * kStoreRowsPerSweep;
+        if (t < r1) __stcs(dst + static_cast<int64_t>(t) * 16, encode_chunk(v[u], s, y, fast));
+      }
+    }
+  }
+  // No CTA leaves while a peer may still store into its shared memory.
+  cluster_sync();
 }
 
 // Self-check of div_by_scale as the encoder uses it: for every positive finite bf16

@@ -290,24 +290,6 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   return r;
 }
 
-// 2^x for two lanes on the MUFU in half precision (two results per instruction):
-// x rounded to f16 (for x <= 8 the spacing is <= 2^-8), result to f32.
-__device__ __forceinline__ uint64_t exp2_f16x2(uint64_t x) {
-  float x0, x1;
-  asm("mov.b64 {%0, %1}, %2;" : "=f"(x0), "=f"(x1) : "l"(x));
-  uint32_t h, e;
-  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(h) : "f"(x1), "f"(x0));
-  asm("ex2.approx.f16x2 %0, %1;" : "=r"(e) : "r"(h));
-  float p0, p1;
-  asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %2;\n\t"
-      "cvt.f32.f16 %0, lo;\n\tcvt.f32.f16 %1, hi;\n\t}"
-      : "=f"(p0), "=f"(p1)
-      : "r"(e));
-  uint64_t r;
-  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(p0), "f"(p1));
-  return r;
-}
-
 // Two fp32 -> packed bf16x2 (round to nearest even); `lo` lands in bits [0,16).
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   uint32_t r;

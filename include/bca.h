@@ -33,7 +33,9 @@
  *    BCA_ERR_DEVICE_TIMEOUT into *dev_status (if dev_status is not NULL), drains
  *    and returns; the host reads *dev_status after synchronising.
  *  - Supported now: head_dim == 128, heads in [1, 256], device pointers 16-byte
- *    aligned, finite inputs.
+ *    aligned, finite inputs.  (An e4m3 quantiser that meets a non-finite value
+ *    writes BCA_ERR_NONFINITE into *dev_status; that head's codes and scale are
+ *    then meaningless.)
  *  - A softmax scale is passed in (1/sqrt(head_dim) for the DiT).
  */
 #ifndef BCA_H_
@@ -53,7 +55,8 @@ typedef enum {
   BCA_ERR_CAPACITY = 3,       /* prefix longer than the slot's cap_tokens          */
   BCA_ERR_STATE = 4,          /* slot not filled for the current request (epoch 0) */
   BCA_ERR_CUDA = 5,           /* a CUDA runtime/driver call or a launch failed     */
-  BCA_ERR_DEVICE_TIMEOUT = 6  /* a bounded device-side wait expired                */
+  BCA_ERR_DEVICE_TIMEOUT = 6, /* a bounded device-side wait expired                */
+  BCA_ERR_NONFINITE = 7       /* an e4m3 quantiser met Inf or NaN (via dev_status) */
 } bca_status;
 
 /* Cache element type, mirroring the recipe's prefix_kv_cache_dtype values. */
@@ -117,11 +120,31 @@ bca_status bca_kv_slot_init(bca_kv_slot* slot, void* base, int32_t cap_tokens,
  * For an e4m3 tensor: amax = max |x| over the n_prefix rows of each head,
  * scale = fp32(amax)/448 (1 when amax == 0), code = e4m3 RNE-satfinite of the
  * correctly rounded fp32 quotient x/scale.  Rows [n_prefix, cap) are not written.
+ * One kernel launch (HBM-bound; the absmax and encode passes of a head run back to
+ * back on the same CTAs, so the second reads its rows from L2).
  * Host side effects (at enqueue): slot->n_tokens = n_prefix, slot->epoch = epoch.
- * dev_status: nullable device int32, see the conventions above. */
+ * dev_status: nullable device int32, see the conventions above (a non-finite value
+ * in an e4m3 tensor: BCA_ERR_NONFINITE). */
 bca_status bca_kv_store(const void* k, const void* v, int32_t n_prefix,
                         int32_t row_stride_elems, bca_kv_slot* slot, uint32_t epoch,
                         int32_t* dev_status, void* stream);
+
+/* One request's part of bca_kv_store_batch: the arguments of bca_kv_store. */
+typedef struct bca_kv_store_item {
+  const void* k;
+  const void* v;
+  int32_t n_prefix;
+  int32_t row_stride_elems;
+  bca_kv_slot* slot;
+} bca_kv_store_item;
+
+/* bca_kv_store for n_items (1..BCA_MAX_BATCH) requests of a same-phase batch in one
+ * kernel launch ("Online serving" on the recipe page batches requests at the same
+ * phase; their prefix stores are one call here).  Every item is checked as
+ * bca_kv_store checks its arguments before anything is launched; the slots must be
+ * distinct (else BCA_ERR_INVALID_ARG).  Each slot is stamped with `epoch`. */
+bca_status bca_kv_store_batch(const bca_kv_store_item* items, int32_t n_items, uint32_t epoch,
+                              int32_t* dev_status, void* stream);
 
 /* Step 1 (prefill) of one request at one layer: block-causal attention over the
  * whole sequence ("What is Qwen-Image-2.1" and "Serving architecture: the
@@ -138,6 +161,20 @@ bca_status bca_prefill(const void* q, const void* k, const void* v, void* o, int
                        const int32_t* block_offsets, int32_t n_blocks, int32_t heads,
                        int32_t head_dim, float scale, bca_kv_slot* slot, uint32_t epoch,
                        int32_t* dev_status, void* stream);
+
+/* bca_prefill with the optional workspace of bca_step_attend (256-byte aligned,
+ * caller-owned, NULL = none; see bca_step_workspace_bytes).  With it the kernel's
+ * schedule balances uneven block-causal work: Q-tile pairs are taken heaviest first
+ * (a pair's work is the number of keys its last block allows), the last partial
+ * round of the heavy pairs is split along the keys into chunks merged by a second
+ * kernel, and the light pairs (e.g. the text rows) fill in after them.  Results
+ * equal bca_prefill's up to the order of the fp32 sums.  Calls sharing a
+ * workspace must not overlap. */
+bca_status bca_prefill_ws(const void* q, const void* k, const void* v, void* o, int32_t seq_len,
+                          const int32_t* block_offsets, int32_t n_blocks, int32_t heads,
+                          int32_t head_dim, float scale, bca_kv_slot* slot, uint32_t epoch,
+                          void* workspace, size_t workspace_bytes, int32_t* dev_status,
+                          void* stream);
 
 /* Steps 2..N of a batch of requests at the same phase: every target row of
  * request r attends to [slot r's cached prefix rows ; request r's own target
@@ -174,8 +211,11 @@ bca_status bca_step_attend(const void* q_t, const void* k_t, const void* v_t, vo
  *                      bca_step_q8_scratch_bytes(cu_target[n_req], n_req, heads).
  *                      After the call it holds the Q codes [heads, rows, 128] at
  *                      offset 0 and the fp32 scales [n_req][heads] (by request
- *                      index) at offset round_up(heads * rows * 128, 256); calls
- *                      sharing it must not overlap.
+ *                      index; not written for requests without rows) at offset
+ *                      round_up(heads * rows * 128, 256); calls sharing it must
+ *                      not overlap.  The quantisation is one launch of the store
+ *                      kernel (as bca_kv_store); a non-finite Q value writes
+ *                      BCA_ERR_NONFINITE into *dev_status.
  * Other arguments, results and errors: as bca_step_attend, plus
  * BCA_ERR_UNSUPPORTED if the slots are not BCA_KV_FP8_KV, BCA_ERR_INVALID_ARG for a
  * NULL or misaligned scratch and BCA_ERR_CAPACITY for a small one. */
@@ -189,10 +229,11 @@ bca_status bca_step_attend_q8(const void* q_t, const void* k_t, const void* v_t,
  * requests (0 for arguments out of range). */
 size_t bca_step_q8_scratch_bytes(int64_t rows, int32_t n_req, int32_t heads);
 
-/* Bytes of the optional bca_step_attend workspace that lets the kernel split the
- * last partial round of work along the keys (so that every SM finishes at the same
- * time) for the current device: one chunk of 256 rows x (128 + 2) fp32 per SM.
- * Without it (workspace NULL or too small for any chunk) nothing is split. */
+/* Bytes of the optional bca_step_attend (and bca_prefill_ws) workspace that lets
+ * the kernel split the last partial round of work along the keys (so that every SM
+ * finishes at the same time) for the current device: one chunk of 256 rows x
+ * (128 + 2) fp32 per SM.  Without it (workspace NULL or too small for any chunk)
+ * nothing is split. */
 size_t bca_step_workspace_bytes(void);
 
 /* bca_step_attend for callers that cannot allocate device memory -- for example a
@@ -205,7 +246,9 @@ size_t bca_step_workspace_bytes(void);
  * until the process exits).  The call allocates nothing.
  *  - The first call on a device looks up the array's device address (once per
  *    device, with that device current); make that first call before any stream
- *    capture.
+ *    capture.  The address is kept for the life of the process: do not go on
+ *    using the library on a device after cudaDeviceReset (the kept address would
+ *    no longer be valid).
  *  - Every call shares the one array and it keeps the previous call's contents.
  *    Nothing in it needs to start at zero: each call writes every chunk it reads.
  *    Calls that overlap on the GPU (other streams, other threads) race on it.

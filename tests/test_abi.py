@@ -115,6 +115,25 @@ def test_kv_store_argument_errors(L):
     assert st(slot=s3) == 2
 
 
+def test_kv_store_batch_argument_errors(L):
+    """bca_kv_store_batch checks every item as bca_kv_store does, and that the slots
+    are distinct, before anything is launched; a failed call stamps no slot."""
+    slots = [_slot(L, cap=16, H=2, epoch=0, n=0) for _ in range(3)]
+    Item = bca.StoreItemStruct
+    mk = lambda n_prefix=8, stride=256, slot=0: Item(FAKE.value, FAKE.value, n_prefix, stride,
+                                                     ctypes.pointer(slots[slot]))
+    call = lambda items, epoch=1: L.bca_kv_store_batch((Item * len(items))(*items), len(items),
+                                                       epoch, None, None)
+    assert L.bca_kv_store_batch(None, 1, 1, None, None) == 1
+    assert L.bca_kv_store_batch((Item * 1)(mk()), 0, 1, None, None) == 1
+    assert call([mk(slot=i % 3) for i in range(65)]) == 1  # more than BCA_MAX_BATCH
+    assert call([mk(slot=0), mk(slot=1), mk(slot=0)]) == 1  # a slot twice
+    assert call([mk(slot=0), mk(n_prefix=17, slot=1)]) == 3  # beyond cap
+    assert call([mk(slot=0), mk(stride=128, slot=1)]) == 1
+    assert call([mk(slot=0)], epoch=0) == 1
+    assert all(s.epoch == 0 and s.n_tokens == 0 for s in slots)
+
+
 def test_step_attend_argument_errors(L):
     cu = (ctypes.c_int32 * 3)(0, 100, 228)
     s0, s1 = _slot(L, n=10), _slot(L, n=20)
@@ -145,7 +164,7 @@ def test_step_attend_q8_argument_errors(L):
     H, rows = 2, 228
     need = L.bca_step_q8_scratch_bytes(rows, 2, H)
     codes = (H * rows * 128 + 255) // 256 * 256
-    assert need == codes + 2 * 256
+    assert need == codes + 256  # codes, then the [n_req][H] fp32 scales
     assert L.bca_step_q8_scratch_bytes(-1, 2, H) == 0
     assert L.bca_step_q8_scratch_bytes(rows, 0, H) == 0
     assert L.bca_step_q8_scratch_bytes(rows, 65, H) == 0

@@ -121,3 +121,73 @@ def test_encoder_division_matches_correct_rounding_exhaustively(cuda_device):
     and every bf16 x with |x| <= amax (about 10^9 pairs), the resulting e4m3 code
     equals the code of the correctly rounded fp32 quotient."""
     assert bca.selftest_e4m3_division(cuda_device) == 0
+
+
+def test_batch_store_equals_oracle_per_request(cuda_device):
+    """bca_kv_store_batch: the requests of a batch (different prefix lengths, head
+    counts and cache dtypes) in one launch; every slot's bytes and scales equal the
+    oracle's, rows past the prefix untouched, every slot stamped."""
+    specs = [(1500, 32, "fp8", 1600), (77, 32, "fp8", 80), (640, 8, "bf16", 700),
+             (300, 4, "fp8_v", 300), (0, 4, "fp8", 16), (5000, 2, "fp8", 5000)]
+    items, srcs = [], []
+    for i, (P, H, mode, cap) in enumerate(specs):
+        k = randn_bf16((max(P, 1), H, 128), 500 + 2 * i, cuda_device) * (1 + i)
+        v = randn_bf16((max(P, 1), H, 128), 501 + 2 * i, cuda_device) * 0.3
+        slot = bca.KVSlot(cap, H, mode)
+        _fill_sentinel(slot)
+        items.append((k, v, P, slot))
+        srcs.append((k, v))
+    status = torch.zeros(1, dtype=torch.int32, device=cuda_device)
+    bca.kv_store_batch(items, epoch=9, dev_status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    for (k, v, P, slot), (P_, H, mode, cap) in zip(items, specs):
+        assert slot.n_tokens == P and slot.epoch == 9
+        for x, codes, scales, q in ((k, slot.k_view(), slot.k_scale_view(), mode == "fp8"),
+                                    (v, slot.v_view(), slot.v_scale_view(), mode != "bf16")):
+            if P == 0:
+                continue
+            if q:
+                want_c, want_s = oracle.quantize_prefix(x.cpu(), P, cap)
+                assert np.array_equal(codes[:, :P].cpu().numpy(), want_c[:, :P]), (P, mode)
+                assert np.array_equal(scales.cpu().numpy(), want_s), (P, mode)
+            else:
+                assert torch.equal(codes[:, :P], x[:P].permute(1, 0, 2)), (P, mode)
+            tail = codes[:, P:].contiguous().view(torch.uint8)
+            assert bool((tail == 0x5A).all()), (P, mode)
+
+
+def test_batch_store_rejects_a_repeated_slot(cuda_device):
+    k = randn_bf16((64, 2, 128), 600, cuda_device)
+    slot = bca.KVSlot(64, 2, "fp8")
+    with pytest.raises(bca.BcaError) as e:
+        bca.kv_store_batch([(k, k, 64, slot), (k, k, 32, slot)], epoch=1)
+    assert e.value.status == 1
+    assert slot.epoch == 0
+
+
+def test_non_finite_input_reports_status(cuda_device):
+    """Inputs must be finite.  An e4m3 tensor with an Inf in one head reports
+    BCA_ERR_NONFINITE through dev_status; the other heads are still encoded
+    exactly.  A bf16 copy of the same rows is exact and reports nothing."""
+    P, H = 257, 4
+    k = randn_bf16((P, H, 128), 610, cuda_device)
+    v = randn_bf16((P, H, 128), 611, cuda_device)
+    k[100, 2, 7] = float("inf")
+    status = torch.zeros(1, dtype=torch.int32, device=cuda_device)
+    slot = bca.KVSlot(P, H, "fp8")
+    bca.kv_store(k, v, P, slot, epoch=1, dev_status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 7  # BCA_ERR_NONFINITE
+    kc, ks = oracle.quantize_prefix(k.cpu(), P)
+    for h in (0, 1, 3):
+        assert np.array_equal(slot.k_view()[h].cpu().numpy(), kc[h])
+        assert slot.k_scale_view()[h].item() == ks[h]
+    vc, vs = oracle.quantize_prefix(v.cpu(), P)
+    assert np.array_equal(slot.v_view().cpu().numpy(), vc)
+    status.zero_()
+    s16 = bca.KVSlot(P, H, "bf16")
+    bca.kv_store(k, v, P, s16, epoch=1, dev_status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    assert torch.equal(s16.k_view(), k.permute(1, 0, 2))

@@ -80,15 +80,18 @@ def test_prefix_outputs_ignore_the_target(cuda_device):
     assert torch.equal(o[:P], o2[:P])
 
 
-@pytest.mark.parametrize("wl_index", [2, 3])
-def test_full_size_sampled_rows(cuda_device, wl_index):
-    """The 4-ref edit and native-2K shapes (H=32) at one layer, sampled rows x all
-    heads, including every block boundary +-1."""
+@pytest.mark.parametrize("ws", [False, True])
+@pytest.mark.parametrize("wl_index", [1, 2, 3])
+def test_full_size_sampled_rows(cuda_device, wl_index, ws):
+    """The T2I, 4-ref edit and native-2K shapes (H=32) at one layer, sampled rows x
+    all heads, including every block boundary +-1; with a workspace (the benchmark's
+    configuration: heavy pairs' last round split) and without."""
     wl = W.workload(wl_index)
     req = wl.requests[0]
     q, k, v = W.qkv(wl, 0, 0, 0, cuda_device)
     o = torch.empty_like(q)
-    bca.prefill(q, k, v, o, req.offsets, wl.scale)
+    bca.prefill(q, k, v, o, req.offsets, wl.scale,
+                workspace=bca.step_workspace(cuda_device) if ws else None)
     torch.cuda.synchronize()
     rows = sample_rows(req.seq_len, 48, seed=wl_index, boundaries=req.offsets[1:-1])
     want = oracle.prefill(q, k, v, req.offsets, wl.scale, rows=rows)
@@ -104,3 +107,25 @@ def test_many_items_per_cta_with_half_empty_q_pairs(cuda_device):
     rows = sample_rows(384, 48, seed=5, boundaries=(100, 128, 256))
     want = oracle.prefill(q, k, v, offsets(blocks), SCALE, rows=rows)
     assert_parity(o[torch.from_numpy(rows).to(cuda_device)], want, what="half-empty pairs")
+
+
+@pytest.mark.parametrize("blocks,H", [
+    ([300, 200, 1500], 8),      # a split pair straddles two block ends
+    ([128, 256], 4),            # the tiny workload
+    ([512, 4096], 2),           # T2I blocks, few heads: every heavy pair split
+    ([77, 130, 300, 2000], 6),
+])
+def test_prefill_with_workspace_all_rows(cuda_device, blocks, H):
+    """bca_prefill_ws: heavy Q-tile pairs first, the last partial round of them split
+    along the keys, light pairs after.  A split chunk may hold rows whose block ends
+    before the chunk's keys begin (their chunk is empty), or a whole Q tile with no
+    key in the chunk; all rows against the oracle."""
+    S = int(sum(blocks))
+    q, k, v = (randn_bf16((S, H, 128), 4000 + S + t, cuda_device) for t in range(3))
+    o = torch.full_like(q, float("nan"))
+    status = torch.zeros(1, dtype=torch.int32, device=cuda_device)
+    bca.prefill(q, k, v, o, offsets(blocks), SCALE, dev_status=status,
+                workspace=bca.step_workspace(cuda_device))
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    assert_parity(o, oracle.prefill(q, k, v, offsets(blocks), SCALE), what=f"ws {blocks}")

@@ -25,18 +25,29 @@ def make_request(T, P, H, seed, device, cap=None, mode="bf16"):
     slot = bca.KVSlot(cap if cap is not None else max(P, 1), H, mode)
     slot.buffer.fill_(0xFF)  # NaN patterns in every unused row: must never be read
     bca.kv_store(pk, pv, P, slot, epoch=seed + 1)
-    return dict(q=q, k=k, v=v, pk=pk[:P], pv=pv[:P], slot=slot, T=T, P=P)
+    return dict(q=q, k=k, v=v, pk=pk, pv=pv, slot=slot, T=T, P=P)
 
 
 def oracle_for(req, rows=None):
+    """The oracle's cached step for a request made by make_request.  A bf16 cache is
+    built on the host from the source prefix rows (the slot's bytes are never read,
+    so a store bug cannot cancel a matching read bug); an e4m3 cache is read from the
+    slot, as the e4m3 rule compares against the same bytes (their equality with the
+    oracle's own encoding is checked by the kv_store tests)."""
     s = req["slot"]
     torch.cuda.synchronize()
     if s.dtype == bca.KV_BF16:
-        kc, vc = s.k_view().cpu(), s.v_view().cpu()
+        kc = req["pk"].cpu().permute(1, 0, 2).contiguous()
+        vc = req["pv"].cpu().permute(1, 0, 2).contiguous()
         return oracle.cached_step(req["q"], req["k"], req["v"], kc, vc, req["P"], SCALE,
                                   rows=rows)
     kk = oracle.KIND_E4M3 if s.dtype == bca.KV_FP8_KV else oracle.KIND_BF16
-    kc = s.k_view().cpu()
+    if kk == oracle.KIND_E4M3:
+        kc = s.k_view().cpu()
+    else:  # "fp8_v": bf16 K from the host rows, padded to the slot's capacity
+        H, cap, P = s.struct.num_heads, s.struct.cap_tokens, req["P"]
+        kc = torch.zeros((H, cap, 128), dtype=torch.bfloat16)
+        kc[:, :P] = req["pk"][:P].cpu().permute(1, 0, 2)
     return oracle.cached_step(req["q"], req["k"], req["v"], kc, s.v_view().cpu(), req["P"],
                               SCALE, k_kind=kk, v_kind=oracle.KIND_E4M3,
                               k_scale=s.k_scale_view().cpu().numpy(),

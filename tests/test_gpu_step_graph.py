@@ -95,7 +95,8 @@ def test_graph_layer_against_oracle(cuda_device):
         s, pk, pv = x["slots"][r]
         sl = slice(cu[r], cu[r + 1])
         want = oracle.cached_step(x["q"][sl].cpu(), x["k"][sl].cpu(), x["v"][sl].cpu(),
-                                  s.k_view().cpu(), s.v_view().cpu(), s.n_tokens, SCALE)
+                                  pk.cpu().permute(1, 0, 2).contiguous(),
+                                  pv.cpu().permute(1, 0, 2).contiguous(), s.n_tokens, SCALE)
         assert_parity(o[sl], want, what=f"graph layer 1 request {r}")
 
 

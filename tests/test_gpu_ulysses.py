@@ -5,11 +5,12 @@
    for 1, 2, 4 and 8 ranks (bit-exact byte moves).
  - N ranks emulated on one GPU with the library's pack/unpack and the attention
    kernel on each head shard (the all-to-all done by slicing): the cached step
-   returned to the row blocks is bit-identical to the unsharded call (each (row,
-   head) unit computes the same arithmetic whatever the sharding; no split
-   workspace, so no schedule-dependent merge).
- - One real rank with NCCL: Ulysses.step_attend through all_to_all_single equals
-   the plain call bit for bit."""
+   returned to the row blocks matches the oracle's unsharded cached step within the
+   bf16 tolerance, and is bit-identical to the unsharded call (each (row, head) unit
+   computes the same arithmetic whatever the sharding; no split workspace, so no
+   schedule-dependent merge).
+ - One real rank with NCCL: Ulysses.step_attend through all_to_all_single matches
+   the oracle and equals the plain call bit for bit."""
 import math
 import os
 import socket
@@ -18,8 +19,10 @@ import pytest
 import torch
 
 import block_causal_attention_dit_b200 as bca
+import oracle
 from block_causal_attention_dit_b200.ulysses import ShardPlan, Ulysses
 from block_causal_attention_dit_b200.workloads import randn_bf16
+from _parity import assert_parity
 
 pytestmark = pytest.mark.gpu
 SCALE = 1.0 / math.sqrt(128)
@@ -41,6 +44,13 @@ def test_pack_unpack_are_the_block_permutation(cuda_device, n):
         bca.ulysses_pack(x, send, 3)  # 32 heads do not split over 3 ranks
 
 
+def _oracle(q, k, v, pk, pv):
+    """The oracle's (unsharded) cached step of one request, its cache built on the
+    host from the prefix rows."""
+    return oracle.cached_step(q.cpu(), k.cpu(), v.cpu(), pk.cpu().permute(1, 0, 2).contiguous(),
+                              pv.cpu().permute(1, 0, 2).contiguous(), pk.shape[0], SCALE)
+
+
 def _slots(prefix_k, prefix_v, heads, device):
     s = bca.KVSlot(prefix_k.shape[0], heads, device=device)
     bca.kv_store(prefix_k, prefix_v, prefix_k.shape[0], s, epoch=1)
@@ -48,7 +58,7 @@ def _slots(prefix_k, prefix_v, heads, device):
 
 
 @pytest.mark.parametrize("n", [2, 4])
-def test_emulated_ranks_equal_unsharded(cuda_device, n):
+def test_emulated_ranks_match_oracle_and_unsharded(cuda_device, n):
     H, P = 16, 300
     cu = [0, 512, 1024]
     T = cu[-1]
@@ -89,6 +99,10 @@ def test_emulated_ranks_equal_unsharded(cuda_device, n):
         bca.ulysses_unpack(recv, part, n)
         out[r0:r1] = part
     torch.cuda.synchronize()
+    for r, (pk, pv) in enumerate(pre):
+        sl = slice(cu[r], cu[r + 1])
+        assert_parity(out[sl], _oracle(q[sl], k[sl], v[sl], pk, pv),
+                      what=f"{n} ranks, request {r}")
     assert torch.equal(out, o_ref)
 
 
@@ -109,6 +123,7 @@ def test_single_rank_nccl_exchange(cuda_device):
         u = Ulysses(ShardPlan(1, 0, T, H))
         u.step_attend(q, k, v, o, [0, T], [slot], SCALE)
         torch.cuda.synchronize()
+        assert_parity(o, _oracle(q, k, v, pk, pv), what="one NCCL rank")
         assert torch.equal(o, o_ref)
     finally:
         dist.destroy_process_group()
