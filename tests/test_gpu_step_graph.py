@@ -150,7 +150,7 @@ def test_e4m3_q_graph_replay_equals_eager(cuda_device):
     g = bca.StepGraph([x["q"] for x in L], [x["k"] for x in L], [x["v"] for x in L],
                       [x["o"] for x in L], cu, [[s for s, *_ in x["slots"]] for x in L], SCALE,
                       workspace=ws, dev_status=status, q8_scratch=scratch)
-    assert g.kernel_nodes >= 2 * 4  # per layer: 3 Q-quantisation kernels + attention
+    assert g.kernel_nodes >= 2 * 2  # per layer: the Q quantisation kernel + attention
     for rnd in range(2):
         if rnd:
             for l, x in enumerate(L):
