@@ -14,7 +14,8 @@ Sources (cited by page title and section):
   "Qwen-Image-2.1 + vLLM-Omni day-0", "Serving architecture: the cross-step
   prefix KV cache"; "Qwen/Qwen-Image-2.1" (vLLM recipe), "Prefix KV cache";
   OCP OFP8 specification, E4M3; "SGLang-Diffusion stöder Qwen-Image-2.1 på dag
-  noll", "Siffrorna, och vad de inte säger" (the Q/K norm next to attention).
+  noll", "Siffrorna, och vad de inte säger" (the Q/K norm between the projection of
+  the target rows and the attention).
 """
 from __future__ import annotations
 
@@ -80,6 +81,9 @@ def _load():
         lib.bca_oracle_rms_norm.argtypes = [P, i64, i64, P, ctypes.c_double, P]
         lib.bca_oracle_rope.restype = None
         lib.bca_oracle_rope.argtypes = [P, i64, i64, i64, P, P, P]
+        lib.bca_oracle_qkv_project.restype = ctypes.c_int
+        lib.bca_oracle_qkv_project.argtypes = [P, i64, i64, P, i64, i64, P, P, P, P,
+                                               ctypes.c_double, P, i64, P, P, P, ctypes.c_int]
         lib.bca_oracle_max_threads.restype = ctypes.c_int
         lib.bca_oracle_max_threads.argtypes = []
         _lib = lib
@@ -239,3 +243,33 @@ def rope(y, cos_t, sin_t) -> np.ndarray:
 def qk_norm_rope(x, gamma, cos_t, sin_t, eps: float) -> np.ndarray:
     """rope(rms_norm(x)) for x [rows, H, d] bf16: the exact (fp64) values."""
     return rope(rms_norm(x, gamma, eps), cos_t, sin_t)
+
+
+def qkv_project(x, w, gamma_q, gamma_k, cos_t, sin_t, eps: float, heads: int, rows=None,
+                nthreads: int = 0):
+    """x [T, D] bf16 rows, w [3*heads*d, D] bf16 (torch Linear layout: Q heads, K
+    heads, V heads) -> (q, k, v), each fp64 [n_rows, heads, d]: the projection
+    y = x w^T, then rope(rms_norm(.)) of every Q and K head vector; V as projected.
+    gamma_*: [d] fp32; cos_t, sin_t: [T, d/2] fp32."""
+    xb, wb = _bits16(x), _bits16(w)
+    T, D = xb.shape
+    N, D2 = wb.shape
+    assert D2 == D and N % (3 * heads) == 0
+    d = N // (3 * heads)
+    gq = np.ascontiguousarray(gamma_q, dtype=np.float32)
+    gk = np.ascontiguousarray(gamma_k, dtype=np.float32)
+    c = np.ascontiguousarray(cos_t, dtype=np.float32)
+    s = np.ascontiguousarray(sin_t, dtype=np.float32)
+    assert gq.shape == (d,) and gk.shape == (d,) and c.shape == (T, d // 2) and s.shape == c.shape
+    rws = None if rows is None else np.ascontiguousarray(rows, dtype=np.int64)
+    n = T if rws is None else len(rws)
+    q = np.empty((n, heads, d), dtype=np.float64)
+    k = np.empty_like(q)
+    v = np.empty_like(q)
+    rc = _load().bca_oracle_qkv_project(_ptr(xb), T, D, _ptr(wb), heads, d, _ptr(gq), _ptr(gk),
+                                        _ptr(c), _ptr(s), float(eps),
+                                        None if rws is None else _ptr(rws), n, _ptr(q), _ptr(k),
+                                        _ptr(v), int(nthreads))
+    if rc != 0:
+        raise ValueError("oracle qkv_project: bad arguments")
+    return q, k, v

@@ -325,20 +325,33 @@ int bca_oracle_cached_step(const uint16_t* q_t, const uint16_t* k_t, const uint1
  * channel pairs by caller-given angles (as cos/sin tables).  fp64 throughout; the
  * fp32 weights and tables are widened exactly. */
 
+/* One vector: y[c] = x[c] / sqrt(mean_c' x[c']^2 + eps) * gamma[c]. */
+static void rms_norm_vec(const double* x, int64_t d, const float* gamma, double eps, double* y) {
+  double ss = 0.0;
+  for (int64_t c = 0; c < d; ++c) ss += x[c] * x[c];
+  double inv = 1.0 / sqrt(ss / (double)d + eps);
+  for (int64_t c = 0; c < d; ++c) y[c] = x[c] * inv * (double)gamma[c];
+}
+
+/* One vector: pair (2i, 2i+1) turned by the angle whose cos/sin are cs[i], sn[i]. */
+static void rope_vec(const double* y, int64_t d, const float* cs, const float* sn, double* out) {
+  for (int64_t i = 0; i < d / 2; ++i) {
+    double c = (double)cs[i], s = (double)sn[i];
+    out[2 * i] = y[2 * i] * c - y[2 * i + 1] * s;
+    out[2 * i + 1] = y[2 * i] * s + y[2 * i + 1] * c;
+  }
+}
+
 /* y[v, c] = x[v, c] / sqrt(mean_c' x[v, c']^2 + eps) * gamma[c], for n_vec vectors
  * of d bf16 values each. */
 void bca_oracle_rms_norm(const uint16_t* x, int64_t n_vec, int64_t d, const float* gamma,
                          double eps, double* y) {
+  double* xv = (double*)malloc(sizeof(double) * (size_t)d);
   for (int64_t v = 0; v < n_vec; ++v) {
-    double ss = 0.0;
-    for (int64_t c = 0; c < d; ++c) {
-      double e = bca_oracle_bf16_to_f64(x[v * d + c]);
-      ss += e * e;
-    }
-    double inv = 1.0 / sqrt(ss / (double)d + eps);
-    for (int64_t c = 0; c < d; ++c)
-      y[v * d + c] = bca_oracle_bf16_to_f64(x[v * d + c]) * inv * (double)gamma[c];
+    for (int64_t c = 0; c < d; ++c) xv[c] = bca_oracle_bf16_to_f64(x[v * d + c]);
+    rms_norm_vec(xv, d, gamma, eps, y + v * d);
   }
+  free(xv);
 }
 
 /* Rotate every pair (2i, 2i+1) of y [rows, H, d] by the angle of row t and pair i:
@@ -348,11 +361,61 @@ void bca_oracle_rope(const double* y, int64_t rows, int64_t H, int64_t d, const 
                      const float* sin_t, double* out) {
   for (int64_t t = 0; t < rows; ++t)
     for (int64_t h = 0; h < H; ++h)
-      for (int64_t i = 0; i < d / 2; ++i) {
-        const double* a = y + (t * H + h) * d + 2 * i;
-        double* o = out + (t * H + h) * d + 2 * i;
-        double cs = (double)cos_t[t * (d / 2) + i], sn = (double)sin_t[t * (d / 2) + i];
-        o[0] = a[0] * cs - a[1] * sn;
-        o[1] = a[0] * sn + a[1] * cs;
+      rope_vec(y + (t * H + h) * d, d, cos_t + t * (d / 2), sin_t + t * (d / 2),
+               out + (t * H + h) * d);
+}
+
+/* ------------------------------------------------------------------------ */
+/* Q/K/V projection with the Q/K norm and rotary embedding                   */
+/* ------------------------------------------------------------------------ */
+/* The same page and section place the Q/K-norm change between the projection of
+ * the target rows and the attention.  Reading taken: one linear projection (no
+ * bias) of the rows x [T, D] by w [3*H*d, D] (the torch Linear layout: output
+ * features Q heads 0..H-1, then K heads, then V heads, d = head_dim each), then the
+ * RMS norm + rotary embedding above on every Q and K head vector; V as projected.
+ *   y[t, n]    = sum_c x[t, c] * w[n, c]                       (fp64)
+ *   q[t, h, :] = rope(rms_norm(y[t, h*d .. h*d+d-1], gamma_q), cos[t], sin[t])
+ *   k[t, h, :] = rope(rms_norm(y[t, (H+h)*d ..], gamma_k), cos[t], sin[t])
+ *   v[t, h, :] = y[t, (2H+h)*d ..]
+ * rows: the rows to compute (NULL: all T); outputs [n_rows, H, d] fp64. */
+int bca_oracle_qkv_project(const uint16_t* x, int64_t T, int64_t D, const uint16_t* w, int64_t H,
+                           int64_t d, const float* gamma_q, const float* gamma_k,
+                           const float* cos_t, const float* sin_t, double eps,
+                           const int64_t* rows, int64_t n_rows, double* q, double* k, double* v,
+                           int nthreads) {
+  if (T < 1 || D < 1 || H < 1 || d < 2 || (d & 1)) return -1;
+  if (!rows) n_rows = T;
+  for (int64_t r = 0; r < n_rows; ++r)
+    if (rows && (rows[r] < 0 || rows[r] >= T)) return -1;
+  const int64_t N = 3 * H * d;
+  set_threads(nthreads);
+#pragma omp parallel
+  {
+    double* xr = (double*)malloc(sizeof(double) * (size_t)D);
+    double* y = (double*)malloc(sizeof(double) * (size_t)N);
+    double* nrm = (double*)malloc(sizeof(double) * (size_t)d);
+#pragma omp for schedule(dynamic, 1)
+    for (int64_t r = 0; r < n_rows; ++r) {
+      int64_t t = rows ? rows[r] : r;
+      for (int64_t c = 0; c < D; ++c) xr[c] = bca_oracle_bf16_to_f64(x[t * D + c]);
+      for (int64_t n = 0; n < N; ++n) {
+        double acc = 0.0;
+        for (int64_t c = 0; c < D; ++c) acc += xr[c] * bca_oracle_bf16_to_f64(w[n * D + c]);
+        y[n] = acc;
       }
+      const float* cs = cos_t + t * (d / 2);
+      const float* sn = sin_t + t * (d / 2);
+      for (int64_t h = 0; h < H; ++h) {
+        rms_norm_vec(y + h * d, d, gamma_q, eps, nrm);
+        rope_vec(nrm, d, cs, sn, q + (r * H + h) * d);
+        rms_norm_vec(y + (H + h) * d, d, gamma_k, eps, nrm);
+        rope_vec(nrm, d, cs, sn, k + (r * H + h) * d);
+        for (int64_t c = 0; c < d; ++c) v[(r * H + h) * d + c] = y[(2 * H + h) * d + c];
+      }
+    }
+    free(xr);
+    free(y);
+    free(nrm);
+  }
+  return 0;
 }
