@@ -17,6 +17,8 @@ three calls of the method mirror include/bca.h one to one:
       the same over e4m3 ("fp8") slots with e4m3 Q against the e4m3 cached keys.
   qk_norm_rope(q, k, gamma_q, gamma_k, cos_t, sin_t, eps)
       Q/K RMS norm + rotary embedding of the rows entering attention (in place).
+  qkv_project(x, w, q, k, v, gamma_q, gamma_k, cos_t, sin_t, eps)
+      the projection of rows into Q, K, V with that norm + rotary in its epilogue.
   StepGraph(q_layers, k_layers, v_layers, o_layers, cu_target, slots_per_layer, scale)
       the cached-step calls of every layer of one layout recorded as one CUDA graph;
       .launch() replays them (bit-identical to the eager calls).
@@ -35,7 +37,7 @@ __all__ = [
     "BcaError", "KVSlot", "KV_BF16", "KV_FP8_V", "KV_FP8_KV", "MAX_BLOCKS", "MAX_BATCH",
     "lib", "prefill", "kv_store", "kv_store_batch", "step_attend", "step_workspace", "step_workspace_bytes",
     "step_attend_q8", "step_q8_scratch", "step_q8_scratch_bytes", "q8_views",
-    "StepGraph", "qk_norm_rope", "ulysses_pack", "ulysses_unpack",
+    "StepGraph", "qk_norm_rope", "qkv_project", "ulysses_pack", "ulysses_unpack",
     "slot_bytes", "set_wait_timeout_ns",
     "selftest_wait_timeout", "selftest_exp2", "selftest_e4m3_division", "status_string",
     "version", "LIB_PATH",
@@ -149,6 +151,8 @@ def lib():
     L.bca_debug_set_trace.argtypes = [P, i32]
     L.bca_qk_norm_rope.restype = ctypes.c_int
     L.bca_qk_norm_rope.argtypes = [P, P, ctypes.c_int64, i32, i32, P, P, P, P, f32, P]
+    L.bca_qkv_project.restype = ctypes.c_int
+    L.bca_qkv_project.argtypes = [P, P, P, P, P, i32, i32, i32, i32, P, P, P, P, f32, P, P]
     for name in ("bca_ulysses_pack", "bca_ulysses_unpack"):
         getattr(L, name).restype = ctypes.c_int
         getattr(L, name).argtypes = [P, P, ctypes.c_int64, i32, i32, i32, P]
@@ -499,6 +503,35 @@ def qk_norm_rope(q, k, gamma_q, gamma_k, cos_t, sin_t, eps: float = 1e-6, stream
     _check(lib().bca_qk_norm_rope(_ptr(q), _ptr(k), rows, H, d, _ptr(gamma_q), _ptr(gamma_k),
                                   _ptr(cos_t), _ptr(sin_t), float(eps),
                                   _stream(stream, ref.device)), "bca_qk_norm_rope")
+
+
+def qkv_project(x, w, q, k, v, gamma_q, gamma_k, cos_t, sin_t, eps: float = 1e-6,
+                dev_status=None, stream=None):
+    """q, k, v ([rows, H, 128] bf16 CUDA, written) from x [rows, D] and w [3*H*128, D]
+    (bf16 CUDA): the projection x w^T with the Q/K RMS norm (gamma_q / gamma_k, [128]
+    fp32) and the rotary embedding (cos_t / sin_t, [rows, 64] fp32) in its epilogue."""
+    import torch
+    call = "bca_qkv_project"
+    _cuda(x, call, "x", torch.bfloat16)
+    _need(x.dim() == 2 and x.is_contiguous(), call, "x must be a contiguous [rows, D]")
+    rows, D = x.shape
+    _cuda(w, call, "w", torch.bfloat16, x.device)
+    _need(w.dim() == 2 and w.is_contiguous() and w.shape[1] == D, call,
+          "w must be a contiguous [3*H*128, D]")
+    _rows_tensor(q, call, "q")
+    _need(q.device == x.device and q.shape[0] == rows, call, "q must have x's rows")
+    for name, t in (("k", k), ("v", v)):
+        _rows_tensor(t, call, name, like=q)
+    H, d = q.shape[1], q.shape[2]
+    _need(w.shape[0] == 3 * H * d, call, "w must have 3*H*head_dim rows")
+    for name, t, n in (("gamma_q", gamma_q, d), ("gamma_k", gamma_k, d),
+                       ("cos_t", cos_t, rows * (d // 2)), ("sin_t", sin_t, rows * (d // 2))):
+        _need(t is not None, call, f"{name} is required")
+        _aux(t, call, name, x.device, torch.float32, n)
+    _aux(dev_status, call, "dev_status", x.device, torch.int32)
+    _check(lib().bca_qkv_project(_ptr(x), _ptr(w), _ptr(q), _ptr(k), _ptr(v), rows, D, H, d,
+                                 _ptr(gamma_q), _ptr(gamma_k), _ptr(cos_t), _ptr(sin_t),
+                                 float(eps), _ptr(dev_status), _stream(stream, x.device)), call)
 
 
 def ulysses_pack(x, send, n_ranks: int, stream=None):

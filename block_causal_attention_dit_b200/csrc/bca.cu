@@ -29,6 +29,7 @@
 #include "attn_kernel.cuh"
 #include "kv_store_kernel.cuh"
 #include "qk_norm_rope_kernel.cuh"
+#include "qkv_proj_kernel.cuh"
 #include "ulysses_kernel.cuh"
 
 namespace {
@@ -936,6 +937,77 @@ extern "C" bca_status bca_qk_norm_rope(void* q, void* k, int64_t rows, int32_t h
   const int64_t want = (2 * rows + bca::kNormWarpsPerBlock - 1) / bca::kNormWarpsPerBlock;
   const int blocks = static_cast<int>(std::min<int64_t>(want, static_cast<int64_t>(sms) * 8));
   bca::qk_norm_rope_kernel<<<blocks, bca::kNormThreads, 0, static_cast<cudaStream_t>(stream)>>>(p);
+  return cudaGetLastError() == cudaSuccess ? BCA_OK : BCA_ERR_CUDA;
+}
+
+// ---------------------------------------------------------------------------
+// Q/K/V projection with the Q/K norm and rotary embedding in the epilogue
+// ---------------------------------------------------------------------------
+namespace {
+// 2-D tiled map, 128-byte swizzle: dims (d0 inner, d1), row stride in bytes.
+bool make_map_2d(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_t stride1,
+                 uint32_t b0, uint32_t b1) {
+  const cuuint64_t dims[2] = {d0, d1};
+  const cuuint64_t strides[1] = {stride1};
+  const cuuint32_t box[2] = {b0, b1};
+  const cuuint32_t estr[2] = {1, 1};
+  return g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+std::vector<char>& proj_attr_flags() {
+  static std::vector<char> done;
+  return done;
+}
+}  // namespace
+
+extern "C" bca_status bca_qkv_project(const void* x, const void* w, void* q, void* k, void* v,
+                                      int32_t rows, int32_t d_model, int32_t heads,
+                                      int32_t head_dim, const float* gamma_q,
+                                      const float* gamma_k, const float* cos_t,
+                                      const float* sin_t, float eps, int32_t* dev_status,
+                                      void* stream) {
+  if (head_dim != 128) return BCA_ERR_UNSUPPORTED;
+  if (d_model < 64 || d_model % 64 != 0) return BCA_ERR_UNSUPPORTED;
+  if (rows < 0 || heads < 1 || heads > 256 || !(eps > 0.0f) || !std::isfinite(eps))
+    return BCA_ERR_INVALID_ARG;
+  if (rows == 0) return BCA_OK;
+  for (const void* ptr : {x, w, static_cast<const void*>(q), static_cast<const void*>(k),
+                          static_cast<const void*>(v), static_cast<const void*>(gamma_q),
+                          static_cast<const void*>(gamma_k), static_cast<const void*>(cos_t),
+                          static_cast<const void*>(sin_t)})
+    if (!ptr || !aligned16(ptr)) return BCA_ERR_INVALID_ARG;
+  if (!get_encode()) return BCA_ERR_CUDA;
+  const int64_t feats = 3ll * heads * 128;
+  bca::ProjParams p;
+  std::memset(&p, 0, sizeof(p));
+  if (!make_map_2d(&p.tm_x, x, d_model, rows, static_cast<uint64_t>(d_model) * 2, bca::kPBK,
+                   bca::kPBM) ||
+      !make_map_2d(&p.tm_w, w, d_model, feats, static_cast<uint64_t>(d_model) * 2, bca::kPBK,
+                   bca::kPBN) ||
+      !map_thd(&p.tm_out[0], q, rows, heads) || !map_thd(&p.tm_out[1], k, rows, heads) ||
+      !map_thd(&p.tm_out[2], v, rows, heads))
+    return BCA_ERR_CUDA;
+  p.gamma_q = gamma_q;
+  p.gamma_k = gamma_k;
+  p.cos_t = cos_t;
+  p.sin_t = sin_t;
+  p.rows = rows;
+  p.heads = heads;
+  p.m_tiles = (rows + bca::kPBM - 1) / bca::kPBM;
+  p.n_tiles = static_cast<int32_t>((feats + bca::kPBN - 1) / bca::kPBN);
+  p.k_steps = d_model / bca::kPBK;
+  p.eps = eps;
+  p.dev_status = dev_status;
+  p.timeout_ns = g_timeout_ns.load();
+  if (!ensure_smem_attr(bca::qkv_proj_kernel, bca::ProjSmem::kDynamicBytes, proj_attr_flags()))
+    return BCA_ERR_CUDA;
+  const int sms = sm_count();
+  if (sms <= 0) return BCA_ERR_CUDA;
+  const int grid = std::min(sms, p.m_tiles * p.n_tiles);
+  bca::qkv_proj_kernel<<<grid, bca::kPThreads, bca::ProjSmem::kDynamicBytes,
+                         static_cast<cudaStream_t>(stream)>>>(p);
   return cudaGetLastError() == cudaSuccess ? BCA_OK : BCA_ERR_CUDA;
 }
 

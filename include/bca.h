@@ -282,6 +282,31 @@ bca_status bca_qk_norm_rope(void* q, void* k, int64_t rows, int32_t heads, int32
                             const float* gamma_q, const float* gamma_k, const float* cos_t,
                             const float* sin_t, float eps, void* stream);
 
+/* The projection that produces the attention's inputs, with the Q/K norm and the
+ * rotary embedding of bca_qk_norm_rope applied in its epilogue (same page and
+ * section: the Q/K-norm change sits between the projection and the attention).
+ * One linear projection (no bias) of the rows x by w, then, per head:
+ *   y          = x w^T                  x [rows, d_model], w [3*heads*128, d_model]
+ *                                       (torch Linear layout; output features: Q
+ *                                       heads, then K heads, then V heads)
+ *   q[t, h, :] = rope(rms_norm(y[t, 128h ..], gamma_q))        (as bca_qk_norm_rope)
+ *   k[t, h, :] = rope(rms_norm(y[t, 128(heads+h) ..], gamma_k))
+ *   v[t, h, :] = y[t, 128(2 heads+h) ..]
+ * Tensor cores with fp32 accumulation; fp32 epilogue; one round-to-nearest-even to
+ * bf16.  q, k, v: device bf16 [rows, heads, 128] each (the layout of
+ * bca_step_attend / bca_prefill), written in full; no separate normalisation pass
+ * reads them again.
+ *   x, w          : device bf16, rows d_model elements apart.
+ *   gamma_q/k     : [128] fp32 device.  cos_t, sin_t: [rows, 64] fp32 device.
+ * Errors: BCA_ERR_UNSUPPORTED for head_dim != 128 or d_model not a positive multiple
+ * of 64; BCA_ERR_INVALID_ARG for rows < 0, heads outside [1, 256], eps not finite
+ * and > 0, or a NULL / non-16-byte-aligned pointer.  rows == 0 enqueues nothing.
+ * dev_status: nullable, receives BCA_ERR_DEVICE_TIMEOUT if a bounded wait expires. */
+bca_status bca_qkv_project(const void* x, const void* w, void* q, void* k, void* v, int32_t rows,
+                           int32_t d_model, int32_t heads, int32_t head_dim,
+                           const float* gamma_q, const float* gamma_k, const float* cos_t,
+                           const float* sin_t, float eps, int32_t* dev_status, void* stream);
+
 /* ---- Head-sharded (Ulysses) sequence parallelism -----------------------------
  * "Qwen/Qwen-Image-2.1" (recipes.vllm.ai), "Overview" and "Limitations": the
  * engine's sequence parallelism is Ulysses; "SGLang-Diffusion stöder Qwen-Image-2.1

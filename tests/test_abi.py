@@ -265,3 +265,23 @@ def test_binding_rejects_host_tensors_before_the_library_is_called():
         with pytest.raises(bca.BcaError) as e:
             call()
         assert e.value.status == 1 and "CUDA tensor" in str(e.value)
+
+
+def test_qkv_project_argument_errors(L):
+    """bca_qkv_project checks shapes, sizes and pointers before any CUDA call."""
+    call = lambda **kw: L.bca_qkv_project(
+        kw.get("x", FAKE), kw.get("w", FAKE), FAKE, FAKE, FAKE, kw.get("rows", 64),
+        kw.get("D", 128), kw.get("H", 2), kw.get("d", 128), FAKE, FAKE, kw.get("cos", FAKE),
+        FAKE, kw.get("eps", 1e-6), None, None)
+    assert call(d=64) == 2
+    assert call(D=100) == 2
+    assert call(D=0) == 2
+    assert call(rows=-1) == 1
+    assert call(H=0) == 1
+    assert call(H=257) == 1
+    assert call(eps=0.0) == 1
+    assert call(eps=float("inf")) == 1
+    assert call(x=None) == 1
+    assert call(w=ctypes.c_void_p((1 << 24) + 8)) == 1  # misaligned
+    assert call(cos=None) == 1
+    assert call(rows=0, x=None) == 0  # nothing to do, nothing checked
