@@ -23,6 +23,8 @@ oracle_extra = the oracle on the tiny workload in full, and its rate on samples 
          the larger workloads extrapolated to 40 steps x 32 layers.
 qk_norm_rope = the Q/K RMS norm + rotary embedding call on the cached step's
          target rows, GB/s against the measured HBM copy bandwidth.
+qkv_project = the projection of the target rows into Q, K, V with that norm and
+         rotary in its epilogue, TFLOP/s against the measured bf16 peak.
 graph  = the same pass with each step's cached-step calls of all layers replayed
          from one CUDA graph (bca_step_graph; one graph per assignment of input
          buffers to layers); the prefill stays eager.
@@ -495,6 +497,73 @@ def store_leg(runner, peaks, reps: int = 5):
             "timing": "CUDA events around each bca_kv_store_batch enqueue"}
 
 
+def qkv_leg(device, peaks, rows: int, heads: int, calls: int = 20):
+    """bca_qkv_project on the cached step's target rows (model width heads x 128):
+    TFLOP/s (2 x rows x width x 3 width) against the measured bf16 peak (burst: the
+    kernel is timed alone).  Beside it, for context: the same projection as one
+    cuBLAS bf16 GEMM (torch.matmul, no epilogue) followed by bca_qk_norm_rope -- the
+    two-pass path the fused epilogue replaces.  Two input sets alternate."""
+    import numpy as np
+    import torch
+    import block_causal_attention_dit_b200 as bca
+    from block_causal_attention_dit_b200 import workloads as W
+    D = heads * 128
+    xs = [W.randn_bf16((rows, D), 95000 + i, device) for i in range(2)]
+    w = (W.randn_bf16((3 * D, D), 95010, device).float() * D ** -0.5).to(torch.bfloat16)
+    rng = np.random.default_rng(1)
+    gq, gk = (torch.from_numpy(rng.uniform(0.5, 1.5, 128).astype(np.float32)).to(device)
+              for _ in range(2))
+    ang = np.arange(rows)[:, None] * 10000.0 ** (-np.arange(64) / 64.0)
+    cos_t = torch.from_numpy(np.cos(ang).astype(np.float32)).to(device)
+    sin_t = torch.from_numpy(np.sin(ang).astype(np.float32)).to(device)
+    q, k, v = (torch.empty((rows, heads, 128), dtype=torch.bfloat16, device=device)
+               for _ in range(3))
+    status = torch.zeros(1, dtype=torch.int32, device=device)
+    y = torch.empty((rows, 3 * D), dtype=torch.bfloat16, device=device)
+
+    def fused(i):
+        bca.qkv_project(xs[i % 2], w, q, k, v, gq, gk, cos_t, sin_t, 1e-6, dev_status=status)
+
+    def two_pass(i):
+        torch.matmul(xs[i % 2], w.t(), out=y)
+        yv = y.view(rows, 3, heads, 128)
+        bca.qk_norm_rope(yv[:, 0].contiguous(), yv[:, 1].contiguous(), gq, gk, cos_t, sin_t)
+
+    def gemm(i):
+        torch.matmul(xs[i % 2], w.t(), out=y)
+
+    def t(fn):
+        for i in range(3):
+            fn(i)
+        torch.cuda.synchronize()
+        ev = []
+        for i in range(calls):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            fn(i)
+            b.record()
+            ev.append((a, b))
+        torch.cuda.synchronize()
+        return statistics.median(a.elapsed_time(b) for a, b in ev)
+
+    ms = t(fused)
+    if int(status.item()) != 0:
+        raise RuntimeError(f"device status {int(status.item())} (qkv leg)")
+    ms_gemm, ms_two = t(gemm), t(two_pass)
+    flops = 2.0 * rows * D * 3 * D
+    burst = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    sus = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
+    tf = flops / (ms / 1e3) / 1e12
+    return {"bound": "tensor", "rows": rows, "d_model": D, "heads": heads, "ms": ms,
+            "achieved": tf, "peak": burst, "unit": "TFLOP/s", "frac": tf / burst,
+            "frac_of_sustained": tf / sus, "peak_kind": "bf16 burst (timed alone)",
+            "context_cublas_gemm_ms": ms_gemm,
+            "context_cublas_gemm_tflops": flops / (ms_gemm / 1e3) / 1e12,
+            "context_two_pass_ms": ms_two,
+            "context_note": "cuBLAS GEMM (torch.matmul) then bca_qk_norm_rope on copies of "
+                            "Q and K: the unfused path, for context only"}
+
+
 def config_leg(index: int, device, peaks, reps: int = 3):
     """One layer of workload `index` on its own: the prefill of every request
     (bca_prefill with the workspace, attention only), the prefix store of all
@@ -625,10 +694,11 @@ DATASHEET_SOURCE = ("NVIDIA HGX B200 datasheet: FP16/BF16 tensor 36 PFLOPS per 8
 
 
 def q8_leg(device, peaks, calls: int = 10):
-    """bca_step_attend_q8 against bca_step_attend on the step-batched serving
+    """The three cached-step paths over an e4m3 cache on the step-batched serving
     workload (8 requests, ragged prefixes, target 4096, H=32, e4m3 K and V cache),
-    one layer's cached step, inputs larger than L2.  The e4m3-Q call includes its Q
-    quantisation pre-pass.  Its peak blends the FP8 peak (the measured bf16 peak x
+    one layer's cached step, inputs larger than L2: bca_step_attend (tiles converted
+    in the kernel), bca_step_attend_dq (cache expanded once, then bf16 tiles) and
+    bca_step_attend_q8 (e4m3 Q x e4m3 K; its Q quantisation pre-pass included).  Its peak blends the FP8 peak (the measured bf16 peak x
     the nominal fp8/bf16 ratio of 2) for the cached keys' Q K^T FLOPs with the bf16
     peak for the rest."""
     import numpy as np
@@ -653,9 +723,14 @@ def q8_leg(device, peaks, calls: int = 10):
         cu.append(cu[-1] + r.target)
     ws = bca.step_workspace(device)
     scratch = bca.step_q8_scratch(cu[-1], len(slots), H, device)
+    dq_scratch = bca.step_dq_scratch(slots, device)
+    o_c = torch.empty_like(q)
     status = torch.zeros(1, dtype=torch.int32, device=device)
     calls_ = {"dequant": lambda: bca.step_attend(q, k, v, o_a, cu, slots, wl.scale, workspace=ws,
                                                  dev_status=status),
+              "dq": lambda: bca.step_attend_dq(q, k, v, o_c, cu, slots, wl.scale,
+                                               dq_scratch=dq_scratch, workspace=ws,
+                                               dev_status=status),
               "q8": lambda: bca.step_attend_q8(q, k, v, o_b, cu, slots, wl.scale,
                                                q8_scratch=scratch, workspace=ws,
                                                dev_status=status)}
@@ -684,6 +759,15 @@ def q8_leg(device, peaks, calls: int = 10):
     t8 = flops / (ms["q8"] / 1e3) / 1e12
     return {"workload": wl.name, "dequant_ms": ms["dequant"], "q8_ms": ms["q8"],
             "dequant_tflops": flops / (ms["dequant"] / 1e3) / 1e12, "q8_tflops": t8,
+            "dq_ms": ms["dq"], "dq_tflops": flops / (ms["dq"] / 1e3) / 1e12,
+            "dq_scratch_bytes": bca.step_dq_scratch_bytes(slots),
+            "dq_bitwise_equal_to_dequant": bool(torch.equal(o_a, o_c)),
+            "paths": {"dequant": "bca_step_attend: e4m3 tiles converted in shared memory by "
+                                 "every CTA that reads them",
+                      "dq": "bca_step_attend_dq: cache expanded to bf16 once per call "
+                            "(expansion kernel included in the time)",
+                      "q8": "bca_step_attend_q8: e4m3 Q x e4m3 K for the cached keys "
+                            "(Q quantisation included)"},
             "speedup": ms["dequant"] / ms["q8"], "fp8_flop_share": flops_f8 / flops,
             "peak": mixed_peak, "frac": t8 / mixed_peak,
             "peak_kind": "fp8 (2x measured bf16 sustained) for the cached keys' Q K^T, "
@@ -876,6 +960,10 @@ def main():
     if not args.no_q8 and n_gpus == 1:
         q8 = q8_leg(device, peaks)
 
+    qkv = None
+    if not args.no_norm:
+        qkv = qkv_leg(device, peaks, sum(r.target for r in wl.requests), wl.heads)
+
     configs = None
     if not args.no_configs and n_gpus == 1:
         configs = {}
@@ -911,7 +999,7 @@ def main():
             "datasheet_bf16": {"tflops": DATASHEET_BF16_DENSE_TFLOPS, "source": DATASHEET_SOURCE,
                                "cached_step_frac": achieved / DATASHEET_BF16_DENSE_TFLOPS},
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "graph": graph,
-            "qk_norm_rope": norm, "kv_store": store, "fp8_q8_step": q8,
+            "qk_norm_rope": norm, "qkv_project": qkv, "kv_store": store, "fp8_q8_step": q8,
             "per_workload_one_layer": configs, "oracle_extra": oracle_extra,
             "gpu_launches": runner.launches_per_step * args.steps, "clocks": clocks}
     if rank == 0:

@@ -15,6 +15,8 @@ three calls of the method mirror include/bca.h one to one:
       ragged batch of requests at the same phase.
   step_attend_q8(q_t, k_t, v_t, o_t, cu_target, slots, scale, q8_scratch)
       the same over e4m3 ("fp8") slots with e4m3 Q against the e4m3 cached keys.
+  step_attend_dq(q_t, k_t, v_t, o_t, cu_target, slots, scale, dq_scratch)
+      step_attend over e4m3 slots with the cache expanded to bf16 once per call.
   qk_norm_rope(q, k, gamma_q, gamma_k, cos_t, sin_t, eps)
       Q/K RMS norm + rotary embedding of the rows entering attention (in place).
   qkv_project(x, w, q, k, v, gamma_q, gamma_k, cos_t, sin_t, eps)
@@ -37,6 +39,7 @@ __all__ = [
     "BcaError", "KVSlot", "KV_BF16", "KV_FP8_V", "KV_FP8_KV", "MAX_BLOCKS", "MAX_BATCH",
     "lib", "prefill", "kv_store", "kv_store_batch", "step_attend", "step_workspace", "step_workspace_bytes",
     "step_attend_q8", "step_q8_scratch", "step_q8_scratch_bytes", "q8_views",
+    "step_attend_dq", "step_dq_scratch", "step_dq_scratch_bytes",
     "StepGraph", "qk_norm_rope", "qkv_project", "ulysses_pack", "ulysses_unpack",
     "slot_bytes", "set_wait_timeout_ns",
     "selftest_wait_timeout", "selftest_exp2", "selftest_e4m3_division", "status_string",
@@ -135,6 +138,11 @@ def lib():
     L.bca_step_attend_q8.restype = ctypes.c_int
     L.bca_step_attend_q8.argtypes = [P, P, P, P, P, SP, i32, i32, i32, f32, P, ctypes.c_size_t,
                                      P, ctypes.c_size_t, P, P]
+    L.bca_step_attend_dq.restype = ctypes.c_int
+    L.bca_step_attend_dq.argtypes = [P, P, P, P, P, SP, i32, i32, i32, f32, P, ctypes.c_size_t,
+                                     P, ctypes.c_size_t, P, P]
+    L.bca_step_dq_scratch_bytes.restype = ctypes.c_size_t
+    L.bca_step_dq_scratch_bytes.argtypes = [SP, i32]
     L.bca_step_q8_scratch_bytes.restype = ctypes.c_size_t
     L.bca_step_q8_scratch_bytes.argtypes = [ctypes.c_int64, i32, i32]
     L.bca_status_string.restype = ctypes.c_char_p
@@ -431,6 +439,40 @@ def step_attend(q_t, k_t, v_t, o_t, cu_target, slots, scale: float, workspace=No
                                  len(slots), H, d, float(scale), _ptr(workspace), ws_bytes,
                                  _ptr(dev_status), _stream(stream, q_t.device)),
            "bca_step_attend")
+
+
+def step_dq_scratch_bytes(slots) -> int:
+    """Bytes of step_attend_dq's scratch for these (filled) slots."""
+    arr = (SlotStruct * len(slots))(*[s.struct for s in slots])
+    return int(lib().bca_step_dq_scratch_bytes(arr, len(slots)))
+
+
+def step_dq_scratch(slots, device="cuda"):
+    import torch
+    return torch.empty(max(step_dq_scratch_bytes(slots), 256), dtype=torch.uint8, device=device)
+
+
+def step_attend_dq(q_t, k_t, v_t, o_t, cu_target, slots, scale: float, dq_scratch=None,
+                   workspace=None, dev_status=None, stream=None):
+    """step_attend over e4m3 ("fp8_v" / "fp8") slots with each cache tensor expanded
+    once to bf16 in dq_scratch before the attention (bit-identical results)."""
+    import torch
+    call = "bca_step_attend_dq"
+    cu = _check_step_args(call, q_t, k_t, v_t, o_t, cu_target, slots)
+    _, H, d = q_t.shape
+    if dq_scratch is None:
+        dq_scratch = step_dq_scratch(slots, q_t.device)
+    _aux(dq_scratch, call, "dq_scratch", q_t.device)
+    _aux(workspace, call, "workspace", q_t.device)
+    _aux(dev_status, call, "dev_status", q_t.device, torch.int32)
+    arr = (SlotStruct * len(slots))(*[s.struct for s in slots])
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib().bca_step_attend_dq(_ptr(q_t), _ptr(k_t), _ptr(v_t), _ptr(o_t), _i32_array(cu),
+                                    arr, len(slots), H, d, float(scale), _ptr(workspace),
+                                    ws_bytes, _ptr(dq_scratch),
+                                    dq_scratch.numel() * dq_scratch.element_size(),
+                                    _ptr(dev_status), _stream(stream, q_t.device)), call)
+    return dq_scratch
 
 
 def step_q8_scratch_bytes(rows: int, n_req: int, heads: int) -> int:

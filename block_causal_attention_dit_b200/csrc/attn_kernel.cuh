@@ -133,6 +133,11 @@ struct AttnParams {
   // the K scale multiplies the scores of cache keys, the V scale their P.
   int32_t k_fp8;
   int32_t v_fp8;
+  // The per-head scales apply to the cache tensor (e4m3 values): 1 for an e4m3
+  // tensor, whether its tiles arrive as codes (k_fp8 / v_fp8) or were expanded to
+  // bf16 beforehand (bca_step_attend_dq).
+  int32_t k_scaled;
+  int32_t v_scaled;
   const float* k_scale[MAXR];
   const float* v_scale[MAXR];
   const float* q_scale[MAXR];  // e4m3-Q mode: [H] scales of request i's Q codes
@@ -725,14 +730,14 @@ __device__ void softmax_role(const AttnParams<MAXR>& p, int w, uint32_t sbase, u
     // by v_scale (folded into the exp2 bias; the row sum keeps the unscaled P).
     float sl2_cache = p.scale_log2, lg_vs = 0.f, inv_vs = 1.f;
     if (!prefill) {
-      if (!BCA_CHECK(p.dev_status, c.req < p.n_req && (!p.k_fp8 || p.k_scale[c.req]) &&
-                                       (!p.v_fp8 || p.v_scale[c.req]), 4))
+      if (!BCA_CHECK(p.dev_status, c.req < p.n_req && (!p.k_scaled || p.k_scale[c.req]) &&
+                                       (!p.v_scaled || p.v_scale[c.req]), 4))
         return;
-      if (p.k_fp8) sl2_cache *= __ldg(p.k_scale[c.req] + c.h);
+      if (p.k_scaled) sl2_cache *= __ldg(p.k_scale[c.req] + c.h);
       // e4m3-Q mode: cached keys' scores are Q8 K8^T, so Q's scale joins K's.
       if (kQ8 && BCA_CHECK(p.dev_status, p.q_scale[c.req] != nullptr, 7))
         sl2_cache *= __ldg(p.q_scale[c.req] + c.h);
-      if (p.v_fp8) {
+      if (p.v_scaled) {
         const float vs = __ldg(p.v_scale[c.req] + c.h);
         lg_vs = __log2f(vs);
         inv_vs = 1.0f / vs;

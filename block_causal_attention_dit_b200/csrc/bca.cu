@@ -27,6 +27,7 @@
 
 #include "../../include/bca.h"
 #include "attn_kernel.cuh"
+#include "kv_expand_kernel.cuh"
 #include "kv_store_kernel.cuh"
 #include "qk_norm_rope_kernel.cuh"
 #include "qkv_proj_kernel.cuh"
@@ -557,12 +558,32 @@ size_t bca_step_q8_scratch_bytes(int64_t rows, int32_t n_req, int32_t heads) {
   return q8_codes_bytes(rows, heads) + q8_table_bytes(n_req, heads);
 }
 
-// The cached step; with q8_scratch, in e4m3-Q mode (bca_step_attend_q8).
+// Bytes of the bf16 expansion of one e4m3 cache tensor (rows x heads x 128).
+static size_t dq_tensor_bytes(int32_t rows, int32_t heads) {
+  return round256(static_cast<size_t>(rows) * static_cast<size_t>(heads) * 128 * 2);
+}
+
+size_t bca_step_dq_scratch_bytes(const bca_kv_slot* slots, int32_t n_req) {
+  if (!slots || n_req < 1 || n_req > BCA_MAX_BATCH) return 0;
+  size_t n = 0;
+  for (int r = 0; r < n_req; ++r) {
+    const bca_kv_slot& s = slots[r];
+    if (s.n_tokens < 0 || s.num_heads < 1 || !dtype_valid(s.dtype)) return 0;
+    if (k_is_fp8(s.dtype)) n += dq_tensor_bytes(s.n_tokens, s.num_heads);
+    if (v_is_fp8(s.dtype)) n += dq_tensor_bytes(s.n_tokens, s.num_heads);
+  }
+  return n;
+}
+
+// The cached step; with q8_scratch, in e4m3-Q mode (bca_step_attend_q8); with dq, the
+// e4m3 cache tensors are first expanded to bf16 in dq_scratch (bca_step_attend_dq).
 static bca_status step_attend_impl(const void* q_t, const void* k_t, const void* v_t, void* o_t,
                                    const int32_t* cu, const bca_kv_slot* slots, int32_t n_req,
                                    int32_t heads, int32_t head_dim, float scale, void* workspace,
                                    size_t workspace_bytes, bool q8, void* q8_scratch,
-                                   size_t q8_bytes, int32_t* dev_status, void* stream) {
+                                   size_t q8_bytes, int32_t* dev_status, void* stream,
+                                   bool dq = false, void* dq_scratch = nullptr,
+                                   size_t dq_bytes = 0) {
   if (workspace && (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return BCA_ERR_INVALID_ARG;
   const size_t ws_chunks = workspace ? workspace_bytes / bca::kChunkBytes : 0;
   if (!cu || !slots) return BCA_ERR_INVALID_ARG;
@@ -592,8 +613,58 @@ static bca_status step_attend_impl(const void* q_t, const void* k_t, const void*
       return BCA_ERR_INVALID_ARG;
     if (q8_bytes < bca_step_q8_scratch_bytes(total, n_req, heads)) return BCA_ERR_CAPACITY;
   }
+  std::vector<void*> dq_k(n_req, nullptr), dq_v(n_req, nullptr);
+  if (dq) {
+    if (slots[0].dtype == BCA_KV_BF16) return BCA_ERR_UNSUPPORTED;
+    if (!dq_scratch || (reinterpret_cast<uintptr_t>(dq_scratch) & 255u) != 0)
+      return BCA_ERR_INVALID_ARG;
+    for (int r = 0; r < n_req; ++r)  // 32-bit chunk indices in the expansion kernel
+      if (static_cast<int64_t>(slots[r].n_tokens) * heads * 8 >= (int64_t{1} << 32))
+        return BCA_ERR_UNSUPPORTED;
+    if (dq_bytes < bca_step_dq_scratch_bytes(slots, n_req)) return BCA_ERR_CAPACITY;
+    char* b = static_cast<char*>(dq_scratch);
+    for (int r = 0; r < n_req; ++r) {
+      if (k_is_fp8(slots[r].dtype)) {
+        dq_k[r] = b;
+        b += dq_tensor_bytes(slots[r].n_tokens, heads);
+      }
+      if (v_is_fp8(slots[r].dtype)) {
+        dq_v[r] = b;
+        b += dq_tensor_bytes(slots[r].n_tokens, heads);
+      }
+    }
+  }
   if (total == 0) return BCA_OK;
   const int32_t dt = slots[0].dtype;
+  if (dq) {
+    // Expand every e4m3 cache tensor that a request with target rows reads.
+    bca::ExpandParams ep;
+    std::memset(&ep, 0, sizeof(ep));
+    int n = 0, max_chunks = 0;
+    for (int r = 0; r < n_req; ++r) {
+      if (cu[r + 1] == cu[r] || slots[r].n_tokens == 0) continue;
+      for (int kv = 0; kv < 2; ++kv) {
+        void* d = kv ? dq_v[r] : dq_k[r];
+        if (!d) continue;
+        bca::ExpandTensor& t = ep.t[n++];
+        t.src = static_cast<const uint8_t*>(kv ? slots[r].v : slots[r].k);
+        t.dst = static_cast<uint16_t*>(d);
+        t.cap = slots[r].cap_tokens;
+        t.rows = slots[r].n_tokens;
+        t.heads = heads;
+        max_chunks = std::max(max_chunks, slots[r].n_tokens * heads * 8);
+      }
+    }
+    ep.n_tensors = n;
+    if (n > 0) {
+      const int sms = std::max(sm_count(), 1);
+      const int bx = std::max(1, std::min((max_chunks + bca::kExpandThreads - 1) / bca::kExpandThreads,
+                                          std::max(1, 8 * sms / n)));
+      bca::kv_expand_kernel<<<dim3(bx, n), bca::kExpandThreads, 0,
+                              static_cast<cudaStream_t>(stream)>>>(ep);
+      if (cudaGetLastError() != cudaSuccess) return BCA_ERR_CUDA;
+    }
+  }
   if (!get_encode()) return BCA_ERR_CUDA;
   uint8_t* q8_codes = static_cast<uint8_t*>(q8_scratch);
   float* q8_scale = q8 ? reinterpret_cast<float*>(q8_codes + q8_codes_bytes(total, heads)) : nullptr;
@@ -635,18 +706,25 @@ static bca_status step_attend_impl(const void* q_t, const void* k_t, const void*
     p.mode = bca::kModeStep;
     p.scale_log2 = scale * 1.4426950408889634f;
     p.n_req = nr;
-    p.k_fp8 = k_is_fp8(dt) ? 1 : 0;
-    p.v_fp8 = v_is_fp8(dt) ? 1 : 0;
+    p.k_fp8 = k_is_fp8(dt) && !dq ? 1 : 0;
+    p.v_fp8 = v_is_fp8(dt) && !dq ? 1 : 0;
+    p.k_scaled = k_is_fp8(dt) ? 1 : 0;
+    p.v_scaled = v_is_fp8(dt) ? 1 : 0;
     int units = 0;
     for (int i = 0; i < nr; ++i) {
       const int r = order[i];
       const bca_kv_slot& sl = slots[r];
-      const bool kok = k_is_fp8(dt)
-                           ? map_cache_e4m3(&p.tm_kc[i], sl.k, sl.n_tokens, sl.cap_tokens, heads)
-                           : map_cache_bf16(&p.tm_kc[i], sl.k, sl.n_tokens, sl.cap_tokens, heads);
-      const bool vok = v_is_fp8(dt)
-                           ? map_cache_e4m3(&p.tm_vc[i], sl.v, sl.n_tokens, sl.cap_tokens, heads)
-                           : map_cache_bf16(&p.tm_vc[i], sl.v, sl.n_tokens, sl.cap_tokens, heads);
+      // dq: the expanded tensors, [H, n_tokens, 128] bf16
+      const bool kok =
+          p.k_fp8 ? map_cache_e4m3(&p.tm_kc[i], sl.k, sl.n_tokens, sl.cap_tokens, heads)
+          : dq_k[r] && sl.n_tokens > 0
+              ? map_cache_bf16(&p.tm_kc[i], dq_k[r], sl.n_tokens, sl.n_tokens, heads)
+                    : map_cache_bf16(&p.tm_kc[i], sl.k, sl.n_tokens, sl.cap_tokens, heads);
+      const bool vok =
+          p.v_fp8 ? map_cache_e4m3(&p.tm_vc[i], sl.v, sl.n_tokens, sl.cap_tokens, heads)
+          : dq_v[r] && sl.n_tokens > 0
+              ? map_cache_bf16(&p.tm_vc[i], dq_v[r], sl.n_tokens, sl.n_tokens, heads)
+                    : map_cache_bf16(&p.tm_vc[i], sl.v, sl.n_tokens, sl.cap_tokens, heads);
       if (!kok || !vok) return BCA_ERR_CUDA;
       p.k_scale[i] = sl.k_scale;
       p.v_scale[i] = sl.v_scale;
@@ -692,6 +770,16 @@ bca_status bca_step_attend(const void* q_t, const void* k_t, const void* v_t, vo
                            size_t workspace_bytes, int32_t* dev_status, void* stream) {
   return step_attend_impl(q_t, k_t, v_t, o_t, cu, slots, n_req, heads, head_dim, scale, workspace,
                           workspace_bytes, false, nullptr, 0, dev_status, stream);
+}
+
+bca_status bca_step_attend_dq(const void* q_t, const void* k_t, const void* v_t, void* o_t,
+                              const int32_t* cu, const bca_kv_slot* slots, int32_t n_req,
+                              int32_t heads, int32_t head_dim, float scale, void* workspace,
+                              size_t workspace_bytes, void* dq_scratch, size_t dq_scratch_bytes,
+                              int32_t* dev_status, void* stream) {
+  return step_attend_impl(q_t, k_t, v_t, o_t, cu, slots, n_req, heads, head_dim, scale, workspace,
+                          workspace_bytes, false, nullptr, 0, dev_status, stream, true, dq_scratch,
+                          dq_scratch_bytes);
 }
 
 bca_status bca_step_attend_q8(const void* q_t, const void* k_t, const void* v_t, void* o_t,

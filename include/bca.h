@@ -225,6 +225,34 @@ bca_status bca_step_attend_q8(const void* q_t, const void* k_t, const void* v_t,
                               size_t workspace_bytes, void* q8_scratch, size_t q8_scratch_bytes,
                               int32_t* dev_status, void* stream);
 
+/* The cached step of bca_step_attend over e4m3 slots ("fp8_v" or "fp8"), with each
+ * e4m3 cache tensor a request reads first expanded, once per call, into a bf16 copy
+ * in dq_scratch (one HBM-bound kernel: read 1 byte, write 2 per value; exact, the
+ * per-head scale is not applied) -- instead of every CTA that visits a cached tile
+ * converting it in shared memory (a tile is visited by each of the request's
+ * Q-tile pairs, 16 for a 4096-row target).  The attention then reads bf16 tiles
+ * and folds the scales in as bca_step_attend does, so the result equals
+ * bca_step_attend's on the same slots bit for bit.  The slots keep their e4m3
+ * bytes: the expansion is transient, one layer's worth at a time.
+ *   dq_scratch,
+ *   dq_scratch_bytes : device, 256-byte aligned, caller-owned, at least
+ *                      bca_step_dq_scratch_bytes(slots, n_req); calls sharing it
+ *                      must not overlap.
+ * Other arguments, results and errors: as bca_step_attend, plus
+ * BCA_ERR_UNSUPPORTED for bf16 slots (nothing to expand) or a slot whose
+ * n_tokens x heads reaches 2^29, BCA_ERR_INVALID_ARG for a NULL or misaligned
+ * scratch, BCA_ERR_CAPACITY for a small one. */
+bca_status bca_step_attend_dq(const void* q_t, const void* k_t, const void* v_t, void* o_t,
+                              const int32_t* cu_target, const bca_kv_slot* slots, int32_t n_req,
+                              int32_t heads, int32_t head_dim, float scale, void* workspace,
+                              size_t workspace_bytes, void* dq_scratch, size_t dq_scratch_bytes,
+                              int32_t* dev_status, void* stream);
+
+/* Bytes of bca_step_attend_dq's scratch for these slots (their n_tokens and dtypes):
+ * per request, a bf16 [heads, n_tokens, 128] tensor for each of its e4m3 K and V,
+ * each 256-byte aligned.  0 for invalid arguments. */
+size_t bca_step_dq_scratch_bytes(const bca_kv_slot* slots, int32_t n_req);
+
 /* Bytes of bca_step_attend_q8's scratch for `rows` packed target rows of n_req
  * requests (0 for arguments out of range). */
 size_t bca_step_q8_scratch_bytes(int64_t rows, int32_t n_req, int32_t heads);

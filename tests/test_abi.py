@@ -285,3 +285,29 @@ def test_qkv_project_argument_errors(L):
     assert call(w=ctypes.c_void_p((1 << 24) + 8)) == 1  # misaligned
     assert call(cos=None) == 1
     assert call(rows=0, x=None) == 0  # nothing to do, nothing checked
+
+
+def test_step_attend_dq_argument_errors(L):
+    """bca_step_attend_dq: e4m3 slots, a non-NULL 256-byte aligned scratch of at
+    least bca_step_dq_scratch_bytes (per request: bf16 [H, n_tokens, 128] for each e4m3
+    tensor, 256-byte aligned), all checked before anything is enqueued."""
+    H = 2
+    fp8 = (bca.SlotStruct * 2)(_slot(L, dt=2, n=10), _slot(L, dt=2, n=20))
+    fp8v = (bca.SlotStruct * 2)(_slot(L, dt=1, n=10), _slot(L, dt=1, n=20))
+    bf = (bca.SlotStruct * 2)(_slot(L, n=10), _slot(L, n=20))
+    r256 = lambda n: (n + 255) // 256 * 256
+    need = L.bca_step_dq_scratch_bytes(fp8, 2)
+    assert need == 2 * r256(10 * H * 256) + 2 * r256(20 * H * 256)
+    assert L.bca_step_dq_scratch_bytes(fp8v, 2) == r256(10 * H * 256) + r256(20 * H * 256)
+    assert L.bca_step_dq_scratch_bytes(bf, 2) == 0
+    assert L.bca_step_dq_scratch_bytes(None, 2) == 0
+    assert L.bca_step_dq_scratch_bytes(fp8, 0) == 0
+    cu = (ctypes.c_int32 * 3)(0, 100, 228)
+    scratch = ctypes.c_void_p(1 << 28)
+    call = lambda **kw: L.bca_step_attend_dq(
+        FAKE, FAKE, FAKE, FAKE, cu, kw.get("arr", fp8), 2, H, 128, 0.1, None, 0,
+        kw.get("scratch", scratch), kw.get("bytes", need), None, None)
+    assert call(arr=bf) == 2
+    assert call(scratch=None) == 1
+    assert call(scratch=ctypes.c_void_p((1 << 28) + 16)) == 1
+    assert call(bytes=need - 1) == 3
