@@ -296,9 +296,37 @@ struct StoreJob {
   bool quant;
 };
 
+// Clusters of the store kernel that can be resident at once on the current device
+// (cached per device; the GPCs' sizes decide how many 8-CTA clusters fit).
+int store_max_clusters() {
+  static std::mutex mu;
+  static std::vector<int> n;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 1;
+  std::lock_guard<std::mutex> lk(mu);
+  if (n.size() <= static_cast<size_t>(dev)) n.resize(dev + 1, 0);
+  if (!n[dev]) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(bca::kStoreCluster));
+    cfg.blockDim = dim3(bca::kStoreThreads);
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = bca::kStoreCluster;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int c = 0;
+    if (cudaOccupancyMaxActiveClusters(&c, bca::kv_store_kernel, &cfg) != cudaSuccess || c < 1)
+      c = std::max(1, sm_count() / bca::kStoreCluster);
+    n[dev] = c;
+  }
+  return n[dev];
+}
+
 // One launch of bca::kv_store_kernel over every job: tensors with the most rows
-// first, clusters of bca::kStoreCluster CTAs, as many clusters as fit one CTA per SM
-// (so that few columns are in flight and the encode pass re-reads them from L2).
+// first, clusters of bca::kStoreCluster CTAs, as many as are resident at once (so
+// that few columns are in flight and the encode pass re-reads them from L2).
 bca_status launch_store(std::vector<StoreJob> jobs, int32_t* dev_status, cudaStream_t stream) {
   jobs.erase(std::remove_if(jobs.begin(), jobs.end(), [](const StoreJob& j) { return j.rows == 0; }),
              jobs.end());
@@ -325,8 +353,7 @@ bca_status launch_store(std::vector<StoreJob> jobs, int32_t* dev_status, cudaStr
   p.n_tensors = static_cast<int32_t>(jobs.size());
   p.n_cols = cols;
   p.dev_status = dev_status;
-  const int sms = std::max(sm_count(), 1);
-  const int clusters = std::max(1, std::min(cols, sms / bca::kStoreCluster));
+  const int clusters = std::max(1, std::min(cols, store_max_clusters()));
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(clusters * bca::kStoreCluster));
   cfg.blockDim = dim3(bca::kStoreThreads);

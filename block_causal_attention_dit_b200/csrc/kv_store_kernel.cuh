@@ -60,7 +60,9 @@ __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w 
 // columns (one per head: rows [0, rows_i) of that head), numbered from col0_i.  A
 // cluster of kStoreCluster CTAs takes whole columns (cluster c: columns c, c +
 // #clusters, ...; the host lists tensors with the most rows first), and its CTAs
-// split the column's rows evenly.
+// split the column's rows evenly.  Only as many clusters are launched as can be
+// resident at once (the cluster loop is persistent; a cluster that had to wait for
+// another to finish would run its whole share of columns after it).
 //  * bf16 column: a copy.
 //  * e4m3 column: pass 1 reads the CTA's rows for the absmax; the CTAs' partial
 //    maxima meet in every CTA's shared memory (distributed shared memory stores,
@@ -70,7 +72,9 @@ __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w 
 //    as there are clusters, ~18 on B200), and writes the codes with streaming
 //    stores.  HBM then sees each source byte read once and each code written once.
 // Every thread owns one 16-byte chunk (8 channels) of a row; 16 threads cover a
-// 256-byte head row, kStoreUnroll rows per thread are loaded before any is used.
+// 256-byte head row.  A thread takes its rows kStoreUnroll at a time, and loads the
+// next kStoreUnroll (a second register buffer) before it uses the current ones, so
+// that ~128 KiB per SM stay in flight.
 // A non-finite value in an e4m3 column makes its amax Inf or NaN: the column's
 // codes and scale are then meaningless and BCA_ERR_NONFINITE is written to
 // *dev_status (the inputs must be finite).
@@ -153,7 +157,8 @@ __global__ void __launch_bounds__(kStoreThreads, 1)
   __shared__ unsigned s_warp[kStoreThreads / 32];
   const uint32_t crank = cluster_rank(), csize = cluster_size();
   const int tid = threadIdx.x, lane16 = tid & 15, rslot = tid >> 4;
-  constexpr int kStep = kStoreRowsPerSweep * kStoreUnroll;
+  constexpr int U = kStoreUnroll;
+  constexpr int kStep = kStoreRowsPerSweep * U;
   int ti = 0, nq = 0;
   for (int col = static_cast<int>(cluster_index()); col < p.n_cols;
        col += static_cast<int>(cluster_count())) {
@@ -165,39 +170,62 @@ __global__ void __launch_bounds__(kStoreThreads, 1)
     const uint16_t* src = T.src + static_cast<int64_t>(h) * 128 + lane16 * 8;
     const int64_t rs = T.row_stride;
     const int64_t drow0 = static_cast<int64_t>(h) * T.head_stride;
+    // U rows of this thread starting at row `base` (rows >= r1 read as zero).
+    auto load = [&](uint4 (&v)[U], int base) {
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int t = base + u * kStoreRowsPerSweep;
+        v[u] = t < r1 ? __ldcs(reinterpret_cast<const uint4*>(src + t * rs))
+                      : make_uint4(0u, 0u, 0u, 0u);
+      }
+    };
+    // Rows are visited in batches of U per thread; the next batch is loaded before the
+    // current one is used (two register buffers), so loads stay in flight.
+    uint4 va[U], vb[U];
     if (!T.quant) {
       uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(T.dst) + drow0 * 128) + lane16;
-      for (int tb = r0 + rslot; tb < r1; tb += kStep) {
-        uint4 v[kStoreUnroll];
+      auto put = [&](const uint4 (&v)[U], int base) {
 #pragma unroll
-        for (int u = 0; u < kStoreUnroll; ++u) {
-          const int t = tb + u * kStoreRowsPerSweep;
-          if (t < r1) v[u] = __ldcs(reinterpret_cast<const uint4*>(src + t * rs));
-        }
-#pragma unroll
-        for (int u = 0; u < kStoreUnroll; ++u) {
-          const int t = tb + u * kStoreRowsPerSweep;
+        for (int u = 0; u < U; ++u) {
+          const int t = base + u * kStoreRowsPerSweep;
           if (t < r1) __stcs(dst + static_cast<int64_t>(t) * 16, v[u]);
         }
+      };
+      int tb = r0 + rslot;
+      if (tb < r1) load(va, tb);
+      while (tb < r1) {
+        if (tb + kStep < r1) load(vb, tb + kStep);
+        put(va, tb);
+        tb += kStep;
+        if (tb >= r1) break;
+        if (tb + kStep < r1) load(va, tb + kStep);
+        put(vb, tb);
+        tb += kStep;
       }
       continue;
     }
     // Pass 1: absmax of this CTA's rows, as bf16 magnitude bits.
     uint32_t m = 0;
-    for (int tb = r0 + rslot; tb < r1; tb += kStep) {
-      uint4 v[kStoreUnroll];
+    auto amax = [&](const uint4 (&v)[U]) {
 #pragma unroll
-      for (int u = 0; u < kStoreUnroll; ++u) {
-        const int t = tb + u * kStoreRowsPerSweep;
-        v[u] = t < r1 ? __ldg(reinterpret_cast<const uint4*>(src + t * rs))
-                      : make_uint4(0u, 0u, 0u, 0u);
-      }
-#pragma unroll
-      for (int u = 0; u < kStoreUnroll; ++u) {
+      for (int u = 0; u < U; ++u) {
         m = max_abs_bf16x2(m, v[u].x);
         m = max_abs_bf16x2(m, v[u].y);
         m = max_abs_bf16x2(m, v[u].z);
         m = max_abs_bf16x2(m, v[u].w);
+      }
+    };
+    {
+      int tb = r0 + rslot;
+      if (tb < r1) load(va, tb);
+      while (tb < r1) {
+        if (tb + kStep < r1) load(vb, tb + kStep);
+        amax(va);
+        tb += kStep;
+        if (tb >= r1) break;
+        if (tb + kStep < r1) load(va, tb + kStep);
+        amax(vb);
+        tb += kStep;
       }
     }
 #pragma unroll
@@ -214,32 +242,39 @@ __global__ void __launch_bounds__(kStoreThreads, 1)
       }
     }
     cluster_sync();
-    uint32_t amax = 0;
-    for (uint32_t q = 0; q < csize; ++q) amax = max(amax, s_part[nq & 1][q]);
+    uint32_t amax_bits = 0;
+    for (uint32_t q = 0; q < csize; ++q) amax_bits = max(amax_bits, s_part[nq & 1][q]);
     ++nq;
-    const float s = scale_from_amax_bits(amax);
+    const float s = scale_from_amax_bits(amax_bits);
     if (crank == 0 && tid == 0) {
       T.scale[h] = s;
-      if (amax >= 0x7F80u && p.dev_status)
+      if (amax_bits >= 0x7F80u && p.dev_status)
         atomicExch(p.dev_status, static_cast<int32_t>(BCA_ERR_NONFINITE));
     }
     const float y = __frcp_rn(s);
-    const bool fast = amax >= kFastDivMinBits;
-    // Pass 2: the same rows, last-read first; codes with streaming stores.
+    const bool fast = amax_bits >= kFastDivMinBits;
+    // Pass 2: the same rows, batches in reverse order (the last read still in L2);
+    // codes with streaming stores.
     uint2* dst = reinterpret_cast<uint2*>(static_cast<uint8_t*>(T.dst) + drow0 * 128) + lane16;
-    const int n = r1 - r0;
-    const int last = r0 + (n > 0 ? ((n - 1 - rslot) / kStep) * kStep : 0) + rslot;
-    for (int tb = last; tb >= r0 && n > rslot; tb -= kStep) {
-      uint4 v[kStoreUnroll];
+    auto enc = [&](const uint4 (&v)[U], int base) {
 #pragma unroll
-      for (int u = 0; u < kStoreUnroll; ++u) {
-        const int t = tb + u * kStoreRowsPerSweep;
-        if (t < r1) v[u] = __ldcs(reinterpret_cast<const uint4*>(src + t * rs));
-      }
-#pragma unroll
-      for (int u = 0; u < kStoreUnroll; ++u) {
-        const int t = tb + u * kStoreRowsPerSweep;
+      for (int u = 0; u < U; ++u) {
+        const int t = base + u * kStoreRowsPerSweep;
         if (t < r1) __stcs(dst + static_cast<int64_t>(t) * 16, encode_chunk(v[u], s, y, fast));
+      }
+    };
+    const int n = r1 - r0;
+    if (n > rslot) {
+      int tb = r0 + ((n - 1 - rslot) / kStep) * kStep + rslot;
+      load(va, tb);
+      while (tb >= r0) {
+        if (tb - kStep >= r0) load(vb, tb - kStep);
+        enc(va, tb);
+        tb -= kStep;
+        if (tb < r0) break;
+        if (tb - kStep >= r0) load(va, tb - kStep);
+        enc(vb, tb);
+        tb -= kStep;
       }
     }
   }

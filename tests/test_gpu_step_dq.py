@@ -24,8 +24,9 @@ def _batch(shapes, H, mode, device, seed):
     reqs = []
     for i, (T, P) in enumerate(shapes):
         q, k, v = (randn_bf16((T, H, 128), seed + 10 * i + t, device) for t in range(3))
-        pk, pv = (randn_bf16((max(P, 1), H, 128), seed + 10 * i + 5 + t, device) * (1 + i)
-                  for t in range(2))
+        # K scaled per request (different per-head scales and sharper softmax rows)
+        pk = randn_bf16((max(P, 1), H, 128), seed + 10 * i + 5, device) * (1 + i)
+        pv = randn_bf16((max(P, 1), H, 128), seed + 10 * i + 6, device)
         slot = bca.KVSlot(P + 7, H, mode)
         slot.buffer.fill_(0xFF)  # NaN codes past the prefix: never read
         bca.kv_store(pk, pv, P, slot, epoch=1)
