@@ -101,11 +101,11 @@ def prefill_split_launches(req, H, sms) -> int:
 # dram__bytes_write.sum) from one ncu capture of the T2I cached step, valid only for
 # the kernel sources it was taken from (their sha256 below); any later change
 # reports null instead.
-ATTN_TRAFFIC = {"bytes_per_launch": 109.24e6 + 15.60e6, "workload": 1,
+ATTN_TRAFFIC = {"bytes_per_launch": 109.28e6 + 15.53e6, "workload": 1,
                 "sources": {"block_causal_attention_dit_b200/csrc/attn_kernel.cuh":
-                            "62fa4d412f679f5ec6ff71e4bdc882816523bcb78718570f549bc38ce9976a9f",
+                            "f6b62b40fda38fb3fba0d8d3b9a2f17c70ca61acffdea9c8ba9f7b58d40c29e9",
                             "block_causal_attention_dit_b200/csrc/ptx.cuh":
-                            "5e3e72b92fd39e9479a83a124160be0c84fbd8c7f66acf214212d88f2723b8c3"}}
+                            "cf462dedfbd63f8e2e730a546a5db830b04e5240296b7864a033c80e029dd256"}}
 
 
 def measured_traffic(workload: int):
