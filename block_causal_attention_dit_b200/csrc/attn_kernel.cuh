@@ -756,9 +756,7 @@ __device__ void softmax_role(const AttnParams<MAXR>& p, int w, uint32_t sbase, u
       const bool trw = lane == 0 && warp > 0;
       if (tr) BCA_TRACE_AT(p, ns, 5 + 5 * w);
       uint32_t r[128];
-#pragma unroll
-      for (int cc = 0; cc < 4; ++cc)
-        tmem_ld_32x32b_x32(tS + 32 * cc, *reinterpret_cast<uint32_t(*)[32]>(&r[32 * cc]));
+      tmem_ld_32x32b_x128(tS, r);
       tmem_wait_ld();
       if (tr) BCA_TRACE_AT(p, ns, 6 + 5 * w);
       int valid, key_base;
