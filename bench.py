@@ -568,7 +568,8 @@ def config_leg(index: int, device, peaks, reps: int = 3):
     """One layer of workload `index` on its own: the prefill of every request
     (bca_prefill with the workspace, attention only), the prefix store of all
     requests (one bca_kv_store_batch launch) and one cached step of all requests
-    (bca_step_attend), each timed with CUDA events around its enqueues.  Two cached-
+    (bca_step_attend; for an e4m3 cache bca_step_attend_dq, the in-kernel conversion
+    timed beside it), each timed with CUDA events around its enqueues.  Two cached-
     step input sets alternate (larger than L2 together).  The 40-step projection is
     32 layers x (prefill + store) + 32 x 39 cached steps from these timings."""
     import torch
@@ -602,7 +603,19 @@ def config_leg(index: int, device, peaks, reps: int = 3):
         epoch[0] += 1
         bca.kv_store_batch(items, epoch[0], dev_status=status)
 
+    e4m3 = wl.kv_dtype != "bf16"
+    dq_scratch = bca.step_dq_scratch(slots, device) if e4m3 else None
+
     def step(n):
+        q, k, v = sets[n % 2]
+        if e4m3:  # the cache expanded to bf16 once per call (bit-identical results)
+            bca.step_attend_dq(q, k, v, o_step, cu, slots, wl.scale, dq_scratch=dq_scratch,
+                               workspace=ws, dev_status=status)
+        else:
+            bca.step_attend(q, k, v, o_step, cu, slots, wl.scale, workspace=ws,
+                            dev_status=status)
+
+    def step_conv(n):  # e4m3 tiles converted in the attention kernel instead
         q, k, v = sets[n % 2]
         bca.step_attend(q, k, v, o_step, cu, slots, wl.scale, workspace=ws, dev_status=status)
 
@@ -624,6 +637,7 @@ def config_leg(index: int, device, peaks, reps: int = 3):
     p_ms = time_it(lambda i: prefill(), reps)
     s_ms = time_it(lambda i: store(), reps)
     c_ms = time_it(step, 2 * reps)
+    cv_ms = time_it(step_conv, 2 * reps) if e4m3 else None
     if int(status.item()) != 0:
         raise RuntimeError(f"device status {int(status.item())} (workload {index})")
     pk_sus = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
@@ -643,7 +657,10 @@ def config_leg(index: int, device, peaks, reps: int = 3):
             "prefill_frac_sustained": t_pre / pk_sus,
             "store_ms_per_layer": s_ms, "store_gbs": st_bytes / (s_ms / 1e3) / 1e9,
             "store_frac_hbm": st_bytes / (s_ms / 1e3) / 1e9 / hbm,
+            "cached_step_call": "bca_step_attend_dq" if e4m3 else "bca_step_attend",
             "cached_step_ms_per_layer": c_ms, "cached_step_tflops": t_step,
+            "cached_step_in_kernel_conversion_tflops":
+                f_step / (cv_ms / 1e3) / 1e12 if cv_ms else None,
             "cached_step_frac_sustained": t_step / pk_sus,
             "cached_step_frac_burst": t_step / pk_burst,
             "projected_ms_per_40step_attn": total_ms,
