@@ -309,6 +309,10 @@ int store_max_clusters() {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(bca::kStoreCluster));
     cfg.blockDim = dim3(bca::kStoreThreads);
+    cfg.dynamicSmemBytes = bca::kStoreRingBytes;
+    if (cudaFuncSetAttribute(bca::kv_store_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             bca::kStoreRingBytes) != cudaSuccess)
+      return 0;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = bca::kStoreCluster;
@@ -321,7 +325,7 @@ int store_max_clusters() {
       c = std::max(1, sm_count() / bca::kStoreCluster);
     n[dev] = c;
   }
-  return n[dev];
+  return n[dev];  // 0 only if the kernel attribute could not be set
 }
 
 // One launch of bca::kv_store_kernel over every job: tensors with the most rows
@@ -353,11 +357,13 @@ bca_status launch_store(std::vector<StoreJob> jobs, int32_t* dev_status, cudaStr
   p.n_tensors = static_cast<int32_t>(jobs.size());
   p.n_cols = cols;
   p.dev_status = dev_status;
-  const int clusters = std::max(1, std::min(cols, store_max_clusters()));
+  const int max_clusters = store_max_clusters();
+  if (max_clusters < 1) return BCA_ERR_CUDA;
+  const int clusters = std::max(1, std::min(cols, max_clusters));
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(clusters * bca::kStoreCluster));
   cfg.blockDim = dim3(bca::kStoreThreads);
-  cfg.dynamicSmemBytes = 0;
+  cfg.dynamicSmemBytes = bca::kStoreRingBytes;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;

@@ -72,9 +72,9 @@ __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w 
 //    as there are clusters, ~18 on B200), and writes the codes with streaming
 //    stores.  HBM then sees each source byte read once and each code written once.
 // Every thread owns one 16-byte chunk (8 channels) of a row; 16 threads cover a
-// 256-byte head row.  A thread takes its rows kStoreUnroll at a time, and loads the
-// next kStoreUnroll (a second register buffer) before it uses the current ones, so
-// that ~128 KiB per SM stay in flight.
+// 256-byte head row.  A thread streams its rows through its own ring of
+// kStoreRing 16-byte slots in shared memory filled by cp.async (128 KiB per CTA in
+// flight without holding registers).
 // A non-finite value in an e4m3 column makes its amax Inf or NaN: the column's
 // codes and scale are then meaningless and BCA_ERR_NONFINITE is written to
 // *dev_status (the inputs must be finite).
@@ -94,7 +94,8 @@ struct StoreTensor {
 constexpr int kMaxStoreTensors = 2 * BCA_MAX_BATCH;
 constexpr int kStoreThreads = 512;
 constexpr int kStoreCluster = 8;
-constexpr int kStoreUnroll = 8;
+constexpr int kStoreRing = 16;  // 16-byte copies in flight per thread
+constexpr int kStoreRingBytes = kStoreRing * kStoreThreads * 16;
 constexpr int kStoreRowsPerSweep = kStoreThreads / 16;
 
 struct StoreParams {
@@ -151,14 +152,51 @@ __device__ __forceinline__ uint2 encode_chunk(const uint4 v, float s, float y, b
   return make_uint2(out[0], out[1]);
 }
 
+// 16-byte asynchronous copy global -> shared (no register staging, L1 bypassed);
+// one commit group per call site.
+__device__ __forceinline__ void cp_async16(uint32_t smem, const void* gmem) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem), "l"(gmem) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+// The rows of one thread, k = 0..n-1 (row first + k * step), streamed through the
+// thread's own ring of kStoreRing 16-byte slots in shared memory: the copy of row
+// k + kStoreRing is issued as soon as row k has been used, so kStoreRing copies per
+// thread (128 KiB per CTA) stay in flight without holding registers.
+template <typename Fn>
+__device__ __forceinline__ void stream_rows(uint32_t ring, const uint16_t* src, int64_t rs,
+                                            int first, int step, int n, Fn&& use) {
+  const uint32_t slot0 = ring + threadIdx.x * 16u;
+#pragma unroll
+  for (int i = 0; i < kStoreRing; ++i) {
+    if (i < n) cp_async16(slot0 + i * (kStoreThreads * 16u), src + (first + i * step) * rs);
+    cp_async_commit();
+  }
+  for (int k = 0; k < n; ++k) {
+    cp_async_wait<kStoreRing - 1>();
+    const uint32_t slot = slot0 + (k % kStoreRing) * (kStoreThreads * 16u);
+    uint4 v;
+    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "r"(slot)
+                 : "memory");
+    use(v, first + k * step);
+    if (k + kStoreRing < n) cp_async16(slot, src + (first + (k + kStoreRing) * step) * rs);
+    cp_async_commit();
+  }
+  cp_async_wait<0>();
+}
+
 __global__ void __launch_bounds__(kStoreThreads, 1)
     kv_store_kernel(const __grid_constant__ StoreParams p) {
+  extern __shared__ __align__(16) uint8_t store_ring[];
   __shared__ unsigned s_part[2][kStoreCluster];  // partial maxima by rank, double-buffered
   __shared__ unsigned s_warp[kStoreThreads / 32];
+  const uint32_t ring = static_cast<uint32_t>(__cvta_generic_to_shared(store_ring));
   const uint32_t crank = cluster_rank(), csize = cluster_size();
   const int tid = threadIdx.x, lane16 = tid & 15, rslot = tid >> 4;
-  constexpr int U = kStoreUnroll;
-  constexpr int kStep = kStoreRowsPerSweep * U;
   int ti = 0, nq = 0;
   for (int col = static_cast<int>(cluster_index()); col < p.n_cols;
        col += static_cast<int>(cluster_count())) {
@@ -170,64 +208,22 @@ __global__ void __launch_bounds__(kStoreThreads, 1)
     const uint16_t* src = T.src + static_cast<int64_t>(h) * 128 + lane16 * 8;
     const int64_t rs = T.row_stride;
     const int64_t drow0 = static_cast<int64_t>(h) * T.head_stride;
-    // U rows of this thread starting at row `base` (rows >= r1 read as zero).
-    auto load = [&](uint4 (&v)[U], int base) {
-#pragma unroll
-      for (int u = 0; u < U; ++u) {
-        const int t = base + u * kStoreRowsPerSweep;
-        v[u] = t < r1 ? __ldcs(reinterpret_cast<const uint4*>(src + t * rs))
-                      : make_uint4(0u, 0u, 0u, 0u);
-      }
-    };
-    // Rows are visited in batches of U per thread; the next batch is loaded before the
-    // current one is used (two register buffers), so loads stay in flight.
-    uint4 va[U], vb[U];
+    // This thread's rows: r0 + rslot + k * kStoreRowsPerSweep, k < n.
+    const int n = r1 - r0 > rslot ? (r1 - r0 - rslot + kStoreRowsPerSweep - 1) / kStoreRowsPerSweep : 0;
     if (!T.quant) {
       uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(T.dst) + drow0 * 128) + lane16;
-      auto put = [&](const uint4 (&v)[U], int base) {
-#pragma unroll
-        for (int u = 0; u < U; ++u) {
-          const int t = base + u * kStoreRowsPerSweep;
-          if (t < r1) __stcs(dst + static_cast<int64_t>(t) * 16, v[u]);
-        }
-      };
-      int tb = r0 + rslot;
-      if (tb < r1) load(va, tb);
-      while (tb < r1) {
-        if (tb + kStep < r1) load(vb, tb + kStep);
-        put(va, tb);
-        tb += kStep;
-        if (tb >= r1) break;
-        if (tb + kStep < r1) load(va, tb + kStep);
-        put(vb, tb);
-        tb += kStep;
-      }
+      stream_rows(ring, src, rs, r0 + rslot, kStoreRowsPerSweep, n,
+                  [&](const uint4& v, int t) { __stcs(dst + static_cast<int64_t>(t) * 16, v); });
       continue;
     }
     // Pass 1: absmax of this CTA's rows, as bf16 magnitude bits.
     uint32_t m = 0;
-    auto amax = [&](const uint4 (&v)[U]) {
-#pragma unroll
-      for (int u = 0; u < U; ++u) {
-        m = max_abs_bf16x2(m, v[u].x);
-        m = max_abs_bf16x2(m, v[u].y);
-        m = max_abs_bf16x2(m, v[u].z);
-        m = max_abs_bf16x2(m, v[u].w);
-      }
-    };
-    {
-      int tb = r0 + rslot;
-      if (tb < r1) load(va, tb);
-      while (tb < r1) {
-        if (tb + kStep < r1) load(vb, tb + kStep);
-        amax(va);
-        tb += kStep;
-        if (tb >= r1) break;
-        if (tb + kStep < r1) load(va, tb + kStep);
-        amax(vb);
-        tb += kStep;
-      }
-    }
+    stream_rows(ring, src, rs, r0 + rslot, kStoreRowsPerSweep, n, [&](const uint4& v, int) {
+      m = max_abs_bf16x2(m, v.x);
+      m = max_abs_bf16x2(m, v.y);
+      m = max_abs_bf16x2(m, v.z);
+      m = max_abs_bf16x2(m, v.w);
+    });
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
     if ((tid & 31) == 0) s_warp[tid >> 5] = m;
@@ -253,30 +249,14 @@ __global__ void __launch_bounds__(kStoreThreads, 1)
     }
     const float y = __frcp_rn(s);
     const bool fast = amax_bits >= kFastDivMinBits;
-    // Pass 2: the same rows, batches in reverse order (the last read still in L2);
-    // codes with streaming stores.
+    // Pass 2: the same rows, last-read first (still in L2); codes with streaming
+    // stores.
     uint2* dst = reinterpret_cast<uint2*>(static_cast<uint8_t*>(T.dst) + drow0 * 128) + lane16;
-    auto enc = [&](const uint4 (&v)[U], int base) {
-#pragma unroll
-      for (int u = 0; u < U; ++u) {
-        const int t = base + u * kStoreRowsPerSweep;
-        if (t < r1) __stcs(dst + static_cast<int64_t>(t) * 16, encode_chunk(v[u], s, y, fast));
-      }
-    };
-    const int n = r1 - r0;
-    if (n > rslot) {
-      int tb = r0 + ((n - 1 - rslot) / kStep) * kStep + rslot;
-      load(va, tb);
-      while (tb >= r0) {
-        if (tb - kStep >= r0) load(vb, tb - kStep);
-        enc(va, tb);
-        tb -= kStep;
-        if (tb < r0) break;
-        if (tb - kStep >= r0) load(va, tb - kStep);
-        enc(vb, tb);
-        tb -= kStep;
-      }
-    }
+    if (n > 0)
+      stream_rows(ring, src, rs, r0 + rslot + (n - 1) * kStoreRowsPerSweep, -kStoreRowsPerSweep,
+                  n, [&](const uint4& v, int t) {
+                    __stcs(dst + static_cast<int64_t>(t) * 16, encode_chunk(v, s, y, fast));
+                  });
   }
   // No CTA leaves while a peer may still store into its shared memory.
   cluster_sync();
