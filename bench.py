@@ -604,12 +604,14 @@ def config_leg(index: int, device, peaks, reps: int = 3):
         bca.kv_store_batch(items, epoch[0], dev_status=status)
 
     e4m3 = wl.kv_dtype != "bf16"
-    dq_scratch = bca.step_dq_scratch(slots, device) if e4m3 else None
+    dq = {}  # bca_step_attend_dq's scratch, sized once the slots are filled
 
     def step(n):
         q, k, v = sets[n % 2]
         if e4m3:  # the cache expanded to bf16 once per call (bit-identical results)
-            bca.step_attend_dq(q, k, v, o_step, cu, slots, wl.scale, dq_scratch=dq_scratch,
+            if "scratch" not in dq:
+                dq["scratch"] = bca.step_dq_scratch(slots, device)
+            bca.step_attend_dq(q, k, v, o_step, cu, slots, wl.scale, dq_scratch=dq["scratch"],
                                workspace=ws, dev_status=status)
         else:
             bca.step_attend(q, k, v, o_step, cu, slots, wl.scale, workspace=ws,

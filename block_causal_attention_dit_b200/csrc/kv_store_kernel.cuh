@@ -67,10 +67,11 @@ __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w 
 //  * e4m3 column: pass 1 reads the CTA's rows for the absmax; the CTAs' partial
 //    maxima meet in every CTA's shared memory (distributed shared memory stores,
 //    then a cluster barrier), so each CTA knows amax_h; rank 0 writes s_h.  Pass 2
-//    reads the same rows again, last-read first, so that they still come from L2
-//    (a cluster's column is at most ~4.4 MB and only as many columns are in flight
-//    as there are clusters, ~18 on B200), and writes the codes with streaming
-//    stores.  HBM then sees each source byte read once and each code written once.
+//    reads the same rows again, last-read first, so that most of them still come
+//    from L2 (a column is at most ~4.4 MB and only as many columns are in flight as
+//    there are resident clusters), and writes the codes with streaming stores.
+//    Measured on the 8-request serving store: clusters of 4 (all SMs busy) beat
+//    clusters of 8 (15 resident, 120 SMs), 0.67 vs 0.72 ms.
 // Every thread owns one 16-byte chunk (8 channels) of a row; 16 threads cover a
 // 256-byte head row.  A thread streams its rows through its own ring of
 // kStoreRing 16-byte slots in shared memory filled by cp.async (128 KiB per CTA in
@@ -93,7 +94,7 @@ struct StoreTensor {
 
 constexpr int kMaxStoreTensors = 2 * BCA_MAX_BATCH;
 constexpr int kStoreThreads = 512;
-constexpr int kStoreCluster = 8;
+constexpr int kStoreCluster = 4;
 constexpr int kStoreRing = 16;  // 16-byte copies in flight per thread
 constexpr int kStoreRingBytes = kStoreRing * kStoreThreads * 16;
 constexpr int kStoreRowsPerSweep = kStoreThreads / 16;
