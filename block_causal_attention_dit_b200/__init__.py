@@ -79,6 +79,7 @@ class StepGraphDesc(ctypes.Structure):
         ("scale", ctypes.c_float), ("workspace", ctypes.c_void_p),
         ("workspace_bytes", ctypes.c_size_t), ("dev_status", ctypes.c_void_p),
         ("q8_scratch", ctypes.c_void_p), ("q8_scratch_bytes", ctypes.c_size_t),
+        ("dq_scratch", ctypes.c_void_p), ("dq_scratch_bytes", ctypes.c_size_t),
     ]
 
 
@@ -598,7 +599,8 @@ def ulysses_unpack(recv, x, n_ranks: int, stream=None):
 
 class StepGraph:
     """The cached-step attention of every layer of one layout as one CUDA graph
-    (with q8_scratch: the e4m3-Q cached step, step_attend_q8, of e4m3 slots).
+    (with q8_scratch: the e4m3-Q cached step, step_attend_q8, of e4m3 slots; with
+    dq_scratch: the expand-once step, step_attend_dq).
 
     q_layers..o_layers: per-layer packed target tensors [sum T_r, H, 128] (bf16,
     CUDA); slots_per_layer: per-layer lists of KVSlot (one per request, in
@@ -607,7 +609,8 @@ class StepGraph:
     graph exists; close() or garbage collection releases it."""
 
     def __init__(self, q_layers, k_layers, v_layers, o_layers, cu_target, slots_per_layer,
-                 scale: float, workspace=None, dev_status=None, q8_scratch=None):
+                 scale: float, workspace=None, dev_status=None, q8_scratch=None,
+                 dq_scratch=None):
         n = len(q_layers)
         assert n == len(k_layers) == len(v_layers) == len(o_layers) == len(slots_per_layer)
         n_req = len(slots_per_layer[0])
@@ -621,9 +624,11 @@ class StepGraph:
         _aux(workspace, call, "workspace", q_layers[0].device)
         _aux(dev_status, call, "dev_status", q_layers[0].device, torch.int32)
         _aux(q8_scratch, call, "q8_scratch", q_layers[0].device)
+        _aux(dq_scratch, call, "dq_scratch", q_layers[0].device)
         _, H, d = q_layers[0].shape
         self._keep = (list(q_layers), list(k_layers), list(v_layers), list(o_layers),
-                      [list(sl) for sl in slots_per_layer], workspace, dev_status, q8_scratch)
+                      [list(sl) for sl in slots_per_layer], workspace, dev_status, q8_scratch,
+                      dq_scratch)
         ptrs = lambda ts: (ctypes.c_void_p * n)(*[t.data_ptr() for t in ts])
         self._q, self._k, self._v, self._o = (ptrs(q_layers), ptrs(k_layers), ptrs(v_layers),
                                               ptrs(o_layers))
@@ -639,7 +644,9 @@ class StepGraph:
             0 if workspace is None else workspace.numel() * workspace.element_size(),
             None if dev_status is None else dev_status.data_ptr(),
             None if q8_scratch is None else q8_scratch.data_ptr(),
-            0 if q8_scratch is None else q8_scratch.numel() * q8_scratch.element_size())
+            0 if q8_scratch is None else q8_scratch.numel() * q8_scratch.element_size(),
+            None if dq_scratch is None else dq_scratch.data_ptr(),
+            0 if dq_scratch is None else dq_scratch.numel() * dq_scratch.element_size())
         self.device = q_layers[0].device
         self._g = ctypes.c_void_p()
         import torch

@@ -23,7 +23,8 @@ LIB_CHECKED = os.path.join(PKG, "libbca_checked.so")
 LIB_TRACE = os.path.join(PKG, "libbca_trace.so")
 SOURCES = [os.path.join(CSRC, "bca.cu")]
 DEPS = SOURCES + [os.path.join(CSRC, f) for f in
-                  ("attn_kernel.cuh", "kv_store_kernel.cuh", "qk_norm_rope_kernel.cuh", "qkv_proj_kernel.cuh",
+                  ("attn_kernel.cuh", "kv_store_kernel.cuh", "kv_expand_kernel.cuh", "qk_norm_rope_kernel.cuh",
+                   "qkv_proj_kernel.cuh",
                    "ulysses_kernel.cuh", "ptx.cuh")] + [
     os.path.join(ROOT, "include", "bca.h")]
 

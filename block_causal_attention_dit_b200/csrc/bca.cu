@@ -961,6 +961,8 @@ extern "C" bca_status bca_step_graph_create(const bca_step_graph_desc* d, bca_st
       !get_encode())
     return BCA_ERR_CUDA;
   const bool q8 = d->q8_scratch != nullptr;
+  const bool dq = d->dq_scratch != nullptr;
+  if (q8 && dq) return BCA_ERR_INVALID_ARG;
   if (q8 && (!prepare_attn<1, true>() || !prepare_attn<8, true>() || !prepare_attn<64, true>()))
     return BCA_ERR_CUDA;
   cudaStream_t cs = nullptr;
@@ -976,7 +978,8 @@ extern "C" bca_status bca_step_graph_create(const bca_step_graph_desc* d, bca_st
       st = step_attend_impl(d->q_t[l], d->k_t[l], d->v_t[l], d->o_t[l], d->cu_target,
                             d->slots + static_cast<size_t>(l) * d->n_req, d->n_req, d->heads,
                             d->head_dim, d->scale, d->workspace, d->workspace_bytes, q8,
-                            d->q8_scratch, d->q8_scratch_bytes, d->dev_status, cs);
+                            d->q8_scratch, d->q8_scratch_bytes, d->dev_status, cs, dq,
+                            d->dq_scratch, d->dq_scratch_bytes);
     if (cudaStreamEndCapture(cs, &graph) != cudaSuccess && st == BCA_OK) st = BCA_ERR_CUDA;
   }
   cudaStreamDestroy(cs);

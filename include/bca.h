@@ -377,8 +377,8 @@ bca_status bca_ulysses_unpack(const void* recv, void* x, int64_t rows_local, int
  * the outputs are bit-identical to the eager bca_step_attend calls on the same
  * contents.  Pointers, row counts, slot shapes and n_tokens are fixed when the
  * graph is created; another layout needs another graph.  bf16 and e4m3 caches are
- * captured alike, and with q8_scratch the e4m3-Q step (its Q quantisation
- * included) is recorded.  The graph object lives in host memory (the CUDA driver keeps
+ * captured alike; with q8_scratch the e4m3-Q step (its Q quantisation included),
+ * with dq_scratch the expand-once step (its expansion kernel included) is recorded.  The graph object lives in host memory (the CUDA driver keeps
  * its own copy of the recorded launches); the library allocates no device memory. */
 typedef struct bca_step_graph bca_step_graph; /* opaque */
 
@@ -398,10 +398,15 @@ typedef struct {
   void* q8_scratch;         /* nullable; non-NULL: the layers' bca_step_attend_q8 calls
                                are recorded instead (e4m3 slots), sharing this scratch */
   size_t q8_scratch_bytes;
+  void* dq_scratch;         /* nullable; non-NULL: the layers' bca_step_attend_dq calls
+                               are recorded instead (e4m3 slots), sharing this scratch
+                               (at least the largest layer's bca_step_dq_scratch_bytes);
+                               not together with q8_scratch */
+  size_t dq_scratch_bytes;
 } bca_step_graph_desc;
 
 /* Builds the graph on the current device.  Errors: BCA_ERR_INVALID_ARG for a NULL
- * desc/graph or a bad array; otherwise the first failing layer's bca_step_attend
+ * desc/graph, a bad array, or both q8_scratch and dq_scratch; otherwise the first failing layer's bca_step_attend
  * status (nothing is created then); BCA_ERR_CUDA if capture or instantiation fails. */
 bca_status bca_step_graph_create(const bca_step_graph_desc* desc, bca_step_graph** graph);
 
@@ -409,7 +414,7 @@ bca_status bca_step_graph_create(const bca_step_graph_desc* desc, bca_step_graph
 bca_status bca_step_graph_launch(const bca_step_graph* graph, void* stream);
 
 /* Kernel launches one replay performs (attention + chunk-merge kernels, and the Q
- * quantisation kernels of an e4m3-Q graph). */
+ * quantisation kernel of an e4m3-Q graph or the expansion kernel of a dq graph). */
 int32_t bca_step_graph_kernel_nodes(const bca_step_graph* graph);
 
 /* Releases the graph (NULL is ignored).  No replay may be pending on the GPU. */

@@ -165,3 +165,39 @@ def test_e4m3_q_graph_replay_equals_eager(cuda_device):
             torch.cuda.synchronize()
             assert torch.equal(x["o"], o)
     g.close()
+
+
+def test_dq_graph_replay_equals_eager(cuda_device):
+    """With a dq scratch the graph records each layer's bca_step_attend_dq (its
+    expansion kernel included): replays, also after new contents are written into the
+    same buffers, are bit-identical to the eager dq calls and to bca_step_attend."""
+    H = 4
+    cu, L = _layout(cuda_device, H, [256, 131, 300], [128, 0, 77], layers=2, mode="fp8",
+                    seed=90)
+    ws = bca.step_workspace(cuda_device)
+    scratch = torch.empty(max(bca.step_dq_scratch_bytes([s for s, *_ in x["slots"]])
+                              for x in L), dtype=torch.uint8, device=cuda_device)
+    status = torch.zeros(1, dtype=torch.int32, device=cuda_device)
+    g = bca.StepGraph([x["q"] for x in L], [x["k"] for x in L], [x["v"] for x in L],
+                      [x["o"] for x in L], cu, [[s for s, *_ in x["slots"]] for x in L], SCALE,
+                      workspace=ws, dev_status=status, dq_scratch=scratch)
+    assert g.kernel_nodes >= 2 * 2  # per layer: the expansion kernel + attention
+    for rnd in range(2):
+        if rnd:
+            for l, x in enumerate(L):
+                x["q"].copy_(randn_bf16(tuple(x["q"].shape), 9600 + l, cuda_device))
+        g.launch()
+        torch.cuda.synchronize()
+        assert int(status.item()) == 0
+        for x in L:
+            slots = [s for s, *_ in x["slots"]]
+            o, o2 = torch.empty_like(x["q"]), torch.empty_like(x["q"])
+            bca.step_attend_dq(x["q"], x["k"], x["v"], o, cu, slots, SCALE, workspace=ws)
+            bca.step_attend(x["q"], x["k"], x["v"], o2, cu, slots, SCALE, workspace=ws)
+            torch.cuda.synchronize()
+            assert torch.equal(x["o"], o) and torch.equal(o, o2)
+    g.close()
+    with pytest.raises(bca.BcaError):
+        bca.StepGraph([x["q"] for x in L], [x["k"] for x in L], [x["v"] for x in L],
+                      [x["o"] for x in L], cu, [[s for s, *_ in x["slots"]] for x in L], SCALE,
+                      q8_scratch=scratch, dq_scratch=scratch)
