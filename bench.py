@@ -461,40 +461,73 @@ def norm_rope_leg(device, peaks, rows: int, heads: int, calls: int = 20):
             "frac": gbs / peak, "l2": "4 input sets cycled (536 MB for the T2I shape)"}
 
 
-def store_leg(runner, peaks, reps: int = 5):
-    """bca_kv_store_batch of every request's prefix (layer 0's inputs) into fresh
-    slots of the workload's cache dtype, one kernel launch per store, timed with
-    events around each enqueue: GB/s on the algorithmic bytes (K and V prefix rows
-    read once, the cache written once, the scales)."""
+# GPU-busy lead before each timed enqueue: a spin kernel of this many cycles keeps
+# the device busy while the host marshals and enqueues the call, so the events
+# that follow bracket the call's device time, not the host's enqueue latency.
+LEAD_CYCLES = 2_000_000
+
+
+def device_time(fn, reps: int) -> float:
+    """Median over `reps` of the device time of fn(i), each enqueue bracketed by CUDA
+    events on the current stream behind a GPU-busy lead (fn(0) runs once untimed)."""
     import torch
-    bca, wl, H = runner.bca, runner.wl, runner.H
+    fn(0)
+    torch.cuda.synchronize()
+    ev = []
+    for i in range(reps):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda._sleep(LEAD_CYCLES)
+        e0.record()
+        fn(i)
+        e1.record()
+        ev.append((e0, e1))
+    torch.cuda.synchronize()
+    return statistics.median(a.elapsed_time(b) for a, b in ev)
+
+
+def store_time(bca, wl, kv, device, peaks, reps: int = 5):
+    """bca_kv_store_batch of every request's prefix rows (K, V in the [S, H, 128]
+    layout the prefill reads) into fresh slots of the workload's cache dtype: one
+    kernel launch per store, device time from events around each enqueue; GB/s on
+    the algorithmic bytes (K and V prefix rows read once, the cache written once,
+    the scales)."""
+    H = wl.heads
     dt = {"bf16": (2, 2), "fp8_v": (2, 1), "fp8": (1, 1)}[wl.kv_dtype]  # bytes of K, V codes
-    slots = [bca.KVSlot(max(r.prefix, 1), H, wl.kv_dtype, device=runner.device)
-             for r in wl.requests]
+    slots = [bca.KVSlot(max(r.prefix, 1), H, wl.kv_dtype, device=device) for r in wl.requests]
     alg = 0
     for r in wl.requests:
         n = r.prefix * H * 128
         alg += 2 * n * 2 + n * (dt[0] + dt[1]) + (8 * H if wl.kv_dtype != "bf16" else 0)
-
-    items = [(runner.pre[0][i][1], runner.pre[0][i][2], r.prefix, slots[i])
-             for i, r in enumerate(wl.requests)]
-    bca.kv_store_batch(items, 1)
-    torch.cuda.synchronize()
-    ev = []
-    for i in range(reps):  # one enqueue (one kernel launch) per store, events around it
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record()
-        bca.kv_store_batch(items, 2 + i)
-        e1.record()
-        ev.append((e0, e1))
-    torch.cuda.synchronize()
-    ms = sum(a.elapsed_time(b) for a, b in ev) / reps
+    items = [(k, v, r.prefix, slots[i]) for i, ((k, v), r) in enumerate(zip(kv, wl.requests))]
+    ms = device_time(lambda i: bca.kv_store_batch(items, 1 + i), reps)
     peak = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
     gbs = alg / (ms / 1e3) / 1e9
-    return {"bound": "hbm", "kv_cache": wl.kv_dtype, "prefix_rows": [r.prefix for r in wl.requests],
-            "ms_per_store": ms, "algorithmic_bytes": alg, "achieved": gbs, "peak": peak,
-            "unit": "GB/s", "frac": gbs / peak, "launches_per_store": 1,
-            "timing": "CUDA events around each bca_kv_store_batch enqueue"}
+    return {"bound": "hbm", "workload": wl.name, "kv_cache": wl.kv_dtype,
+            "prefix_rows": [r.prefix for r in wl.requests], "ms_per_store": ms,
+            "algorithmic_bytes": alg, "achieved": gbs, "peak": peak, "unit": "GB/s",
+            "frac": gbs / peak, "launches_per_store": 1,
+            "timing": "CUDA events around one bca_kv_store_batch enqueue (all requests, one "
+                      "kernel launch) behind a GPU-busy lead; median of 5"}
+
+
+def store_leg(runner, peaks):
+    """The prefix store of the step-batched serving workload (8 requests, e4m3 K and
+    V: two passes over 1.4 GB of prefix rows) and, nested, that of the timed
+    workload (layer 0's prefill inputs)."""
+    import torch
+    from block_causal_attention_dit_b200 import workloads as W
+    wl4 = W.workload(4)
+    kv = []
+    for i in range(len(wl4.requests)):
+        q, k, v = W.qkv(wl4, 0, 0, i, runner.device)
+        del q
+        kv.append((k, v))
+    out = store_time(runner.bca, wl4, kv, runner.device, peaks)
+    del kv
+    torch.cuda.empty_cache()
+    out["timed_workload"] = store_time(
+        runner.bca, runner.wl, [(x[1], x[2]) for x in runner.pre[0]], runner.device, peaks)
+    return out
 
 
 def qkv_leg(device, peaks, rows: int, heads: int, calls: int = 20):
@@ -569,8 +602,9 @@ def config_leg(index: int, device, peaks, reps: int = 3):
     (bca_prefill with the workspace, attention only), the prefix store of all
     requests (one bca_kv_store_batch launch) and one cached step of all requests
     (bca_step_attend; for an e4m3 cache bca_step_attend_dq, the in-kernel conversion
-    timed beside it), each timed with CUDA events around its enqueues.  Two cached-
-    step input sets alternate (larger than L2 together).  The 40-step projection is
+    timed beside it), each timed with CUDA events around its enqueues behind a
+    GPU-busy lead (device time only).  Two cached-step input sets alternate (larger
+    than L2 together).  The 40-step projection is
     32 layers x (prefill + store) + 32 x 39 cached steps from these timings."""
     import torch
     import block_causal_attention_dit_b200 as bca
@@ -621,19 +655,7 @@ def config_leg(index: int, device, peaks, reps: int = 3):
         q, k, v = sets[n % 2]
         bca.step_attend(q, k, v, o_step, cu, slots, wl.scale, workspace=ws, dev_status=status)
 
-    def time_it(fn, n):
-        fn(0)
-        torch.cuda.synchronize()
-        ev = []
-        for i in range(n):
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record()
-            fn(i)
-            e1.record()
-            ev.append((e0, e1))
-        torch.cuda.synchronize()
-        return statistics.median(a.elapsed_time(b) for a, b in ev)
-
+    time_it = device_time
     store()
     torch.cuda.synchronize()
     p_ms = time_it(lambda i: prefill(), reps)

@@ -296,78 +296,144 @@ struct StoreJob {
   bool quant;
 };
 
-// Clusters of the store kernel that can be resident at once on the current device
-// (cached per device; the GPCs' sizes decide how many 8-CTA clusters fit).
-int store_max_clusters() {
+// Store-kernel cluster shapes of the current device (cached per device): for each
+// size 4, 8, 16 (up to bca::kStoreMaxCluster; 16 needs the non-portable cluster
+// attribute), how many such clusters can be resident at once -- the GPCs' sizes
+// decide it.  0: that size cannot be launched.
+struct StoreShapes {
+  int clusters[3] = {0, 0, 0};  // sizes 4, 8, 16
+  bool ok = false;
+};
+const StoreShapes& store_shapes() {
   static std::mutex mu;
-  static std::vector<int> n;
+  static std::vector<StoreShapes> n;
+  static const StoreShapes none;
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return 1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return none;
   std::lock_guard<std::mutex> lk(mu);
-  if (n.size() <= static_cast<size_t>(dev)) n.resize(dev + 1, 0);
-  if (!n[dev]) {
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(static_cast<unsigned>(bca::kStoreCluster));
-    cfg.blockDim = dim3(bca::kStoreThreads);
-    cfg.dynamicSmemBytes = bca::kStoreRingBytes;
+  if (n.size() <= static_cast<size_t>(dev)) n.resize(dev + 1);
+  StoreShapes& sh = n[dev];
+  if (!sh.ok) {
     if (cudaFuncSetAttribute(bca::kv_store_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              bca::kStoreRingBytes) != cudaSuccess)
-      return 0;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = bca::kStoreCluster;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    int c = 0;
-    if (cudaOccupancyMaxActiveClusters(&c, bca::kv_store_kernel, &cfg) != cudaSuccess || c < 1)
-      c = std::max(1, sm_count() / bca::kStoreCluster);
-    n[dev] = c;
+      return none;
+    const bool big = bca::kStoreMaxCluster > 8 &&
+                     cudaFuncSetAttribute(bca::kv_store_kernel,
+                                          cudaFuncAttributeNonPortableClusterSizeAllowed,
+                                          1) == cudaSuccess;
+    for (int i = 0; i < 3; ++i) {
+      const int size = 4 << i;
+      if (size > bca::kStoreMaxCluster || (size > 8 && !big)) break;
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3(static_cast<unsigned>(size));
+      cfg.blockDim = dim3(bca::kStoreThreads);
+      cfg.dynamicSmemBytes = bca::kStoreRingBytes;
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = static_cast<unsigned>(size);
+      attr[0].val.clusterDim.y = 1;
+      attr[0].val.clusterDim.z = 1;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      int c = 0;
+      if (cudaOccupancyMaxActiveClusters(&c, bca::kv_store_kernel, &cfg) != cudaSuccess) c = 0;
+      sh.clusters[i] = c;
+    }
+    cudaGetLastError();  // a size the device refuses leaves no sticky error
+    if (sh.clusters[0] < 1) return none;
+    sh.ok = true;
   }
-  return n[dev];  // 0 only if the kernel attribute could not be set
+  return sh;
 }
 
-// One launch of bca::kv_store_kernel over every job: tensors with the most rows
-// first, clusters of bca::kStoreCluster CTAs, as many as are resident at once (so
-// that few columns are in flight and the encode pass re-reads them from L2).
+// Source map of one store job: {128 channels, heads, rows} bf16 bits with the
+// caller's row stride, box {128, 1, kStoreTileRows}, no swizzle.
+bool map_store_src(CUtensorMap* m, const StoreJob& j) {
+  const cuuint64_t dims[3] = {128, static_cast<cuuint64_t>(j.heads), static_cast<cuuint64_t>(j.rows)};
+  const cuuint64_t strides[2] = {256, static_cast<cuuint64_t>(j.row_stride) * 2};
+  const cuuint32_t box[3] = {128, 1, static_cast<cuuint32_t>(bca::kStoreTileRows)};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return g_encode(m, CU_TENSOR_MAP_DATA_TYPE_UINT16, 3, const_cast<void*>(j.src), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// One launch of bca::kv_store_kernel over every job, in clusters of 4 to
+// bca::kStoreMaxCluster CTAs, as many as are resident at once (so that few columns
+// are in flight and the encode pass re-reads them from L2).  bf16 heads are cut into
+// row pieces when there are too few of them to keep every cluster busy (about 8
+// columns per cluster); e4m3 heads stay whole.  Tensors with the longest columns go
+// first.
 bca_status launch_store(std::vector<StoreJob> jobs, int32_t* dev_status, cudaStream_t stream) {
   jobs.erase(std::remove_if(jobs.begin(), jobs.end(), [](const StoreJob& j) { return j.rows == 0; }),
              jobs.end());
   if (jobs.empty()) return BCA_OK;
   if (jobs.size() > static_cast<size_t>(bca::kMaxStoreTensors)) return BCA_ERR_INVALID_ARG;
-  std::stable_sort(jobs.begin(), jobs.end(),
-                   [](const StoreJob& a, const StoreJob& b) { return a.rows > b.rows; });
+  if (!get_encode()) return BCA_ERR_CUDA;
+  const StoreShapes& sh = store_shapes();
+  if (!sh.ok) return BCA_ERR_CUDA;
+  int64_t quant_cols = 0, copy_cols = 0;
+  for (const StoreJob& j : jobs) (j.quant ? quant_cols : copy_cols) += j.heads;
+  // e4m3 heads: the largest clusters that still cover three quarters of the SMs
+  // (fewest columns in flight for the encode pass's L2 re-reads); copies only: 4.
+  int csize = 4, max_clusters = sh.clusters[0];
+  if (quant_cols > 0) {
+    const int sms = sm_count();
+    for (int i = 2; i >= 1; --i)
+      if (sh.clusters[i] > 0 && 4 * (sh.clusters[i] << (2 + i)) >= 3 * sms) {
+        csize = 4 << i;
+        max_clusters = sh.clusters[i];
+        break;
+      }
+  }
+  std::vector<int> pieces(jobs.size(), 1);
+  const int64_t want = 8LL * max_clusters;
+  if (copy_cols > 0 && quant_cols + copy_cols < want) {
+    const int64_t per = (want - quant_cols + copy_cols - 1) / copy_cols;
+    for (size_t i = 0; i < jobs.size(); ++i) {
+      if (jobs[i].quant) continue;
+      // at least 2 tiles per CTA of the cluster in every piece
+      const int64_t tiles = (jobs[i].rows + bca::kStoreTileRows - 1) / bca::kStoreTileRows;
+      pieces[i] = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(per, tiles / (2 * csize))));
+    }
+  }
+  std::vector<size_t> order(jobs.size());
+  std::iota(order.begin(), order.end(), size_t{0});
+  std::stable_sort(order.begin(), order.end(), [&](size_t a, size_t b) {
+    return static_cast<int64_t>(jobs[a].rows) * pieces[b] > static_cast<int64_t>(jobs[b].rows) * pieces[a];
+  });
+  static_assert(sizeof(bca::StoreParams) <= 32764, "kernel parameter limit");
   bca::StoreParams p;
   std::memset(&p, 0, sizeof(p));
   int cols = 0;
-  for (size_t i = 0; i < jobs.size(); ++i) {
-    bca::StoreTensor& t = p.t[i];
-    t.src = static_cast<const uint16_t*>(jobs[i].src);
-    t.dst = jobs[i].dst;
-    t.scale = jobs[i].scale;
-    t.row_stride = jobs[i].row_stride;
-    t.head_stride = jobs[i].head_stride;
-    t.rows = jobs[i].rows;
-    t.heads = jobs[i].heads;
-    t.quant = jobs[i].quant ? 1 : 0;
+  for (size_t k = 0; k < order.size(); ++k) {
+    const StoreJob& j = jobs[order[k]];
+    if (!map_store_src(&p.map[k], j)) return BCA_ERR_INVALID_ARG;
+    bca::StoreTensor& t = p.t[k];
+    t.dst = j.dst;
+    t.scale = j.scale;
+    t.head_stride = j.head_stride;
+    t.rows = j.rows;
+    t.heads = j.heads;
+    t.quant = j.quant ? 1 : 0;
     t.col0 = cols;
-    cols += jobs[i].heads;
+    t.pieces = pieces[order[k]];
+    cols += j.heads * t.pieces;
   }
   p.n_tensors = static_cast<int32_t>(jobs.size());
   p.n_cols = cols;
   p.dev_status = dev_status;
-  const int max_clusters = store_max_clusters();
-  if (max_clusters < 1) return BCA_ERR_CUDA;
+  p.timeout_ns = g_timeout_ns.load();
   const int clusters = std::max(1, std::min(cols, max_clusters));
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(clusters * bca::kStoreCluster));
+  cfg.gridDim = dim3(static_cast<unsigned>(clusters * csize));
   cfg.blockDim = dim3(bca::kStoreThreads);
   cfg.dynamicSmemBytes = bca::kStoreRingBytes;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = bca::kStoreCluster;
+  attr[0].val.clusterDim.x = static_cast<unsigned>(csize);
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
