@@ -101,11 +101,11 @@ def prefill_split_launches(req, H, sms) -> int:
 # dram__bytes_write.sum) from one ncu capture of the T2I cached step, valid only for
 # the kernel sources it was taken from (their sha256 below); any later change
 # reports null instead.
-ATTN_TRAFFIC = {"bytes_per_launch": 109.28e6 + 15.53e6, "workload": 1,
+ATTN_TRAFFIC = {"bytes_per_launch": 109.36e6 + 15.57e6, "workload": 1,
                 "sources": {"block_causal_attention_dit_b200/csrc/attn_kernel.cuh":
-                            "f6b62b40fda38fb3fba0d8d3b9a2f17c70ca61acffdea9c8ba9f7b58d40c29e9",
+                            "ab3dde20c1de7ef509a371e62ec7c2a3ef4d5e1de907a89287a7912b455894ef",
                             "block_causal_attention_dit_b200/csrc/ptx.cuh":
-                            "cf462dedfbd63f8e2e730a546a5db830b04e5240296b7864a033c80e029dd256"}}
+                            "b7d801c899a2fe276d1041dddb3a3be5a03f2005b26d4375aa4e2a3b160f409b"}}
 
 
 def measured_traffic(workload: int):
