@@ -191,3 +191,56 @@ def test_non_finite_input_reports_status(cuda_device):
     torch.cuda.synchronize()
     assert int(status.item()) == 0
     assert torch.equal(s16.k_view(), k.permute(1, 0, 2))
+
+
+def test_batch_store_many_columns_per_cluster(cuda_device):
+    """512 e4m3 columns in one launch (8 requests x K and V x 32 heads): every
+    cluster of the store kernel takes a dozen or more columns in turn, so the
+    interleaving of one column's encode pass with the next column's absmax pass and
+    the rotation of the rank-exchange buffers over many columns both run.  Bytes and
+    scales equal the oracle's for every slot."""
+    prefixes = [611, 97, 420, 333, 800, 5, 256, 129]
+    items = []
+    for i, P in enumerate(prefixes):
+        k = randn_bf16((P, 32, 128), 700 + 2 * i, cuda_device) * (0.5 + i)
+        v = randn_bf16((P, 32, 128), 701 + 2 * i, cuda_device) * (3.0 / (1 + i))
+        slot = bca.KVSlot(P + 3, 32, "fp8")
+        _fill_sentinel(slot)
+        items.append((k, v, P, slot))
+    status = torch.zeros(1, dtype=torch.int32, device=cuda_device)
+    bca.kv_store_batch(items, epoch=4, dev_status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    for k, v, P, slot in items:
+        for x, codes, scales in ((k, slot.k_view(), slot.k_scale_view()),
+                                 (v, slot.v_view(), slot.v_scale_view())):
+            want_c, want_s = oracle.quantize_prefix(x.cpu(), P, P + 3)
+            assert np.array_equal(codes[:, :P].cpu().numpy(), want_c[:, :P]), P
+            assert np.array_equal(scales.cpu().numpy(), want_s), P
+            assert bool((codes[:, P:].contiguous().view(torch.uint8) == 0x5A).all()), P
+
+
+def test_batch_store_bf16_row_pieces(cuda_device):
+    """Few long bf16 heads are cut into row pieces across clusters (here 4 heads of
+    5000 rows, and the bf16 K of an "fp8_v" slot next to its e4m3 V): the copies are
+    exact, the e4m3 V bit-exact, and nothing past the prefix is written."""
+    specs = [(5000, 4, "bf16", 5004), (3001, 4, "fp8_v", 3001)]
+    items = []
+    for i, (P, H, mode, cap) in enumerate(specs):
+        k = randn_bf16((P, H, 128), 720 + 2 * i, cuda_device)
+        v = randn_bf16((P, H, 128), 721 + 2 * i, cuda_device) * 7.0
+        slot = bca.KVSlot(cap, H, mode)
+        _fill_sentinel(slot)
+        items.append((k, v, P, slot, mode, cap))
+    bca.kv_store_batch([it[:4] for it in items], epoch=2)
+    torch.cuda.synchronize()
+    for k, v, P, slot, mode, cap in items:
+        assert torch.equal(slot.k_view()[:, :P], k.permute(1, 0, 2)), mode
+        if mode == "bf16":
+            assert torch.equal(slot.v_view()[:, :P], v.permute(1, 0, 2))
+        else:
+            want_c, want_s = oracle.quantize_prefix(v.cpu(), P, cap)
+            assert np.array_equal(slot.v_view()[:, :P].cpu().numpy(), want_c[:, :P])
+            assert np.array_equal(slot.v_scale_view().cpu().numpy(), want_s)
+        for codes in (slot.k_view(), slot.v_view()):
+            assert bool((codes[:, P:].contiguous().view(torch.uint8) == 0x5A).all()), mode
