@@ -493,11 +493,14 @@ def store_time(bca, wl, kv, device, peaks, reps: int = 5):
     the scales)."""
     H = wl.heads
     dt = {"bf16": (2, 2), "fp8_v": (2, 1), "fp8": (1, 1)}[wl.kv_dtype]  # bytes of K, V codes
+    n_quant = {"bf16": 0, "fp8_v": 1, "fp8": 2}[wl.kv_dtype]  # tensors read twice
     slots = [bca.KVSlot(max(r.prefix, 1), H, wl.kv_dtype, device=device) for r in wl.requests]
-    alg = 0
+    alg = moved = 0
     for r in wl.requests:
         n = r.prefix * H * 128
-        alg += 2 * n * 2 + n * (dt[0] + dt[1]) + (8 * H if wl.kv_dtype != "bf16" else 0)
+        a = 2 * n * 2 + n * (dt[0] + dt[1]) + (8 * H if wl.kv_dtype != "bf16" else 0)
+        alg += a
+        moved += a + n_quant * n * 2  # the encode pass reads an e4m3 tensor's rows again
     items = [(k, v, r.prefix, slots[i]) for i, ((k, v), r) in enumerate(zip(kv, wl.requests))]
     ms = device_time(lambda i: bca.kv_store_batch(items, 1 + i), reps)
     peak = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
@@ -505,7 +508,8 @@ def store_time(bca, wl, kv, device, peaks, reps: int = 5):
     return {"bound": "hbm", "workload": wl.name, "kv_cache": wl.kv_dtype,
             "prefix_rows": [r.prefix for r in wl.requests], "ms_per_store": ms,
             "algorithmic_bytes": alg, "achieved": gbs, "peak": peak, "unit": "GB/s",
-            "frac": gbs / peak, "launches_per_store": 1,
+            "frac": gbs / peak, "moved_bytes": moved,
+            "achieved_on_moved_bytes": moved / (ms / 1e3) / 1e9, "launches_per_store": 1,
             "timing": "CUDA events around one bca_kv_store_batch enqueue (all requests, one "
                       "kernel launch) behind a GPU-busy lead; median of 5"}
 
