@@ -42,7 +42,7 @@ __all__ = [
     "step_attend_dq", "step_dq_scratch", "step_dq_scratch_bytes",
     "StepGraph", "qk_norm_rope", "qkv_project", "ulysses_pack", "ulysses_unpack",
     "slot_bytes", "set_wait_timeout_ns",
-    "selftest_wait_timeout", "selftest_exp2", "selftest_e4m3_division", "status_string",
+    "selftest_wait_timeout", "selftest_e4m3_division", "status_string",
     "version", "LIB_PATH",
 ]
 
@@ -154,8 +154,6 @@ def lib():
     L.bca_selftest_wait_timeout.argtypes = [P, u64, P]
     L.bca_selftest_e4m3_division.restype = ctypes.c_int
     L.bca_selftest_e4m3_division.argtypes = [P, P]
-    L.bca_selftest_exp2.restype = ctypes.c_int
-    L.bca_selftest_exp2.argtypes = [P, P, P, i32, P]
     L.bca_debug_set_trace.restype = ctypes.c_int
     L.bca_debug_set_trace.argtypes = [P, i32]
     L.bca_qk_norm_rope.restype = ctypes.c_int
@@ -689,11 +687,3 @@ def selftest_e4m3_division(device="cuda", stream=None):
            "bca_selftest_e4m3_division")
     return int(n.item())
 
-
-def selftest_exp2(x, stream=None):
-    """(software 2^x, hardware ex2.approx) of a float32 CUDA tensor x."""
-    import torch
-    yp, ym = torch.empty_like(x), torch.empty_like(x)
-    _check(lib().bca_selftest_exp2(_ptr(x), _ptr(yp), _ptr(ym), x.numel(),
-                                   _stream(stream, x.device)), "bca_selftest_exp2")
-    return yp, ym

@@ -920,39 +920,10 @@ extern "C" bca_status bca_selftest_wait_timeout(int32_t* dev_status, uint64_t ti
   return cudaGetLastError() == cudaSuccess ? BCA_OK : BCA_ERR_CUDA;
 }
 
-// ---------------------------------------------------------------------------
-// Software exp2 self-check: the kernel's FMA-pipe 2^x next to the MUFU ex2.
-// ---------------------------------------------------------------------------
-namespace {
-__global__ void selftest_exp2_kernel(const float* x, float* y_poly, float* y_mufu, int n) {
-  const int i = 2 * (blockIdx.x * blockDim.x + threadIdx.x);
-  if (i >= n) return;
-  const float a = x[i], b = (i + 1 < n) ? x[i + 1] : 0.0f;
-  float p0, p1;
-  bca::f2_unpack(bca::exp2_poly2(bca::f2_pack(a, b)), p0, p1);
-  y_poly[i] = p0;
-  y_mufu[i] = bca::ex2_approx(a);
-  if (i + 1 < n) {
-    y_poly[i + 1] = p1;
-    y_mufu[i + 1] = bca::ex2_approx(b);
-  }
-}
-}  // namespace
-
 extern "C" bca_status bca_selftest_e4m3_division(unsigned long long* mismatches, void* stream) {
   if (!mismatches) return BCA_ERR_INVALID_ARG;
   bca::e4m3_division_selftest_kernel<<<0x7F7F, 256, 0, static_cast<cudaStream_t>(stream)>>>(
       mismatches);
-  return cudaGetLastError() == cudaSuccess ? BCA_OK : BCA_ERR_CUDA;
-}
-
-extern "C" bca_status bca_selftest_exp2(const float* x, float* y_poly, float* y_mufu, int32_t n,
-                                        void* stream) {
-  if (n < 0 || (n > 0 && (!x || !y_poly || !y_mufu))) return BCA_ERR_INVALID_ARG;
-  if (n == 0) return BCA_OK;
-  const int threads = 256, pairs = (n + 1) / 2;
-  selftest_exp2_kernel<<<(pairs + threads - 1) / threads, threads, 0,
-                         static_cast<cudaStream_t>(stream)>>>(x, y_poly, y_mufu, n);
   return cudaGetLastError() == cudaSuccess ? BCA_OK : BCA_ERR_CUDA;
 }
 

@@ -350,30 +350,4 @@ __device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
   return r;
 }
 
-// 2^x for two lanes on the FMA pipe (keeps the MUFU free for the other lanes):
-//  * clamp x >= -127 (2^-127 and below, -inf included, come out as exactly 0);
-//  * range reduction: t = x + 1.5*2^23 rounds x to the integer n held in the low
-//    mantissa bits of t; f = x - n lies in [-1/2, 1/2];
-//  * 2^f by a degree-3 polynomial whose coefficients were fitted here by a Remez
-//    exchange for minimax relative error on [-1/2, 1/2] (max 7.5e-5);
-//  * 2^n built directly as float bits: (bits(t) << 23) + bits(1.0), which is +0.0
-//    for n = -127 (the low 9 bits of bits(1.5*2^23) are zero, so they shift out).
-// Valid for x <= 127 (callers pass x <= 8).
-__device__ __forceinline__ uint64_t exp2_poly2(uint64_t x) {
-  float x0, x1;
-  f2_unpack(x, x0, x1);
-  x = f2_pack(fmaxf(x0, -127.0f), fmaxf(x1, -127.0f));
-  const uint64_t kMagic = f2_pack(12582912.0f, 12582912.0f);
-  const uint64_t t = f2_add(x, kMagic);
-  const uint64_t f = f2_sub(x, f2_sub(t, kMagic));
-  uint64_t q = f2_fma(f, f2_pack(0.0551716685f, 0.0551716685f), f2_pack(0.242611125f, 0.242611125f));
-  q = f2_fma(f, q, f2_pack(0.693260968f, 0.693260968f));
-  q = f2_fma(f, q, f2_pack(0.999928057f, 0.999928057f));
-  float t0, t1;
-  f2_unpack(t, t0, t1);
-  const uint32_t s0 = (__float_as_uint(t0) << 23) + 0x3F800000u;
-  const uint32_t s1 = (__float_as_uint(t1) << 23) + 0x3F800000u;
-  return f2_mul(q, f2_pack(__uint_as_float(s0), __uint_as_float(s1)));
-}
-
 }  // namespace bca

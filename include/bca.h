@@ -433,14 +433,6 @@ void bca_set_wait_timeout_ns(uint64_t timeout_ns);
  * device timeout without hanging or faulting the GPU. */
 bca_status bca_selftest_wait_timeout(int32_t* dev_status, uint64_t timeout_ns, void* stream);
 
-/* Self-check of the software 2^x that the attention kernel can evaluate on the FMA
- * pipe for part of each softmax row (builds with BCA_POLY_PAIRS > 0; the default
- * build uses MUFU ex2 only): range reduction to [-1/2, 1/2] plus a degree-3
- * minimax polynomial; inputs <= -127 give exactly 0.  Writes it to y_poly and the
- * hardware ex2.approx to y_mufu for the n device floats x[].  Diagnostic only. */
-bca_status bca_selftest_exp2(const float* x, float* y_poly, float* y_mufu, int32_t n,
-                             void* stream);
-
 /* Self-check of the e4m3 encoder's division: for every positive finite bf16 amax
  * and every bf16 x with |x| <= amax, counts (atomically adds to *mismatches, a
  * device uint64 the caller zeroes) the pairs whose e4m3 code from the encoder's
