@@ -101,11 +101,11 @@ def prefill_split_launches(req, H, sms) -> int:
 # dram__bytes_write.sum) from one ncu capture of the T2I cached step, valid only for
 # the kernel sources it was taken from (their sha256 below); any later change
 # reports null instead.
-ATTN_TRAFFIC = {"bytes_per_launch": 109.36e6 + 15.57e6, "workload": 1,
+ATTN_TRAFFIC = {"bytes_per_launch": 109.36e6 + 15.03e6, "workload": 1,
                 "sources": {"block_causal_attention_dit_b200/csrc/attn_kernel.cuh":
                             "ab3dde20c1de7ef509a371e62ec7c2a3ef4d5e1de907a89287a7912b455894ef",
                             "block_causal_attention_dit_b200/csrc/ptx.cuh":
-                            "b7d801c899a2fe276d1041dddb3a3be5a03f2005b26d4375aa4e2a3b160f409b"}}
+                            "ff28b151b435b8539e9ec163c92ee0881e60791f27d19e3ff29424d4f68e65dd"}}
 
 
 def measured_traffic(workload: int):
