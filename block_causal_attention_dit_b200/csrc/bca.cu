@@ -296,54 +296,37 @@ struct StoreJob {
   bool quant;
 };
 
-// Store-kernel cluster shapes of the current device (cached per device): for each
-// size 4, 8, 16 (up to bca::kStoreMaxCluster; 16 needs the non-portable cluster
-// attribute), how many such clusters can be resident at once -- the GPCs' sizes
-// decide it.  0: that size cannot be launched.
-struct StoreShapes {
-  int clusters[3] = {0, 0, 0};  // sizes 4, 8, 16
-  bool ok = false;
-};
-const StoreShapes& store_shapes() {
+// Clusters of the store kernel that can be resident at once on the current device
+// (cached per device; the GPCs' sizes decide how many clusters of bca::kStoreCluster
+// CTAs fit).  0: the kernel attribute could not be set.
+int store_max_clusters() {
   static std::mutex mu;
-  static std::vector<StoreShapes> n;
-  static const StoreShapes none;
+  static std::vector<int> n;
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return none;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
   std::lock_guard<std::mutex> lk(mu);
-  if (n.size() <= static_cast<size_t>(dev)) n.resize(dev + 1);
-  StoreShapes& sh = n[dev];
-  if (!sh.ok) {
+  if (n.size() <= static_cast<size_t>(dev)) n.resize(dev + 1, 0);
+  if (!n[dev]) {
     if (cudaFuncSetAttribute(bca::kv_store_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              bca::kStoreRingBytes) != cudaSuccess)
-      return none;
-    const bool big = bca::kStoreMaxCluster > 8 &&
-                     cudaFuncSetAttribute(bca::kv_store_kernel,
-                                          cudaFuncAttributeNonPortableClusterSizeAllowed,
-                                          1) == cudaSuccess;
-    for (int i = 0; i < 3; ++i) {
-      const int size = 4 << i;
-      if (size > bca::kStoreMaxCluster || (size > 8 && !big)) break;
-      cudaLaunchConfig_t cfg = {};
-      cfg.gridDim = dim3(static_cast<unsigned>(size));
-      cfg.blockDim = dim3(bca::kStoreThreads);
-      cfg.dynamicSmemBytes = bca::kStoreRingBytes;
-      cudaLaunchAttribute attr[1];
-      attr[0].id = cudaLaunchAttributeClusterDimension;
-      attr[0].val.clusterDim.x = static_cast<unsigned>(size);
-      attr[0].val.clusterDim.y = 1;
-      attr[0].val.clusterDim.z = 1;
-      cfg.attrs = attr;
-      cfg.numAttrs = 1;
-      int c = 0;
-      if (cudaOccupancyMaxActiveClusters(&c, bca::kv_store_kernel, &cfg) != cudaSuccess) c = 0;
-      sh.clusters[i] = c;
-    }
-    cudaGetLastError();  // a size the device refuses leaves no sticky error
-    if (sh.clusters[0] < 1) return none;
-    sh.ok = true;
+      return 0;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(bca::kStoreCluster));
+    cfg.blockDim = dim3(bca::kStoreThreads);
+    cfg.dynamicSmemBytes = bca::kStoreRingBytes;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = bca::kStoreCluster;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int c = 0;
+    if (cudaOccupancyMaxActiveClusters(&c, bca::kv_store_kernel, &cfg) != cudaSuccess || c < 1)
+      c = std::max(1, sm_count() / bca::kStoreCluster);
+    n[dev] = c;
   }
-  return sh;
+  return n[dev];
 }
 
 // Source map of one store job: {128 channels, heads, rows} bf16 bits with the
@@ -359,34 +342,22 @@ bool map_store_src(CUtensorMap* m, const StoreJob& j) {
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// One launch of bca::kv_store_kernel over every job, in clusters of 4 to
-// bca::kStoreMaxCluster CTAs, as many as are resident at once (so that few columns
-// are in flight and the encode pass re-reads them from L2).  bf16 heads are cut into
-// row pieces when there are too few of them to keep every cluster busy (about 8
-// columns per cluster); e4m3 heads stay whole.  Tensors with the longest columns go
-// first.
+// One launch of bca::kv_store_kernel over every job, in clusters of
+// bca::kStoreCluster CTAs, as many as are resident at once (so that few columns are
+// in flight and the encode pass re-reads them from L2).  bf16 heads are cut into row
+// pieces when there are too few of them to keep every cluster busy (about 8 columns
+// per cluster); e4m3 heads stay whole.  Tensors with the longest columns go first.
 bca_status launch_store(std::vector<StoreJob> jobs, int32_t* dev_status, cudaStream_t stream) {
   jobs.erase(std::remove_if(jobs.begin(), jobs.end(), [](const StoreJob& j) { return j.rows == 0; }),
              jobs.end());
   if (jobs.empty()) return BCA_OK;
   if (jobs.size() > static_cast<size_t>(bca::kMaxStoreTensors)) return BCA_ERR_INVALID_ARG;
   if (!get_encode()) return BCA_ERR_CUDA;
-  const StoreShapes& sh = store_shapes();
-  if (!sh.ok) return BCA_ERR_CUDA;
+  const int max_clusters = store_max_clusters();
+  if (max_clusters < 1) return BCA_ERR_CUDA;
+  constexpr int csize = bca::kStoreCluster;
   int64_t quant_cols = 0, copy_cols = 0;
   for (const StoreJob& j : jobs) (j.quant ? quant_cols : copy_cols) += j.heads;
-  // e4m3 heads: the largest clusters that still cover three quarters of the SMs
-  // (fewest columns in flight for the encode pass's L2 re-reads); copies only: 4.
-  int csize = 4, max_clusters = sh.clusters[0];
-  if (quant_cols > 0) {
-    const int sms = sm_count();
-    for (int i = 2; i >= 1; --i)
-      if (sh.clusters[i] > 0 && 4 * (sh.clusters[i] << (2 + i)) >= 3 * sms) {
-        csize = 4 << i;
-        max_clusters = sh.clusters[i];
-        break;
-      }
-  }
   std::vector<int> pieces(jobs.size(), 1);
   const int64_t want = 8LL * max_clusters;
   if (copy_cols > 0 && quant_cols + copy_cols < want) {
@@ -433,7 +404,7 @@ bca_status launch_store(std::vector<StoreJob> jobs, int32_t* dev_status, cudaStr
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = static_cast<unsigned>(csize);
+  attr[0].val.clusterDim.x = csize;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;

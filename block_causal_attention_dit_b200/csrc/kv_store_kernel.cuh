@@ -91,10 +91,10 @@ __device__ __forceinline__ uint2 encode_chunk(const uint4 v, float s, uint64_t y
 // The store kernel.  A launch stores a list of tensors; tensor i has heads_i x
 // pieces_i columns (one per head and row piece: e4m3 tensors are never split,
 // pieces_i = 1, since a head's scale needs all its rows), numbered from col0_i.  A
-// cluster of CTAs (its size chosen by the host, at most kStoreMaxCluster) takes
+// cluster takes
 // whole columns (cluster c: columns c, c + #clusters, ...; the host lists the
 // tensors with the longest columns first and launches only as many clusters as are
-// resident at once), and its CTAs split a column's tiles evenly.
+// resident at once), and its kStoreCluster CTAs split a column's tiles evenly.
 //
 // Warp specialisation (one CTA per SM):
 //  * producer warp (one lane) schedules the CTA's work as a sequence of items, each
@@ -108,15 +108,15 @@ __device__ __forceinline__ uint2 encode_chunk(const uint4 v, float s, uint64_t y
 //    overlaps the instruction-bound encode pass of the previous one, and the rank
 //    exchange has those lead tiles' time to complete.  The slot's item descriptor
 //    is written before the slot's barrier is armed.
-//    Measured on the 8-request serving store (e4m3 K and V, 2.13 GB): clusters of
-//    4 with a lag of 1 and interleaving, 4 chunks per thread, 0.588 ms; clusters of
-//    8 0.647 ms and of 16 0.75 ms (fewer columns in flight, so more of the encode
-//    pass hits L2, but fewer SMs and more per-column exchanges per CTA); the encode
-//    pass run after the lead instead of interleaved 0.652 ms; 2 chunks per thread
+//    Measured on the 8-request serving store (e4m3 K and V, 2.13 GB): this shape
+//    0.588 ms; clusters of 8 0.647 ms and of 16 0.75 ms (fewer columns in flight, so
+//    more of the encode pass hits L2, but fewer SMs and more per-column exchanges
+//    per CTA); each column's encode pass a whole step later 0.632 ms; the encode
+//    pass after the lead instead of interleaved 0.652 ms; 2 chunks per thread
 //    0.780 ms.
 //  * kStoreConsumerWarps consumer warps read every item (a tile: kStoreChunks
-//    16-byte chunks per thread, kStoreStepRows rows apart, independent of one another) and each
-//    warp releases the slot on its own:
+//    16-byte chunks per thread, kStoreStepRows rows apart, independent of one
+//    another) and each warp releases the slot on its own:
 //      copy tile    : the chunk goes straight to the cache row (streaming store);
 //      absmax tile  : packed 16-bit max of the magnitudes;
 //      absmax done  : every warp leaves its maximum in shared memory and arrives
@@ -154,37 +154,19 @@ struct StoreTensor {
   int32_t pieces;       // row pieces per head (1 for e4m3)
 };
 
-#ifndef BCA_STORE_MAX_CLUSTER
-#define BCA_STORE_MAX_CLUSTER 4
-#endif
-#ifndef BCA_STORE_CHUNKS
-#define BCA_STORE_CHUNKS 4
-#endif
-#ifndef BCA_STORE_CONSUMER_WARPS
-#define BCA_STORE_CONSUMER_WARPS 16
-#endif
 constexpr int kMaxStoreTensors = 2 * BCA_MAX_BATCH;
-constexpr int kStoreConsumerWarps = BCA_STORE_CONSUMER_WARPS;
+constexpr int kStoreConsumerWarps = 16;
 constexpr int kStoreConsumers = 32 * kStoreConsumerWarps;
 constexpr int kStoreThreads = kStoreConsumers + 32;  // + the producer warp
-constexpr int kStoreMaxCluster = BCA_STORE_MAX_CLUSTER;
-constexpr int kStoreChunks = BCA_STORE_CHUNKS;  // 16-byte chunks per consumer thread per tile
+constexpr int kStoreCluster = 4;
+constexpr int kStoreChunks = 4;  // 16-byte chunks per consumer thread per tile
 constexpr int kStoreStepRows = kStoreConsumers / 16;  // rows covered by one chunk of every thread
 constexpr int kStoreTileRows = kStoreStepRows * kStoreChunks;
 constexpr int kStoreTileBytes = kStoreTileRows * 256;
 constexpr int kStoreRingBytes = 128 * 1024;
 constexpr int kStoreStages = kStoreRingBytes / kStoreTileBytes;
 constexpr int kStoreLead = kStoreStages / 2;  // first-pass tiles ahead of an encode pass
-#ifndef BCA_STORE_LAG
-#define BCA_STORE_LAG 1
-#endif
-constexpr int kStoreLag = BCA_STORE_LAG;      // steps between a column's two passes (1 or 2)
-#ifndef BCA_STORE_INTERLEAVE
-#define BCA_STORE_INTERLEAVE 1
-#endif
-constexpr bool kStoreInterleave = BCA_STORE_INTERLEAVE != 0;  // 0: encode tiles first
 constexpr int kStoreXBufs = 4;
-static_assert(kStoreLag == 1 || kStoreLag == 2, "exchange buffers cover a lag of 1 or 2");
 static_assert(kStoreConsumers * kStoreChunks * 16 == kStoreTileBytes, "tile split");
 static_assert(kStoreConsumerWarps <= 32, "one warp maximum per lane in the reduction");
 static_assert(kStoreTileRows <= 256, "TMA box rows");
@@ -326,51 +308,43 @@ __device__ __forceinline__ void store_abort(volatile int* abort, int32_t* dev_st
   if (dev_status) atomicExch(dev_status, static_cast<int32_t>(BCA_ERR_DEVICE_TIMEOUT));
 }
 
-// The producer's schedule over the CTA's columns (see above).  Steps: in step i the
-// first-pass tiles of column i are interleaved with the encode tiles of the e4m3
-// column whose first pass ended kStoreLag steps earlier (kStoreLag 2: the rank
-// exchange of a column has a whole step to complete before its encode pass
-// begins).  next() returns the next item; `load` says whether it is a tile to fetch.
+// The producer's schedule over the CTA's columns (see above): step i interleaves the
+// first-pass tiles of column i with the encode tiles of column i - 1 (if e4m3).
+// next() returns the next item; `load` says whether it is a tile to fetch.
 struct StoreSchedule {
   const StoreParams& p;
   uint32_t crank, csize;
   int col, col_step, ti_scan = 0;
-  StoreCol cur;               // first pass in progress
-  StoreCol wait[kStoreLag];   // wait[0]: being encoded; wait[j]: j steps from encoding
+  StoreCol cur;   // first pass in progress
+  StoreCol prev;  // e4m3 column being encoded
   int a_done = 0, b_done = 0;
   bool abs_done_sent = false, enc_begun = false, toggle = false;
 
   __device__ StoreSchedule(const StoreParams& p_, uint32_t r, uint32_t n, int c0, int step)
       : p(p_), crank(r), csize(n), col(c0), col_step(step) {
-    for (int j = 0; j < kStoreLag; ++j) wait[j].valid = false;
+    prev.valid = false;
     cur = store_col(p, col, ti_scan, crank, csize);
     col += col_step;
   }
   __device__ StoreItem next(bool& load) {
     load = false;
     for (;;) {
-      const StoreCol& prev = wait[0];
       const int a_total = cur.valid ? cur.t1 - cur.t0 : 0;
       const int b_total = prev.valid ? prev.t1 - prev.t0 : 0;
       const bool a_left = cur.valid && a_done < a_total;
-      // With a lag of 2 the encode pass opens the step (its exchange has had the
-      // whole previous step); with a lag of 1 it follows kStoreLead first-pass tiles.
-      // Either way a column's "absmax done" follows the "encode begins" of the e4m3
-      // column two before it, which the kStoreXBufs = 4 exchange buffers rely on.
-      if (kStoreLag > 1 && prev.valid && !enc_begun) {
-        enc_begun = true;
-        return StoreItem{kItemEncBegin, static_cast<uint32_t>(prev.ti), prev.h, 0};
-      }
       if (a_left && a_done < kStoreLead) return first_pass_tile(load);
       if (cur.valid && !a_left && cur.quant && !abs_done_sent) {
         abs_done_sent = true;
         return StoreItem{kItemAbsDone, static_cast<uint32_t>(cur.ti), cur.h, 0};
       }
+      // After the lead: "encode begins" of prev, so a column's "absmax done" always
+      // follows the "encode begins" of the e4m3 column two before it, which the
+      // kStoreXBufs = 4 exchange buffers rely on.
       if (prev.valid && !enc_begun) {
         enc_begun = true;
         return StoreItem{kItemEncBegin, static_cast<uint32_t>(prev.ti), prev.h, 0};
       }
-      if (prev.valid && b_done < b_total && (!kStoreInterleave || toggle || !a_left)) {
+      if (prev.valid && b_done < b_total && (toggle || !a_left)) {
         toggle = false;
         load = true;
         const int tile = prev.t1 - 1 - b_done++;
@@ -381,12 +355,9 @@ struct StoreSchedule {
         return first_pass_tile(load);
       }
       // The step is complete: cur's first pass and prev's encode pass are done.
-      bool pending = cur.valid;
-      for (int j = 1; j < kStoreLag; ++j) pending = pending || wait[j].valid;
-      if (!pending) return StoreItem{kItemEnd, 0, 0, 0};
-      for (int j = 0; j + 1 < kStoreLag; ++j) wait[j] = wait[j + 1];
-      wait[kStoreLag - 1] = cur;
-      wait[kStoreLag - 1].valid = cur.valid && cur.quant;
+      if (!cur.valid) return StoreItem{kItemEnd, 0, 0, 0};
+      prev = cur;
+      prev.valid = cur.quant;
       b_done = 0;
       enc_begun = false;
       cur = store_col(p, col, ti_scan, crank, csize);
@@ -409,7 +380,7 @@ __global__ void __launch_bounds__(kStoreThreads, 1)
   __shared__ __align__(8) uint64_t s_full[kStoreStages], s_empty[kStoreStages];
   __shared__ __align__(8) uint64_t s_xbar[kStoreXBufs], s_rbar[kStoreXBufs];
   __shared__ StoreSlot s_item[kStoreStages];
-  __shared__ uint32_t s_part[kStoreXBufs][kStoreMaxCluster];     // CTA maxima by rank
+  __shared__ uint32_t s_part[kStoreXBufs][kStoreCluster];        // CTA maxima by rank
   __shared__ uint32_t s_red[kStoreXBufs][kStoreConsumerWarps];  // warp maxima
   __shared__ int s_abort;
   const uint32_t ring = smem_u32(store_ring);
