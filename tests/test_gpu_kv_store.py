@@ -244,3 +244,55 @@ def test_batch_store_bf16_row_pieces(cuda_device):
             assert np.array_equal(slot.v_scale_view().cpu().numpy(), want_s)
         for codes in (slot.k_view(), slot.v_view()):
             assert bool((codes[:, P:].contiguous().view(torch.uint8) == 0x5A).all()), mode
+
+
+def test_serving_store_full_size_sampled_heads(cuda_device):
+    """The 8-request serving store at its full size (e4m3 K and V, prefixes 996 ..
+    17075 rows, 32 heads: 512 columns in one launch, the call the bench times):
+    sixteen sampled (request, tensor, head) columns are bit-exact against the oracle
+    quantising that head's rows (codes and scale), and rows past each prefix are
+    untouched."""
+    from block_causal_attention_dit_b200 import workloads as W
+    wl = W.workload(4)
+    items, srcs = [], []
+    for i, r in enumerate(wl.requests):
+        _, k, v = W.qkv(wl, 0, 0, i, cuda_device)
+        slot = bca.KVSlot(r.prefix + 5, wl.heads, "fp8")
+        _fill_sentinel(slot)
+        items.append((k, v, r.prefix, slot))
+    status = torch.zeros(1, dtype=torch.int32, device=cuda_device)
+    bca.kv_store_batch(items, epoch=5, dev_status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    rng = np.random.default_rng(44)
+    for _ in range(16):
+        i = int(rng.integers(len(items)))
+        kv = int(rng.integers(2))
+        h = int(rng.integers(wl.heads))
+        k, v, P, slot = items[i]
+        x = (k, v)[kv][:P, h:h + 1, :].cpu()
+        want_c, want_s = oracle.quantize_prefix(x, P, P + 5)
+        codes = (slot.k_view(), slot.v_view())[kv][h:h + 1]
+        scales = (slot.k_scale_view(), slot.v_scale_view())[kv][h:h + 1]
+        assert np.array_equal(codes[:, :P].cpu().numpy(), want_c[:, :P]), (i, kv, h)
+        assert np.array_equal(scales.cpu().numpy(), want_s), (i, kv, h)
+        assert bool((codes[:, P:].contiguous().view(torch.uint8) == 0x5A).all()), (i, kv, h)
+
+
+def test_edit_store_full_size_bf16(cuda_device):
+    """The 4-ref edit's bf16 prefix store at full size (16864 rows x 32 heads, K and
+    V: 64 long heads cut into row pieces across the clusters) is an exact copy, and
+    nothing past the prefix is written."""
+    from block_causal_attention_dit_b200 import workloads as W
+    wl = W.workload(2)
+    r = wl.requests[0]
+    _, k, v = W.qkv(wl, 0, 0, 0, cuda_device)
+    slot = bca.KVSlot(r.prefix + 7, wl.heads, "bf16")
+    _fill_sentinel(slot)
+    bca.kv_store_batch([(k, v, r.prefix, slot)], epoch=3)
+    torch.cuda.synchronize()
+    P = r.prefix
+    assert torch.equal(slot.k_view()[:, :P], k[:P].permute(1, 0, 2))
+    assert torch.equal(slot.v_view()[:, :P], v[:P].permute(1, 0, 2))
+    for codes in (slot.k_view(), slot.v_view()):
+        assert bool((codes[:, P:].contiguous().view(torch.uint8) == 0x5A).all())
