@@ -120,8 +120,9 @@ bca_status bca_kv_slot_init(bca_kv_slot* slot, void* base, int32_t cap_tokens,
  * For an e4m3 tensor: amax = max |x| over the n_prefix rows of each head,
  * scale = fp32(amax)/448 (1 when amax == 0), code = e4m3 RNE-satfinite of the
  * correctly rounded fp32 quotient x/scale.  Rows [n_prefix, cap) are not written.
- * One kernel launch (HBM-bound; the absmax and encode passes of a head run back to
- * back on the same CTAs, so the second reads its rows from L2).
+ * One kernel launch (HBM-bound; a head's encode pass re-reads its rows on the same
+ * CTAs right after its absmax pass, interleaved with the next head's absmax pass,
+ * so that rows still in L2 come from there).
  * Host side effects (at enqueue): slot->n_tokens = n_prefix, slot->epoch = epoch.
  * dev_status: nullable device int32, see the conventions above (a non-finite value
  * in an e4m3 tensor: BCA_ERR_NONFINITE). */
